@@ -1,0 +1,7 @@
+"""fp64 CPU oracle for AXELRAM decode attention (test infrastructure only).
+
+Only tests/, __graft_entry__.smoke() and bench.py's CPU baseline / reference arm may import this package.  The
+product path (kv_cache_quantized_b200) never imports it, and the two share no code.
+"""
+from .axelram import *  # noqa: F401,F403
+from .axelram import __all__  # noqa: F401
