@@ -1,0 +1,379 @@
+"""Benchmark of the AXELRAM decode hot path on B200 (one JSON line on stdout, rank 0).
+
+Step = one decode step over a resident quantized KV cache: the new token's key and value of every (batch row, KV
+head) go through the write path (rotate + quantize + pack, appended at position T-1), then decode attention runs
+over all T cached tokens (LUT scores, split-T online softmax, value product, split merge, one inverse transform for
+quantized values).  The codebook is design-time (computed once at setup); sign selection is offline
+(``--workload select`` times it separately).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl axr|reference]
+
+Multi-GPU: every rank runs an independent replica of the workload (decode units are independent; no collective on
+the data path), value = units of all ranks / max over ranks of the device time ("scaling": "weak").
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_quantized_b200 import workloads as W  # noqa: E402
+
+METRIC = "quantized-KV decode attention: keys·heads/s and HBM GB/s vs B200 peak"
+UNIT = "keys·heads/s"
+L2_BYTES = 126 * 1024 * 1024
+
+WORKLOADS = {
+    "long_context": W.LONG_CONTEXT,
+    "llama8b": W.LLAMA8B_DECODE,
+}
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _bytes_per_key_head(w):
+    """Algorithmic HBM bytes per (cached token, KV head) of one attend launch: key codes + key norm + values."""
+    R = w.d * w.bits // 8
+    kb = R + 2
+    vb = (R + 2) if w.v_quant else 2 * w.d
+    return kb + vb
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def cpu_baseline(w, seconds=10.0):
+    """The fp64 oracle, as it stands, on one core: decode steps of single (batch row, KV head) units of the same
+    workload (G query heads over T cached tokens, plus the new token's write), repeated for about `seconds`."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_limits
+    except ImportError:  # pragma: no cover
+        threadpool_limits = None
+    inp = W.decode_inputs(w, B=1)
+    k, v, q, s = inp["k"][0], inp["v"][0], inp["q"][0], inp["signs"]
+    scale = 1.0 / math.sqrt(w.d)
+    ctx = threadpool_limits(1) if threadpool_limits else None
+    if ctx:
+        ctx.__enter__()
+    try:
+        units = 0
+        t_total = 0.0
+        hk = 0
+        while t_total < seconds and hk < w.Hkv:
+            kc, kn = oracle.write(k[hk], s, w.bits)  # cache state (setup, not timed)
+            vc, vn = oracle.write(v[hk], s, w.bits) if w.v_quant else (None, None)
+            t0 = time.perf_counter()
+            nk = oracle.write(k[hk, -1:], s, w.bits)  # the step's append of the new token
+            if w.v_quant:
+                oracle.write(v[hk, -1:], s, w.bits)
+            qq = q[hk * w.G:(hk + 1) * w.G][None]
+            kc[-1:], kn[-1:] = nk
+            if w.v_quant:
+                oracle.decode_attention(qq, kc[None, None], kn[None, None], s, w.bits, scale, vcodes=vc[None, None],
+                                        vn16=vn[None, None])
+            else:
+                oracle.decode_attention(qq, kc[None, None], kn[None, None], s, w.bits, scale, v=v[None, hk:hk + 1])
+            t_total += time.perf_counter() - t0
+            units += 1
+            hk += 1
+    finally:
+        if ctx:
+            ctx.__exit__(None, None, None)
+    key_heads = units * w.T * w.G
+    return {"value": key_heads / t_total, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{units} of {w.B * w.Hkv} (batch row, KV head) units of {w.name}: {w.G} query heads x "
+                      f"{w.T} tokens each, plus the new token's write; fp64 numpy, 1 thread, {t_total:.1f} s"}
+
+
+def run_axr(args, w):
+    import torch
+    import torch.distributed as dist
+    from kv_cache_quantized_b200 import ops
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    B, Hq, Hkv, T, d, bits = w.B, w.Hq, w.Hkv, w.T, w.d, w.bits
+    R = d * bits // 8
+    seed = w.seed + 1000 * rank
+    signs = torch.as_tensor(W.sign_vector(d, w.seed + 4), device=dev)
+    # --- setup: cache written once through the write path (not timed) ---
+    if w.keys == "outlier":
+        k = W.outlier_keys_device((B, Hkv, T, d), seed, dev)
+    else:
+        k = W.lognormal_rows_device((B, Hkv, T, d), seed, dev)
+    v = (W.lognormal_rows_device if w.v_quant else W.normal_device)((B, Hkv, T, d), seed + 2, dev)
+    kc, kn = ops.write_keys(k, signs, bits)
+    if w.v_quant:
+        vc, vn = ops.write_keys(v, signs, bits)
+        del v
+        v = None
+    del k
+    q = W.normal_device((B, Hq, d), seed + 3, dev, dtype=torch.float32)
+    knew = W.normal_device((B, Hkv, d), seed + 5, dev)
+    vnew = W.normal_device((B, Hkv, d), seed + 6, dev)
+    dst = ((torch.arange(B, device=dev)[:, None] * Hkv + torch.arange(Hkv, device=dev)[None, :]) * T + (T - 1))
+    dst = dst.reshape(-1).to(torch.int64)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    wsb = ops.attend_workspace_bytes(B, Hq, Hkv, T, d)
+    wsp = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def append(kn_in, vn_in):
+        ops.write_keys(kn_in, signs, bits, codes=kc.view(-1, R), norms=kn.view(-1), dst_rows=dst)
+        if w.v_quant:
+            ops.write_keys(vn_in, signs, bits, codes=vc.view(-1, R), norms=vn.view(-1), dst_rows=dst)
+        else:
+            v.view(-1, d).index_copy_(0, dst, vn_in.view(-1, d))  # fp16 values are stored as they are
+
+    def attend(q_in):
+        if w.v_quant:
+            ops.attend_decode(q_in, kc, kn, signs, bits, vcodes=vc, vnorms=vn, out=out, workspace=wsp)
+        else:
+            ops.attend_decode(q_in, kc, kn, signs, bits, v=v, out=out, workspace=wsp)
+
+    launches_per_step = (2 if w.v_quant else 1) + 2  # write(s) + partial + merge
+    if not w.v_quant:
+        launches_per_step += 0  # the fp16 value append is a torch copy, not one of the library's kernels
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        append(knew, vnew)
+        attend(q)
+    torch.cuda.synchronize()
+
+    # --- timed region: K steps, L2 flushed between steps (outside the per-step events) ---
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            flush.zero_()
+            e0, e1, e2 = ev[i]
+            e0.record(stream)
+            append(knew, vnew)
+            e1.record(stream)
+            attend(q)
+            e2.record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    step_ms = sum(e0.elapsed_time(e2) for e0, _, e2 in ev)
+    attend_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    clocks = clk.summary()
+
+    # --- end to end through the public API: pinned host inputs in, result out, every step ---
+    q_h = torch.empty_like(q, device="cpu").pin_memory().copy_(q.cpu())
+    k_h = torch.empty_like(knew, device="cpu").pin_memory().copy_(knew.cpu())
+    v_h = torch.empty_like(vnew, device="cpu").pin_memory().copy_(vnew.cpu())
+    o_h = torch.empty_like(out, device="cpu").pin_memory()
+    q_d, k_d, v_d = torch.empty_like(q), torch.empty_like(knew), torch.empty_like(vnew)
+    e2e = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        a, b_ = e2e[i]
+        a.record(stream)
+        q_d.copy_(q_h, non_blocking=True)
+        k_d.copy_(k_h, non_blocking=True)
+        v_d.copy_(v_h, non_blocking=True)
+        append(k_d, v_d)
+        attend(q_d)
+        o_h.copy_(out, non_blocking=True)
+        b_.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b_) for a, b_ in e2e)
+    h2d = q_h.numel() * 4 + k_h.numel() * 2 + v_h.numel() * 2
+    d2h = o_h.numel() * 4
+
+    # the scorer alone (axr_score) on the same cache, both table read modes, L2 flushed before each call
+    scorer = {}
+    if not args.no_scorer:
+        sc_out = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+        for mode in ("factored", "table"):
+            ops.set_gather(mode)
+            for _ in range(3):
+                ops.score(q, kc, kn, signs, bits, scale=1.0 / math.sqrt(d), out=sc_out)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)]
+            for a_, b2 in evs:
+                flush.zero_()
+                a_.record(stream)
+                ops.score(q, kc, kn, signs, bits, scale=1.0 / math.sqrt(d), out=sc_out)
+                b2.record(stream)
+            torch.cuda.synchronize()
+            ms = float(np.mean([a_.elapsed_time(b2) for a_, b2 in evs]))
+            sbytes = (R + 2 + 4 * w.G) * B * Hkv * T
+            scorer[mode] = {"ms": ms, "achieved_gbs": sbytes / (ms / 1e3) / 1e9, "algorithmic_bytes": sbytes}
+        ops.set_gather("factored")
+        del sc_out
+
+    # max over ranks
+    t = torch.tensor([step_ms, e2e_ms, float(np.mean(attend_ms))], device=dev, dtype=torch.float64)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    step_ms, e2e_ms, attend_avg_ms = t.tolist()
+    if ws > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return None
+
+    key_heads = B * T * Hq * ws * args.steps
+    value = key_heads / (step_ms / 1e3)
+    alg_bytes = _bytes_per_key_head(w) * B * Hkv * T
+    achieved = alg_bytes / (attend_avg_ms / 1e3) / 1e9
+    peak, peak_src = _peaks()
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": step_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8 codes / f32 math", "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "T": T, "Hq": Hq, "Hkv": Hkv, "d": d, "bits": bits,
+                   "values": "quantized b=%d" % bits if w.v_quant else "fp16", "parallelism": f"replicas x{ws}",
+                   "l2": "flushed between steps (256 MiB write outside the per-step events)"},
+        "hbm_gbs": alg_bytes * ws * args.steps / (step_ms / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "kernel": "attend_decode (partial + merge)", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "algorithmic_bytes": alg_bytes, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6.65 TB/s"},
+        "e2e": {"value": key_heads / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "scorer": {m: dict(v_, frac=v_["achieved_gbs"] / _peaks()[0]) for m, v_ in scorer.items()},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    return line
+
+
+def run_reference(args, w):
+    """The oracle as it stands on this host's cores, in place of the reference implementation (the pages ship no
+    code); one bounded sample per step."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        pass
+    vals = []
+    cb = None
+    for _ in range(args.steps):
+        cb = cpu_baseline(w, seconds=args.cpu_seconds / max(args.steps, 1))
+        vals.append(cb["value"])
+    value = float(np.mean(vals))
+    cb["value"] = value
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "bits": w.bits},
+            "cpu_baseline": cb, "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["axr", "reference"], default="axr")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="long_context")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU time budget of the oracle baseline")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch size (small ncu cases)")
+    ap.add_argument("--no-scorer", action="store_true", help="skip the separate axr_score measurement")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = WORKLOADS[args.workload]
+    if args.batch is not None:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch, name=w.name.replace(f"_b{w.B}_", f"_b{args.batch}_"))
+    if args.impl == "reference":
+        line = run_reference(args, w)
+    else:
+        line = run_axr(args, w)
+        if line is not None:
+            line["cpu_baseline"] = None if args.no_cpu_baseline else cpu_baseline(w, args.cpu_seconds)
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,173 @@
+/*
+ * axr.h -- C ABI of the B200 (sm_100a) implementation of AXELRAM decode-time attention from quantized key indices.
+ *
+ * Method source: "AXELRAM: Quantize Once, Never Dequantize" (arXiv 2604.02638), as carried by the ai-navigate-news
+ * digest (Key Points, Abstract) and the mlsanity index card (Abstract).  Keys are written once through a fixed
+ * orthogonal transform and a design-time scalar codebook ("transform on write"); attention scores are read by table
+ * lookup on the stored indices with no inverse transform and no reconstruction of the key ("table lookup on read").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Plain C types only.  fp16 tensors are passed as uint16_t* holding IEEE binary16 bit patterns.  `stream` is a
+ *    cudaStream_t (NULL = the legacy default stream).  Device pointers are marked [dev], host pointers [host].
+ *  - The caller owns every buffer.  The library never allocates device memory; entry points that need scratch take
+ *    a caller-provided workspace whose size comes from the matching *_workspace_bytes() function.
+ *  - Device work is asynchronous on `stream`.  Argument errors are detected on the host and returned before any
+ *    launch (no device work is queued).  Launch errors come from cudaGetLastError and return AXR_ECUDA.
+ *  - On any status other than AXR_OK, axr_last_error() returns a thread-local human-readable message.
+ *  - Fixed notation: d head dim (power of two), b bits per index, L = 2^b levels, s the +-1 sign vector, H the
+ *    Sylvester Walsh-Hadamard matrix scaled by 1/sqrt(d) (symmetric, H*H = I), G = Hq/Hkv (query head h reads KV
+ *    head h / G).
+ *  - Cache layouts (row-major, innermost last):
+ *      codes  [B, Hkv, Tcap, R] uint8, R = d*b/8 bytes per token: an LSB-first bitstream in which coordinate j
+ *             holds bits [j*b, j*b+b); index k means centroid c_k, k = 0 the most negative;
+ *      norms  [B, Hkv, Tcap] fp16, the token's L2 norm rounded to nearest even;
+ *      values [B, Hkv, Tcap, d] fp16 (AXR_V_F16), or codes + norms of the same shape as the keys (AXR_V_QUANT);
+ *      q      [B, Hq, d] fp32;  out [B, Hq, d] fp32;  scores [B, Hq, T] fp32.
+ *    Tcap >= T is the allocated capacity (row stride); only tokens t < seq_lens[b] (or t < T when seq_lens is
+ *    NULL) are read.
+ *  - Alignment: codes base 16 bytes, norms 4 bytes, q/out/scores 16 bytes, fp16 values 16 bytes.
+ *  - Supported: d in {64, 128} (the writer and the selector also take d = 8), b in {1, 2, 3, 4},
+ *    G in {1, 2, 4, 8}.  Anything else returns AXR_EUNSUPPORTED.
+ */
+#ifndef AXR_H_
+#define AXR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define AXR_API __attribute__((visibility("default")))
+#else
+#define AXR_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum axr_status {
+  AXR_OK = 0,
+  AXR_EINVAL = 1,        /* null pointer, negative or inconsistent size, misaligned pointer */
+  AXR_EUNSUPPORTED = 2,  /* d, b or G outside the compiled set */
+  AXR_ECUDA = 3,         /* a CUDA runtime call or a kernel launch failed */
+  AXR_EWORKSPACE = 4     /* workspace missing or smaller than the matching *_workspace_bytes() */
+} axr_status;
+
+typedef enum axr_dtype { AXR_F32 = 0, AXR_F16 = 1 } axr_dtype;
+typedef enum axr_vkind { AXR_V_F16 = 0, AXR_V_QUANT = 1 } axr_vkind;
+
+/* Thread-local message for the last non-OK status returned on this thread (empty string if none). */
+AXR_API const char* axr_last_error(void);
+
+/* ABI version: major*10000 + minor*100 + patch. */
+AXR_API int axr_version(void);
+
+/*
+ * axr_codebook -- design-time codebook (AXELRAM Abstract: the transform makes each coordinate ~N(0, 1/d), so the
+ * optimal scalar quantizer depends only on d and b).  Lloyd-Max quantizer of N(0,1), symmetrised, scaled by
+ * 1/sqrt(d).  Host only; no CUDA call.
+ *   centroids  [host] out, L doubles, increasing (unit scale: gamma_k / sqrt(d));
+ *   thresholds [host] out, L-1 doubles, increasing, t_k = (c_{k-1} + c_k) / 2.
+ * Errors: AXR_EINVAL for null outputs; AXR_EUNSUPPORTED for d not a power of two in [1, 4096] or b outside 1..4.
+ */
+AXR_API axr_status axr_codebook(int d, int bits, double* centroids, double* thresholds);
+
+/*
+ * axr_write_keys -- write path (AXELRAM Key Points, 2nd item, and Abstract: transform on write).  For each input
+ * vector x (also used for V when values are quantized):
+ *   n = ||x||_2 (fp32);  y = H (s .* x);  u = y / n (u = 0 when n = 0);
+ *   idx_j = #{k >= 1 : u_j >= t_k}  (a value on a threshold goes up);  pack idx LSB-first;  norm = fp16_rne(n).
+ *   x         [dev] [n_vec, d] of x_dtype (AXR_F32 or AXR_F16), contiguous rows;
+ *   signs     [dev] [d] int8, negative = -1, otherwise +1;
+ *   dst_rows  [dev] [n_vec] int64 destination row of each vector in codes/norms, or NULL for row i -> row i
+ *             (appending one token per (batch, KV head) into a [B, Hkv, Tcap] cache uses (b*Hkv + h)*Tcap + t);
+ *   codes     [dev] out, rows of R = d*b/8 bytes;  norms [dev] out, fp16 per row.
+ * Errors: AXR_EINVAL (null pointer, n_vec < 0, bad dtype, misalignment), AXR_EUNSUPPORTED (d or b), AXR_ECUDA.
+ * n_vec == 0 is a no-op.
+ */
+AXR_API axr_status axr_write_keys(const void* x, axr_dtype x_dtype, int64_t n_vec, int d, int bits, const int8_t* signs,
+                          const int64_t* dst_rows, uint8_t* codes, uint16_t* norms, void* stream);
+
+/*
+ * axr_score -- read-path scores (AXELRAM Key Points, 1st and 2nd items; Abstract: scores straight from the indices
+ * by table lookup, no inverse transform).  Per (batch b, query head h): q~ = H (s .* q); a d x L table
+ * LUT[j][k] = scale * q~_j * c_k is built in shared memory; for each token t < len_b
+ *   scores[b, h, t] = norm_t * sum_j LUT[j][idx_{t,j}],   and scores[b, h, t] = -inf for len_b <= t < T.
+ *   q [dev] [B,Hq,d] f32;  kcodes/knorms [dev] cache layout;  seq_lens [dev] [B] int32 or NULL (all T);
+ *   scores [dev] out [B, Hq, T] f32.
+ * Errors: AXR_EINVAL (pointers, sizes, T > Tcap, Hq not a multiple of Hkv, alignment), AXR_EUNSUPPORTED, AXR_ECUDA.
+ * T == 0 or B == 0 is a no-op.  seq_lens entries are clamped to [0, T].
+ */
+AXR_API axr_status axr_score(const float* q, const uint8_t* kcodes, const uint16_t* knorms, const int32_t* seq_lens, int B,
+                     int Hq, int Hkv, int T, int Tcap, int d, int bits, const int8_t* signs, float scale,
+                     float* scores, void* stream);
+
+/*
+ * Table read mode of axr_score (process-wide; default AXR_GATHER_FACTORED).  Both modes compute the same table
+ * entries LUT[j][k] = scale * q~_j * c_k (AXELRAM Key Points, 2nd item) and agree to fp32 rounding:
+ *   AXR_GATHER_TABLE     the d x 2^b table (G heads wide) is materialised in shared memory and gathered entry by
+ *                        entry, one thread per token;
+ *   AXR_GATHER_FACTORED  the table is held factored -- row factor q~_j in registers, column factor c_k gathered two
+ *                        coordinates at a time from a byte-indexed pair table -- and each entry is formed by the
+ *                        packed FMA that accumulates it; on B200 this takes half the shared-memory wavefronts.
+ * axr_attend_decode always reads the table in factored form.  Errors: AXR_EINVAL for an unknown mode.
+ */
+typedef enum axr_gather { AXR_GATHER_FACTORED = 0, AXR_GATHER_TABLE = 1 } axr_gather;
+AXR_API axr_status axr_set_gather(axr_gather mode);
+AXR_API axr_gather axr_get_gather(void);
+
+/* Bytes of workspace that axr_attend_decode / axr_dense_decode need for these sizes (0 when B, Hq or T is 0).
+ * Depends only on the arguments. */
+AXR_API size_t axr_attend_workspace_bytes(int B, int Hq, int Hkv, int T, int d);
+
+/*
+ * axr_attend_decode -- one decode step of attention over a quantized key cache: the scores of axr_score (scaled by
+ * `scale`, typically 1/sqrt(d)), an online softmax per split of the token axis, the value product, and a merge of
+ * the splits.  Values are fp16 (AXR_V_F16: out = sum_t p_t v_t) or quantized like the keys with the same signs
+ * (AXR_V_QUANT: the weighted sum is formed in the rotated domain and mapped back once, out = s .* H (sum_t p_t
+ * n^V_t c[idx^V_t])).  The softmax, the value product and the split merge are not on the pages (an SRAM macro only
+ * scores); they are the standard definitions.  A batch row with len_b = 0 gets out = 0.
+ *   v [dev] fp16 values or value codes;  vnorms [dev] value norms (AXR_V_QUANT) or NULL (AXR_V_F16);
+ *   out [dev] [B, Hq, d] f32;  workspace [dev] >= axr_attend_workspace_bytes(B, Hq, Hkv, T, d) bytes, 16-aligned.
+ * Errors: as axr_score, plus AXR_EWORKSPACE.
+ */
+AXR_API axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, const uint16_t* knorms, axr_vkind vkind,
+                             const void* v, const uint16_t* vnorms, const int32_t* seq_lens, int B, int Hq, int Hkv,
+                             int T, int Tcap, int d, int bits, const int8_t* signs, float scale, float* out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * axr_dense_decode -- the same decode step over an unquantized fp16 K/V cache (k, v [dev] [B, Hkv, Tcap, d] fp16):
+ * out = softmax(scale * q . k_t) . v.  Not part of the method: the bandwidth reference the quantized path is
+ * measured against.  Same workspace rule and errors as axr_attend_decode.
+ */
+AXR_API axr_status axr_dense_decode(const float* q, const uint16_t* k, const uint16_t* v, const int32_t* seq_lens, int B,
+                            int Hq, int Hkv, int T, int Tcap, int d, float scale, float* out, void* workspace,
+                            size_t ws_bytes, void* stream);
+
+/* Bytes of workspace for axr_select_signs with these sizes. */
+AXR_API size_t axr_select_workspace_bytes(int n_layers, int n_seq, int n_tok, int Hq, int Hkv, int d, int n_cand);
+
+/*
+ * axr_select_signs -- one-time, gradient-free sign-pattern selection (AXELRAM Key Points, 4th item; Abstract:
+ * candidates scored on a few calibration samples, no hardware cost).  Objective per candidate s^(c): the mean over
+ * every (layer, sequence, query head, position, coordinate) of (o_quant - o_ref)^2, where o_ref is unquantized
+ * softmax attention (computed once in fp64) and o_quant the same attention with every key written through
+ * axr_write_keys' path with signs s^(c) (values unquantized).  Softmax scale 1/sqrt(d); causal != 0 lets
+ * position i see keys 0..i only.
+ *   q [dev] [n_layers, n_seq, Hq, n_tok, d] f32;  k, v [dev] [n_layers, n_seq, Hkv, n_tok, d] fp16;
+ *   candidates [dev] [n_cand, d] int8 (+-1);  mse_out [dev] out [n_cand] f64;
+ *   best_out [dev] out, one int32: the first index of the minimum of mse_out;
+ *   workspace [dev] >= axr_select_workspace_bytes(...) bytes, 16-aligned.
+ * Errors: AXR_EINVAL, AXR_EUNSUPPORTED (d not in {8, 64, 128}, b, G), AXR_EWORKSPACE, AXR_ECUDA.
+ */
+AXR_API axr_status axr_select_signs(const float* q, const uint16_t* k, const uint16_t* v, int n_layers, int n_seq, int n_tok,
+                            int Hq, int Hkv, int d, int bits, const int8_t* candidates, int n_cand, int causal,
+                            double* mse_out, int32_t* best_out, void* workspace, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* AXR_H_ */

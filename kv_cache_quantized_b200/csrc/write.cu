@@ -1,0 +1,166 @@
+// Write path: rotate + normalise + quantize + pack, one warp per vector.
+//
+// AXELRAM Key Points (2nd item) and Abstract: "transform on write" into the domain where the fixed design-time
+// codebook applies.  Transform here: sign flip s .* x, then the Walsh-Hadamard butterfly (Sylvester order) held in
+// registers across the warp; norm ||x|| in fp32; index = number of thresholds at or below the unit coordinate.
+#include "axr_host.h"
+
+namespace axr {
+namespace {
+
+constexpr int kWriteWarps = 8;
+
+template <typename TIn, int VPL>
+__device__ __forceinline__ void load_lane(const TIn* row, int lane, float (&v)[VPL]);
+
+template <>
+__device__ __forceinline__ void load_lane<float, 4>(const float* row, int lane, float (&v)[4]) {
+  float4 a = reinterpret_cast<const float4*>(row)[lane];
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+template <>
+__device__ __forceinline__ void load_lane<float, 2>(const float* row, int lane, float (&v)[2]) {
+  float2 a = reinterpret_cast<const float2*>(row)[lane];
+  v[0] = a.x; v[1] = a.y;
+}
+template <>
+__device__ __forceinline__ void load_lane<float, 1>(const float* row, int lane, float (&v)[1]) {
+  v[0] = row[lane];
+}
+template <>
+__device__ __forceinline__ void load_lane<__half, 4>(const __half* row, int lane, float (&v)[4]) {
+  uint2 a = reinterpret_cast<const uint2*>(row)[lane];
+  float2 lo = __half22float2(*reinterpret_cast<__half2*>(&a.x));
+  float2 hi = __half22float2(*reinterpret_cast<__half2*>(&a.y));
+  v[0] = lo.x; v[1] = lo.y; v[2] = hi.x; v[3] = hi.y;
+}
+template <>
+__device__ __forceinline__ void load_lane<__half, 2>(const __half* row, int lane, float (&v)[2]) {
+  float2 a = __half22float2(reinterpret_cast<const __half2*>(row)[lane]);
+  v[0] = a.x; v[1] = a.y;
+}
+template <>
+__device__ __forceinline__ void load_lane<__half, 1>(const __half* row, int lane, float (&v)[1]) {
+  v[0] = __half2float(row[lane]);
+}
+
+template <int D, int BITS, typename TIn>
+__global__ void __launch_bounds__(kWriteWarps * kWarp)
+write_kernel(const TIn* __restrict__ x, int64_t n_vec, const int8_t* __restrict__ signs,
+             const int64_t* __restrict__ dst_rows, uint8_t* __restrict__ codes, __half* __restrict__ norms,
+             Codebook cb) {
+  constexpr int VPL = WarpVec<D>::VPL;
+  constexpr int LANES = WarpVec<D>::LANES;
+  constexpr int L = 1 << BITS;
+  constexpr int R = D * BITS / 8;  // bytes per packed row
+  __shared__ uint8_t idx_s[kWriteWarps][D];
+
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const bool active = lane < LANES;
+  float sg[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) sg[i] = active ? sign_of(signs[lane * VPL + i]) : 0.0f;
+  float tau[L - 1];
+#pragma unroll
+  for (int k = 0; k < L - 1; ++k) tau[k] = cb.tau[k];
+
+  for (int64_t vec = static_cast<int64_t>(blockIdx.x) * kWriteWarps + warp; vec < n_vec;
+       vec += static_cast<int64_t>(gridDim.x) * kWriteWarps) {
+    float v[VPL];
+    if (active) {
+      load_lane<TIn, VPL>(x + vec * D, lane, v);
+    } else {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) v[i] = 0.0f;
+    }
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      ss = fmaf(v[i], v[i], ss);
+      v[i] *= sg[i];
+    }
+    ss = warp_sum(ss);
+    const float n = sqrtf(ss);
+    fwht_warp<D>(v, lane);  // v = FWHT(s .* x) = sqrt(D) * H (s .* x)
+    if (active) {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const float w = n > 0.0f ? v[i] / n : 0.0f;  // = sqrt(D) * u
+        int q = 0;
+#pragma unroll
+        for (int k = 0; k < L - 1; ++k) q += (w >= tau[k]) ? 1 : 0;
+        idx_s[warp][lane * VPL + i] = static_cast<uint8_t>(q);
+      }
+    }
+    __syncwarp();
+    const int64_t row = dst_rows ? dst_rows[vec] : vec;
+    uint8_t* out = codes + row * R;
+    for (int byte = lane; byte < R; byte += kWarp) {
+      uint32_t acc = 0;
+      const int first = (byte * 8) / BITS, last = (byte * 8 + 7) / BITS;
+      for (int j = first; j <= last && j < D; ++j) {
+        const int pos = j * BITS - byte * 8;  // bit offset of coordinate j relative to this byte (may be < 0)
+        const uint32_t code = idx_s[warp][j];
+        acc |= pos >= 0 ? (code << pos) : (code >> (-pos));
+      }
+      out[byte] = static_cast<uint8_t>(acc & 0xffu);
+    }
+    if (lane == 0) norms[row] = __float2half_rn(n);
+    __syncwarp();
+  }
+}
+
+template <int D, int BITS>
+axr_status launch_write(const void* x, axr_dtype dt, int64_t n_vec, const int8_t* signs, const int64_t* dst,
+                        uint8_t* codes, uint16_t* norms, const Codebook& cb, cudaStream_t st) {
+  int64_t blocks = (n_vec + kWriteWarps - 1) / kWriteWarps;
+  const int64_t cap = static_cast<int64_t>(kSmCount) * 16;
+  if (blocks > cap) blocks = cap;
+  __half* nh = reinterpret_cast<__half*>(norms);
+  if (dt == AXR_F16)
+    write_kernel<D, BITS, __half><<<static_cast<unsigned>(blocks), kWriteWarps * kWarp, 0, st>>>(
+        static_cast<const __half*>(x), n_vec, signs, dst, codes, nh, cb);
+  else
+    write_kernel<D, BITS, float><<<static_cast<unsigned>(blocks), kWriteWarps * kWarp, 0, st>>>(
+        static_cast<const float*>(x), n_vec, signs, dst, codes, nh, cb);
+  return check_launch("axr_write_keys");
+}
+
+template <int D>
+axr_status dispatch_bits(int bits, const void* x, axr_dtype dt, int64_t n, const int8_t* s, const int64_t* dst,
+                         uint8_t* c, uint16_t* nr, const Codebook& cb, cudaStream_t st) {
+  switch (bits) {
+    case 1: return launch_write<D, 1>(x, dt, n, s, dst, c, nr, cb, st);
+    case 2: return launch_write<D, 2>(x, dt, n, s, dst, c, nr, cb, st);
+    case 3: return launch_write<D, 3>(x, dt, n, s, dst, c, nr, cb, st);
+    case 4: return launch_write<D, 4>(x, dt, n, s, dst, c, nr, cb, st);
+  }
+  return set_error(AXR_EUNSUPPORTED, "axr_write_keys: bits=%d", bits);
+}
+
+}  // namespace
+}  // namespace axr
+
+extern "C" axr_status axr_write_keys(const void* x, axr_dtype x_dtype, int64_t n_vec, int d, int bits,
+                                     const int8_t* signs, const int64_t* dst_rows, uint8_t* codes, uint16_t* norms,
+                                     void* stream) {
+  using namespace axr;
+  if (n_vec < 0) return set_error(AXR_EINVAL, "axr_write_keys: n_vec=%lld < 0", static_cast<long long>(n_vec));
+  if (x_dtype != AXR_F32 && x_dtype != AXR_F16) return set_error(AXR_EINVAL, "axr_write_keys: bad dtype");
+  if (d != 8 && d != 64 && d != 128) return set_error(AXR_EUNSUPPORTED, "axr_write_keys: d=%d not in {8,64,128}", d);
+  if (bits < 1 || bits > 4) return set_error(AXR_EUNSUPPORTED, "axr_write_keys: bits=%d outside 1..4", bits);
+  if (n_vec == 0) return set_error(AXR_OK, "");
+  if (!x || !signs || !codes || !norms) return set_error(AXR_EINVAL, "axr_write_keys: null pointer");
+  const uintptr_t xa = (x_dtype == AXR_F32 ? 4u : 2u) * (d >= 32 ? d / 32 : 1);
+  if (!aligned(x, xa)) return set_error(AXR_EINVAL, "axr_write_keys: x not %u-byte aligned", (unsigned)xa);
+  if (!aligned(norms, 2)) return set_error(AXR_EINVAL, "axr_write_keys: norms not 2-byte aligned");
+  if (dst_rows && !aligned(dst_rows, 8)) return set_error(AXR_EINVAL, "axr_write_keys: dst_rows not 8-byte aligned");
+  const Codebook* cb = codebook_for(d, bits);
+  if (!cb) return set_error(AXR_EINVAL, "axr_write_keys: codebook unavailable");
+  cudaStream_t st = as_stream(stream);
+  switch (d) {
+    case 8: return dispatch_bits<8>(bits, x, x_dtype, n_vec, signs, dst_rows, codes, norms, *cb, st);
+    case 64: return dispatch_bits<64>(bits, x, x_dtype, n_vec, signs, dst_rows, codes, norms, *cb, st);
+    default: return dispatch_bits<128>(bits, x, x_dtype, n_vec, signs, dst_rows, codes, norms, *cb, st);
+  }
+}

@@ -1,0 +1,231 @@
+"""Torch-tensor front end of libaxr: argument marshalling only.
+
+Every function here checks devices, dtypes and shapes, passes raw device pointers and the current CUDA stream to
+the C ABI (include/axr.h), and raises AxrError on a non-OK status.  All arithmetic runs in the library's kernels;
+tensors on the CPU are rejected (there is no fallback).
+
+Layouts (see include/axr.h): codes [B, Hkv, Tcap, d*b/8] uint8, norms [B, Hkv, Tcap] float16, values
+[B, Hkv, Tcap, d] float16, q [B, Hq, d] float32.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+
+import numpy as np
+import torch
+
+from . import _abi
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (libaxr has no CPU path)")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def row_bytes(d: int, bits: int) -> int:
+    return d * bits // 8
+
+
+def codebook(d: int, bits: int):
+    """(centroids [2^b], thresholds [2^b - 1]) float64 numpy arrays from the library's host codebook."""
+    L = 1 << bits
+    c = np.zeros(L, dtype=np.float64)
+    t = np.zeros(max(L - 1, 1), dtype=np.float64)
+    st = _abi.lib().axr_codebook(d, bits, c.ctypes.data_as(ctypes.c_void_p), t.ctypes.data_as(ctypes.c_void_p))
+    _abi.check(st, "axr_codebook")
+    return c, t[: L - 1]
+
+
+def write_keys(x: torch.Tensor, signs: torch.Tensor, bits: int, codes: torch.Tensor | None = None,
+               norms: torch.Tensor | None = None, dst_rows: torch.Tensor | None = None):
+    """Quantize rows of x [..., d] (float16 or float32).  Returns (codes uint8 [..., d*b/8], norms float16 [...]).
+
+    With dst_rows (int64 [n_vec]) the rows land at those row indices of the given codes/norms buffers (e.g. a cache
+    viewed as [B*Hkv*Tcap, R]); codes and norms are then required.
+    """
+    _need_cuda("x", x)
+    _need_cuda("signs", signs, torch.int8)
+    if x.dtype not in (torch.float16, torch.float32):
+        raise TypeError("x must be float16 or float32")
+    d = x.shape[-1]
+    n_vec = x.numel() // d if d else 0
+    R = row_bytes(d, bits)
+    if dst_rows is None:
+        if codes is None:
+            codes = torch.empty(x.shape[:-1] + (R,), dtype=torch.uint8, device=x.device)
+        if norms is None:
+            norms = torch.empty(x.shape[:-1], dtype=torch.float16, device=x.device)
+    else:
+        _need_cuda("dst_rows", dst_rows, torch.int64)
+        if codes is None or norms is None:
+            raise ValueError("dst_rows needs the destination codes and norms buffers")
+        if dst_rows.numel() != n_vec:
+            raise ValueError("dst_rows must hold one row index per vector")
+    _need_cuda("codes", codes, torch.uint8)
+    _need_cuda("norms", norms, torch.float16)
+    if dst_rows is None and (codes.numel() != n_vec * R or norms.numel() != n_vec):
+        raise ValueError("codes/norms do not match x")
+    dt = _abi.F16 if x.dtype == torch.float16 else _abi.F32
+    st = _abi.lib().axr_write_keys(_ptr(x), dt, n_vec, d, bits, _ptr(signs), _ptr(dst_rows), _ptr(codes),
+                                   _ptr(norms), _stream())
+    _abi.check(st, "axr_write_keys")
+    return codes, norms
+
+
+def _cache_dims(q, kcodes, knorms, d, bits, T):
+    _need_cuda("q", q, torch.float32)
+    _need_cuda("kcodes", kcodes, torch.uint8)
+    _need_cuda("knorms", knorms, torch.float16)
+    if q.dim() != 3 or kcodes.dim() != 4 or knorms.dim() != 3:
+        raise ValueError("q [B,Hq,d], kcodes [B,Hkv,Tcap,R], knorms [B,Hkv,Tcap] expected")
+    B, Hq, _ = q.shape
+    _, Hkv, Tcap, R = kcodes.shape
+    if R != row_bytes(d, bits) or kcodes.shape[0] != B or tuple(knorms.shape) != (B, Hkv, Tcap):
+        raise ValueError("cache shapes do not match q, d and bits")
+    T = Tcap if T is None else int(T)
+    return B, Hq, Hkv, Tcap, T
+
+
+def _lens(seq_lens, B):
+    if seq_lens is None:
+        return None
+    _need_cuda("seq_lens", seq_lens, torch.int32)
+    if seq_lens.numel() != B:
+        raise ValueError("seq_lens must have B entries")
+    return seq_lens
+
+
+def score(q, kcodes, knorms, signs, bits, scale=1.0, seq_lens=None, T=None, out=None):
+    """Scores [B, Hq, T] float32 = scale * norm_t * sum_j LUT[j][idx_{t,j}] (tokens >= seq_lens[b] get -inf)."""
+    d = q.shape[-1]
+    B, Hq, Hkv, Tcap, T = _cache_dims(q, kcodes, knorms, d, bits, T)
+    _need_cuda("signs", signs, torch.int8)
+    seq_lens = _lens(seq_lens, B)
+    if out is None:
+        out = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    _need_cuda("out", out, torch.float32)
+    st = _abi.lib().axr_score(_ptr(q), _ptr(kcodes), _ptr(knorms), _ptr(seq_lens), B, Hq, Hkv, T, Tcap, d, bits,
+                              _ptr(signs), float(scale), _ptr(out), _stream())
+    _abi.check(st, "axr_score")
+    return out
+
+
+def set_gather(mode: str) -> None:
+    """Table read mode of score(): "factored" (default) or "table" (the materialised table, gathered per entry)."""
+    code = {"factored": _abi.GATHER_FACTORED, "table": _abi.GATHER_TABLE}[mode]
+    _abi.check(_abi.lib().axr_set_gather(code), "axr_set_gather")
+
+
+def get_gather() -> str:
+    return "table" if _abi.lib().axr_get_gather() == _abi.GATHER_TABLE else "factored"
+
+
+def attend_workspace_bytes(B, Hq, Hkv, T, d) -> int:
+    return int(_abi.lib().axr_attend_workspace_bytes(B, Hq, Hkv, T, d))
+
+
+def _workspace(nbytes, device, ws):
+    if ws is None:
+        return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    _need_cuda("workspace", ws, torch.uint8)
+    return ws
+
+
+def attend_decode(q, kcodes, knorms, signs, bits, v=None, vcodes=None, vnorms=None, scale=None, seq_lens=None,
+                  T=None, out=None, workspace=None):
+    """One decode step over a quantized key cache.  Values: v (float16 [B,Hkv,Tcap,d]) or vcodes/vnorms (quantized
+    like the keys with the same signs).  Returns out [B, Hq, d] float32."""
+    d = q.shape[-1]
+    B, Hq, Hkv, Tcap, T = _cache_dims(q, kcodes, knorms, d, bits, T)
+    _need_cuda("signs", signs, torch.int8)
+    seq_lens = _lens(seq_lens, B)
+    if (v is None) == (vcodes is None):
+        raise ValueError("pass exactly one of v or vcodes")
+    if v is not None:
+        _need_cuda("v", v, torch.float16)
+        if tuple(v.shape) != (B, Hkv, Tcap, d):
+            raise ValueError("v must be [B, Hkv, Tcap, d]")
+        vkind, vptr, vnptr = _abi.V_F16, _ptr(v), None
+    else:
+        _need_cuda("vcodes", vcodes, torch.uint8)
+        _need_cuda("vnorms", vnorms, torch.float16)
+        if vcodes.shape != kcodes.shape or vnorms.shape != knorms.shape:
+            raise ValueError("vcodes/vnorms must have the key cache's shapes")
+        vkind, vptr, vnptr = _abi.V_QUANT, _ptr(vcodes), _ptr(vnorms)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    _need_cuda("out", out, torch.float32)
+    nbytes = attend_workspace_bytes(B, Hq, Hkv, T, d)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = _abi.lib().axr_attend_decode(_ptr(q), _ptr(kcodes), _ptr(knorms), vkind, vptr, vnptr, _ptr(seq_lens), B, Hq,
+                                      Hkv, T, Tcap, d, bits, _ptr(signs), scale, _ptr(out), _ptr(ws), ws.numel(),
+                                      _stream())
+    _abi.check(st, "axr_attend_decode")
+    return out
+
+
+def dense_decode(q, k, v, scale=None, seq_lens=None, T=None, out=None, workspace=None):
+    """Decode attention over an unquantized float16 K/V cache [B, Hkv, Tcap, d] (the bandwidth reference)."""
+    _need_cuda("q", q, torch.float32)
+    _need_cuda("k", k, torch.float16)
+    _need_cuda("v", v, torch.float16)
+    B, Hq, d = q.shape
+    _, Hkv, Tcap, _ = k.shape
+    if tuple(v.shape) != tuple(k.shape) or k.shape[0] != B or k.shape[3] != d:
+        raise ValueError("k, v must be [B, Hkv, Tcap, d]")
+    T = Tcap if T is None else int(T)
+    seq_lens = _lens(seq_lens, B)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    nbytes = attend_workspace_bytes(B, Hq, Hkv, T, d)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = _abi.lib().axr_dense_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(seq_lens), B, Hq, Hkv, T, Tcap, d, scale,
+                                     _ptr(out), _ptr(ws), ws.numel(), _stream())
+    _abi.check(st, "axr_dense_decode")
+    return out
+
+
+def select_workspace_bytes(layers, seqs, tokens, Hq, Hkv, d, n_cand) -> int:
+    return int(_abi.lib().axr_select_workspace_bytes(layers, seqs, tokens, Hq, Hkv, d, n_cand))
+
+
+def select_signs(q, k, v, candidates, bits, causal=True, workspace=None):
+    """Score candidate sign vectors [C, d] int8 on calibration q [Ly,S,Hq,N,d] f32, k/v [Ly,S,Hkv,N,d] f16.
+    Returns (mse float64 [C], best int32 [1]) as CUDA tensors."""
+    _need_cuda("q", q, torch.float32)
+    _need_cuda("k", k, torch.float16)
+    _need_cuda("v", v, torch.float16)
+    _need_cuda("candidates", candidates, torch.int8)
+    Ly, S, Hq, N, d = q.shape
+    Hkv = k.shape[2]
+    if tuple(k.shape) != (Ly, S, Hkv, N, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k, v must be [Ly, S, Hkv, N, d]")
+    C = candidates.shape[0]
+    if tuple(candidates.shape) != (C, d):
+        raise ValueError("candidates must be [C, d]")
+    mse = torch.empty(C, dtype=torch.float64, device=q.device)
+    best = torch.empty(1, dtype=torch.int32, device=q.device)
+    nbytes = select_workspace_bytes(Ly, S, N, Hq, Hkv, d, C)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = _abi.lib().axr_select_signs(_ptr(q), _ptr(k), _ptr(v), Ly, S, N, Hq, Hkv, d, bits, _ptr(candidates), C,
+                                     1 if causal else 0, _ptr(mse), _ptr(best), _ptr(ws), ws.numel(), _stream())
+    _abi.check(st, "axr_select_signs")
+    return mse, best

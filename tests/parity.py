@@ -1,0 +1,84 @@
+"""Parity criteria between the CUDA path and the fp64 oracle (test infrastructure).
+
+* Indices: bit-exact, except coordinates whose oracle unit value u lies within 1e-6 of the threshold that separates
+  the two indices (adjacent cells only); such mismatches are counted and must stay below 1e-5 of all coordinates.
+* Norms: the fp16 bits are exact, except where the fp64 norm lies within a few fp32 ulps of an fp16 rounding
+  midpoint (the kernel rounds its fp32 norm, the oracle its fp64 norm).
+* Scores: |s_gpu - s_oracle| <= 1e-6 + 1e-5 * A_t, with A_t = scale * n16_t * sum_j |q~_j c_{idx_t,j}| (fp32
+  summation error is bounded by the sum of the absolute terms, not by |s|); the strict |s|-relative reading is
+  reported alongside.
+* Attention outputs: per (batch, head) ||o_gpu - o_oracle|| / ||o_oracle|| <= 2e-3.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+
+BOUNDARY = 1e-6
+MISMATCH_FRACTION = 1e-5
+SCORE_ABS = 1e-6
+SCORE_REL = 1e-5
+OUT_REL_L2 = 2e-3
+
+
+def check_indices(gpu_codes, x, signs, d, bits):
+    """Compare packed GPU codes with the oracle's for the same inputs.  Returns (n_mismatch, n_coords)."""
+    idx, n, n16, u = oracle.quantize_rows(x, signs, bits)
+    g = oracle.unpack(np.asarray(gpu_codes).reshape(idx.shape[:-1] + (-1,)), d, bits)
+    mism = g != idx
+    nm = int(mism.sum())
+    if nm:
+        _, t = oracle.codebook(d, bits)
+        gi, oi, uu = g[mism], idx[mism], u[mism]
+        assert np.all(np.abs(gi - oi) == 1), "index mismatch by more than one cell"
+        k = np.maximum(gi, oi)
+        dist = np.abs(uu - t[k - 1])
+        assert np.all(dist < BOUNDARY), f"index mismatch {dist.max():.3e} away from a threshold"
+    assert nm < MISMATCH_FRACTION * idx.size + 1, f"{nm} index mismatches of {idx.size}"
+    return nm, idx.size
+
+
+def check_norms(gpu_n16, x):
+    x = np.asarray(x, dtype=np.float64)
+    n = np.sqrt(np.sum(x * x, axis=-1))
+    want = n.astype(np.float16)
+    got = np.asarray(gpu_n16).reshape(want.shape)
+    mism = got.view(np.uint16) != want.view(np.uint16)
+    if mism.any():
+        nn = n[mism]
+        lo = nn.astype(np.float16).astype(np.float64)
+        # the fp16 neighbour on the other side and the midpoint between them
+        up = np.nextafter(nn.astype(np.float16), np.float16(np.inf)).astype(np.float64)
+        dn = np.nextafter(nn.astype(np.float16), np.float16(-np.inf)).astype(np.float64)
+        mid = np.where(np.abs(up - nn) < np.abs(dn - nn), (lo + up) / 2, (lo + dn) / 2)
+        assert np.all(np.abs(nn - mid) <= 4 * 2.0 ** -23 * nn), "fp16 norm differs away from a rounding midpoint"
+    return int(mism.sum())
+
+
+def abs_score_scale(q, codes, n16, signs, bits, scale):
+    """A_t = scale * n16_t * sum_j |LUT[j, idx_{t,j}]| for one query q [d] and rows codes [T, R]."""
+    d = q.shape[-1]
+    lut = np.abs(oracle.query_lut(q, signs, bits))
+    idx = oracle.unpack(codes, d, bits)
+    return abs(scale) * np.asarray(n16, np.float64) * lut[np.arange(d)[None, :], idx].sum(-1)
+
+
+def check_scores(gpu, want, A):
+    gpu = np.asarray(gpu, np.float64)
+    err = np.abs(gpu - want)
+    bound = SCORE_ABS + SCORE_REL * A
+    bad = err > bound
+    assert not bad.any(), f"{int(bad.sum())} scores out of tolerance; worst ratio {np.max(err / bound):.3g}"
+    strict = err > SCORE_ABS + SCORE_REL * np.abs(want)
+    return float(np.max(err / bound)), int(strict.sum())
+
+
+def check_outputs(gpu, want):
+    gpu = np.asarray(gpu, np.float64)
+    num = np.linalg.norm(gpu - want, axis=-1)
+    den = np.linalg.norm(want, axis=-1)
+    rel = np.where(den > 0, num / np.where(den > 0, den, 1), num)
+    assert np.all(rel <= OUT_REL_L2), f"max relative L2 error {rel.max():.3e}"
+    return float(rel.max())

@@ -1,0 +1,126 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every function include/axr.h declares, its
+host codebook matches the oracle's, and bad arguments come back as error statuses before any CUDA call."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from kv_cache_quantized_b200 import _abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(_abi.LIB_PATH):
+        from kv_cache_quantized_b200 import build
+        build.build()
+    return _abi.lib()
+
+
+def _declared():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"AXR_API\s+[\w\s\*]+?\b(axr_\w+)\s*\(", txt)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = _declared()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in _abi.SIGNATURES, f"{n} has no ctypes signature"
+
+
+def test_version(L):
+    assert L.axr_version() == 100
+
+
+@pytest.mark.parametrize("d", [8, 64, 128])
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+def test_host_codebook_matches_oracle(L, d, bits):
+    n = 1 << bits
+    c = np.zeros(n)
+    t = np.zeros(n - 1 if n > 1 else 1)
+    st = L.axr_codebook(d, bits, c.ctypes.data_as(ctypes.c_void_p), t.ctypes.data_as(ctypes.c_void_p))
+    assert st == 0
+    oc, ot = oracle.codebook(d, bits)
+    assert np.max(np.abs(c - oc)) < 1e-13
+    assert np.max(np.abs(t[: n - 1] - ot)) < 1e-13
+    assert t[n // 2 - 1] == 0.0  # exact middle threshold
+
+
+def test_codebook_errors(L):
+    buf = np.zeros(16)
+    p = buf.ctypes.data_as(ctypes.c_void_p)
+    assert L.axr_codebook(100, 2, p, p) == 2
+    assert L.axr_codebook(128, 5, p, p) == 2
+    assert L.axr_codebook(128, 2, None, p) == 1
+    assert b"null" in L.axr_last_error()
+
+
+FAKE = 0x10000  # a 64 KiB-aligned non-null address; never dereferenced because every call below fails validation
+
+
+def test_write_argument_errors(L):
+    assert L.axr_write_keys(FAKE, 0, -1, 128, 4, FAKE, None, FAKE, FAKE, None) == 1
+    assert L.axr_write_keys(FAKE, 0, 5, 96, 4, FAKE, None, FAKE, FAKE, None) == 2
+    assert L.axr_write_keys(FAKE, 0, 5, 128, 5, FAKE, None, FAKE, FAKE, None) == 2
+    assert L.axr_write_keys(FAKE, 7, 5, 128, 4, FAKE, None, FAKE, FAKE, None) == 1
+    assert L.axr_write_keys(None, 0, 5, 128, 4, FAKE, None, FAKE, FAKE, None) == 1
+    assert L.axr_write_keys(FAKE + 4, 0, 5, 128, 4, FAKE, None, FAKE, FAKE, None) == 1  # fp32 rows need 16 B
+    assert L.axr_write_keys(None, 0, 0, 128, 4, None, None, None, None, None) == 0  # empty is a no-op
+
+
+def test_score_argument_errors(L):
+    args = lambda **kw: dict(dict(q=FAKE, kc=FAKE, kn=FAKE, sl=None, B=2, Hq=8, Hkv=2, T=10, Tcap=16, d=128,
+                                  bits=4, s=FAKE, scale=1.0, out=FAKE), **kw)
+    call = lambda a: L.axr_score(a["q"], a["kc"], a["kn"], a["sl"], a["B"], a["Hq"], a["Hkv"], a["T"], a["Tcap"],
+                                 a["d"], a["bits"], a["s"], a["scale"], a["out"], None)
+    assert call(args(Hq=6, Hkv=4)) == 1          # Hq not a multiple of Hkv
+    assert call(args(T=20)) == 1                 # T > Tcap
+    assert call(args(d=32)) == 2
+    assert call(args(Hq=6, Hkv=2)) == 2          # G = 3
+    assert call(args(bits=0)) == 2
+    assert call(args(q=None)) == 1
+    assert call(args(kc=FAKE + 8)) == 1          # codes need 16-byte alignment
+    assert call(args(scale=float("inf"))) == 1
+    assert call(args(B=0)) == 0
+
+
+def test_attend_workspace_rules(L):
+    ws = L.axr_attend_workspace_bytes(8, 32, 8, 32768, 128)
+    assert ws > 0 and ws % 256 == 0
+    assert L.axr_attend_workspace_bytes(8, 32, 8, 32768, 128) == ws
+    assert L.axr_attend_workspace_bytes(0, 32, 8, 32768, 128) == 0
+    assert L.axr_attend_workspace_bytes(1, 32, 8, 100, 128) > 0
+    call = lambda wsb, vk=0, vn=None: L.axr_attend_decode(FAKE, FAKE, FAKE, vk, FAKE, vn, None, 8, 32, 8, 32768,
+                                                          32768, 128, 4, FAKE, 0.088, FAKE, FAKE, wsb, None)
+    assert call(ws - 1) == 4
+    assert L.axr_attend_decode(FAKE, FAKE, FAKE, 0, FAKE, None, None, 8, 32, 8, 32768, 32768, 128, 4, FAKE, 0.088,
+                               FAKE, None, ws, None) == 4
+    assert call(ws, vk=1, vn=None) == 1          # quantized V needs value norms
+    assert call(ws, vk=3) == 1
+    assert L.axr_dense_decode(FAKE, FAKE, FAKE, None, 8, 32, 8, 32768, 32768, 128, 0.088, FAKE, FAKE, ws - 1,
+                              None) == 4
+
+
+def test_select_argument_errors(L):
+    ws = L.axr_select_workspace_bytes(2, 2, 64, 16, 2, 128, 8)
+    assert ws > 0
+    call = lambda **kw: L.axr_select_signs(FAKE, FAKE, FAKE, kw.get("Ly", 2), 2, 64, kw.get("Hq", 16), 2,
+                                           kw.get("d", 128), kw.get("bits", 4), FAKE, 8, 1, FAKE, FAKE,
+                                           kw.get("ws", FAKE), kw.get("wsb", ws), None)
+    assert call(d=32) == 2
+    assert call(bits=7) == 2
+    assert call(Hq=15) == 1
+    assert call(Ly=0) == 1
+    assert call(wsb=ws - 1) == 4
+    assert call(ws=None) == 4

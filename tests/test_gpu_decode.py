@@ -1,0 +1,195 @@
+"""GPU parity of the read path: LUT scores (axr_score), split-T decode attention over fp16 or quantized values
+(axr_attend_decode) and the dense fp16 reference (axr_dense_decode), against the oracle on the same inputs.
+
+Small cases span several 256-token tiles, several splits and a ragged tail; the full-size workloads run in the
+launch configuration the benchmark uses and are checked on sampled (batch, head) outputs."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from kv_cache_quantized_b200 import ops
+from kv_cache_quantized_b200 import workloads as W
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def cuda(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def padded(a, Tcap, axis=2, fill=0):
+    pad = [(0, 0)] * a.ndim
+    pad[axis] = (0, Tcap - a.shape[axis])
+    return np.pad(a, pad, constant_values=fill)
+
+
+def oracle_cache(B, Hkv, T, d, bits, seed, vq, keys="lognormal"):
+    """Host inputs and oracle-written codes for a small decode case."""
+    shape = (B, Hkv, T, d)
+    k = W.outlier_keys(shape, seed) if keys == "outlier" else W.lognormal_rows(shape, seed, dtype=np.float16)
+    v = W.lognormal_rows(shape, seed + 1, dtype=np.float16) if vq else W.normal(shape, seed + 1, np.float16)
+    s = W.sign_vector(d, seed + 2)
+    kc, kn = oracle.write(k, s, bits)
+    vc, vn = oracle.write(v, s, bits) if vq else (None, None)
+    return k, v, s, kc, kn, vc, vn
+
+
+SMALL = [(d, b, 4, vq) for d in (64, 128) for b in (1, 2, 3, 4) for vq in (False, True)]
+SMALL += [(128, 3, g, vq) for g in (1, 2, 8) for vq in (False, True)]
+SMALL += [(64, 4, g, False) for g in (1, 2, 8)]
+
+
+@pytest.mark.parametrize("d,bits,G", sorted({(d, b, g) for d, b, g, _ in SMALL}))
+def test_score_matches_oracle(d, bits, G):
+    B, Hkv, T, Tcap = 2, 2, 2500, 2560
+    Hq = G * Hkv
+    k, v, s, kc, kn, _, _ = oracle_cache(B, Hkv, T, d, bits, 300 + d + bits + G, False)
+    q = W.normal((B, Hq, d), 400 + G, np.float32)
+    lens = np.array([T, 1111], np.int32)
+    scale = 0.7
+    out = ops.score(cuda(q), cuda(padded(kc, Tcap)), cuda(padded(kn, Tcap)), cuda(s), bits, scale=scale,
+                    seq_lens=cuda(lens), T=T).cpu().numpy()
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            Tb = lens[b]
+            want = oracle.score_lut(q[b, h], kc[b, hk, :Tb], kn[b, hk, :Tb], s, bits, scale)
+            A = parity.abs_score_scale(q[b, h].astype(np.float64), kc[b, hk, :Tb], kn[b, hk, :Tb], s, bits, scale)
+            parity.check_scores(out[b, h, :Tb], want, A)
+            assert np.all(np.isneginf(out[b, h, Tb:]))
+
+
+@pytest.mark.parametrize("d,bits,G,vq", SMALL)
+def test_attend_matches_oracle(d, bits, G, vq):
+    B, Hkv, T, Tcap = 2, 2, 2500, 2600
+    Hq = G * Hkv
+    k, v, s, kc, kn, vc, vn = oracle_cache(B, Hkv, T, d, bits, 500 + d + bits + G, vq)
+    q = W.normal((B, Hq, d), 600 + G, np.float32)
+    lens = np.array([T, 777], np.int32)
+    scale = 1.0 / math.sqrt(d)
+    args = dict(seq_lens=cuda(lens), T=T, scale=scale)
+    if vq:
+        out = ops.attend_decode(cuda(q), cuda(padded(kc, Tcap)), cuda(padded(kn, Tcap)), cuda(s), bits,
+                                vcodes=cuda(padded(vc, Tcap)), vnorms=cuda(padded(vn, Tcap)), **args)
+        want = oracle.decode_attention(q, kc, kn, s, bits, scale, vcodes=vc, vn16=vn, seq_lens=lens)
+    else:
+        out = ops.attend_decode(cuda(q), cuda(padded(kc, Tcap)), cuda(padded(kn, Tcap)), cuda(s), bits,
+                                v=cuda(padded(v, Tcap)), **args)
+        want = oracle.decode_attention(q, kc, kn, s, bits, scale, v=v, seq_lens=lens)
+    parity.check_outputs(out.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("vq", [False, True])
+def test_attend_edge_cases(vq):
+    d, bits, Hkv, G = 128, 4, 2, 4
+    Hq = Hkv * G
+    B, T, Tcap = 4, 300, 320
+    k, v, s, kc, kn, vc, vn = oracle_cache(B, Hkv, T, d, bits, 700, vq)
+    q = W.normal((B, Hq, d), 701, np.float32)
+    q[3] = 0.0  # zero query: uniform softmax
+    lens = np.array([1, 0, 300, 257], np.int32)
+    vargs = dict(vcodes=cuda(padded(vc, Tcap)), vnorms=cuda(padded(vn, Tcap))) if vq else dict(v=cuda(padded(v, Tcap)))
+    out = ops.attend_decode(cuda(q), cuda(padded(kc, Tcap)), cuda(padded(kn, Tcap)), cuda(s), bits, seq_lens=cuda(lens),
+                            T=T, **vargs).cpu().numpy()
+    okw = dict(vcodes=vc, vn16=vn) if vq else dict(v=v)
+    want = oracle.decode_attention(q, kc, kn, s, bits, 1 / math.sqrt(d), seq_lens=lens, **okw)
+    parity.check_outputs(out, want)
+    assert np.all(out[1] == 0.0)  # empty row
+    # T = 0 gives zeros
+    out0 = ops.attend_decode(cuda(q), cuda(padded(kc, Tcap)), cuda(padded(kn, Tcap)), cuda(s), bits, T=0,
+                             **vargs).cpu().numpy()
+    assert np.all(out0 == 0.0)
+
+
+def test_dense_matches_oracle_attention():
+    B, Hkv, G, T, Tcap, d = 3, 2, 4, 2100, 2200, 128
+    k = W.lognormal_rows((B, Hkv, T, d), 800, dtype=np.float16)
+    v = W.normal((B, Hkv, T, d), 801, np.float16)
+    q = W.normal((B, Hkv * G, d), 802, np.float32)
+    lens = np.array([T, 5, 1500], np.int32)
+    out = ops.dense_decode(cuda(q), cuda(padded(k, Tcap)), cuda(padded(v, Tcap)), seq_lens=cuda(lens),
+                           T=T).cpu().numpy()
+    for b in range(B):
+        Tb = lens[b]
+        want = oracle.attention(q[b][:, None, :], k[b, :, :Tb], v[b, :, :Tb], causal=False)[:, 0, :]
+        parity.check_outputs(out[b], want)
+
+
+def test_split_count_invariance():
+    """The same row attended with B=1 (many splits) and inside B=8 (fewer splits) agrees to fp32 noise."""
+    d, bits, Hkv, G, T = 128, 4, 8, 4, 32768
+    shape = (8, Hkv, T, d)
+    k = W.lognormal_rows(shape, 900, dtype=np.float16)
+    v = W.normal(shape, 901, np.float16)
+    s = W.sign_vector(d, 902)
+    q = W.normal((8, Hkv * G, d), 903, np.float32)
+    kc, kn = ops.write_keys(cuda(k), cuda(s), bits)
+    vt = cuda(v)
+    qt = cuda(q)
+    st = cuda(s)
+    full = ops.attend_decode(qt, kc, kn, st, bits, v=vt)
+    one = ops.attend_decode(qt[:1].contiguous(), kc[:1].contiguous(), kn[:1].contiguous(), st, bits,
+                            v=vt[:1].contiguous())
+    assert ops.attend_workspace_bytes(1, 32, 8, T, d) // 1 != ops.attend_workspace_bytes(8, 32, 8, T, d) // 8
+    a, b = full[0].cpu().numpy(), one[0].cpu().numpy()
+    assert np.max(np.abs(a - b)) <= 1e-5 * np.max(np.abs(a))
+
+
+def _full_size(w, samples, seed_q=None):
+    """Full-size workload in the benchmark's launch configuration: the cache is written on the GPU, attention runs
+    on the GPU; sampled (batch, head) outputs are recomputed by the oracle from the same host inputs."""
+    inp = W.decode_inputs(w)
+    k, v, q, s = inp["k"], inp["v"], inp["q"], inp["signs"]
+    st = cuda(s)
+    kc, kn = ops.write_keys(cuda(k), st, w.bits)
+    if w.v_quant:
+        vc, vn = ops.write_keys(cuda(v), st, w.bits)
+        out = ops.attend_decode(cuda(q), kc, kn, st, w.bits, vcodes=vc, vnorms=vn)
+    else:
+        out = ops.attend_decode(cuda(q), kc, kn, st, w.bits, v=cuda(v))
+    out = out.cpu().numpy()
+    kc_h, kn_h = kc.cpu().numpy(), kn.cpu().numpy()
+    vc_h = vn_h = None
+    if w.v_quant:
+        vc_h, vn_h = vc.cpu().numpy(), vn.cpu().numpy()
+    scale = 1.0 / math.sqrt(w.d)
+    for b, h in samples:
+        hk = h // w.G
+        nmk, _ = parity.check_indices(kc_h[b, hk], k[b, hk], s, w.d, w.bits)
+        parity.check_norms(kn_h[b, hk], k[b, hk])
+        okc, okn = oracle.write(k[b, hk], s, w.bits)
+        if w.v_quant:
+            parity.check_indices(vc_h[b, hk], v[b, hk], s, w.d, w.bits)
+            ovc, ovn = oracle.write(v[b, hk], s, w.bits)
+            want = oracle.decode_attention(q[b:b + 1, h:h + 1], okc[None, None], okn[None, None], s, w.bits, scale,
+                                           vcodes=ovc[None, None], vn16=ovn[None, None])
+        else:
+            want = oracle.decode_attention(q[b:b + 1, h:h + 1], okc[None, None], okn[None, None], s, w.bits, scale,
+                                           v=v[b:b + 1, hk:hk + 1])
+        parity.check_outputs(out[b:b + 1, h:h + 1], want)
+        # and the scores of this head against the oracle on the oracle's codes
+        sc = ops.score(cuda(q[b:b + 1, hk * w.G:(hk + 1) * w.G]), cuda(okc[None, None]), cuda(okn[None, None]), st,
+                       w.bits, scale=scale).cpu().numpy()[0, h - hk * w.G]
+        want_s = oracle.score_lut(q[b, h], okc, okn, s, w.bits, scale)
+        A = parity.abs_score_scale(q[b, h].astype(np.float64), okc, okn, s, w.bits, scale)
+        parity.check_scores(sc, want_s, A)
+
+
+def test_llama8b_shaped_decode_full_size():
+    _full_size(W.LLAMA8B_DECODE, [(0, 0), (3, 13), (7, 31)])
+
+
+def test_long_context_kv_quantized_full_size():
+    _full_size(W.LONG_CONTEXT, [(0, 1), (5, 22), (7, 31)])
+
+
+@pytest.mark.parametrize("B,T,bits,d", [(1, 131072, 1, 64), (1, 131072, 3, 128), (64, 4096, 2, 128),
+                                        (8, 32768, 4, 64)])
+def test_sweep_rows_sampled(B, T, bits, d):
+    w = W.sweep_case(B, T, bits, d)
+    _full_size(w, [(0, 0), (B - 1, 31)])
