@@ -138,6 +138,28 @@ AXR_API axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, cons
                              void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * axr_attend_decode_static -- axr_attend_decode without a workspace argument, for callers that cannot allocate
+ * device memory (code running inside a memory pool it does not own, plugins handed only input and output pointers,
+ * decode steps that must not touch an allocator).  The paper has no counterpart: this is a deployment convenience.
+ * The split partials live in a fixed library-owned device array of axr_attend_static_scratch_bytes() bytes (4 MiB),
+ * which every GPU that loads the library holds until the process exits.  Nothing is allocated per call: no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *   Arguments, layouts and results are those of axr_attend_decode.
+ *   Sizes whose axr_attend_workspace_bytes() exceeds the fixed array return AXR_EWORKSPACE (use axr_attend_decode).
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress, with that device
+ *   current); make that first call before any stream capture.
+ *   All calls share the one array: calls that may overlap on the GPU (different streams, or different host threads
+ *   on one device) race and must be serialised by the caller.  The array keeps the last call's contents; every slot
+ *   a call reads is written by that call first, so no clearing is needed.
+ */
+AXR_API axr_status axr_attend_decode_static(const float* q, const uint8_t* kcodes, const uint16_t* knorms,
+                                            axr_vkind vkind, const void* v, const uint16_t* vnorms,
+                                            const int32_t* seq_lens, int B, int Hq, int Hkv, int T, int Tcap, int d,
+                                            int bits, const int8_t* signs, float scale, float* out, void* stream);
+/* Size in bytes of the fixed device array axr_attend_decode_static uses. */
+AXR_API size_t axr_attend_static_scratch_bytes(void);
+
+/*
  * axr_dense_decode -- the same decode step over an unquantized fp16 K/V cache (k, v [dev] [B, Hkv, Tcap, d] fp16):
  * out = softmax(scale * q . k_t) . v.  Not part of the method: the bandwidth reference the quantized path is
  * measured against.  Same workspace rule and errors as axr_attend_decode.

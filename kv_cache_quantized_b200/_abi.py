@@ -34,6 +34,8 @@ SIGNATURES = {
     "axr_dense_decode": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
     "axr_select_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "axr_select_signs": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _p, _p, _p, _sz, _p]),
+    "axr_attend_decode_static": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p]),
+    "axr_attend_static_scratch_bytes": (_sz, []),
     "axr_set_gather": (_i, [_i]),
     "axr_get_gather": (_i, []),
 }
