@@ -101,15 +101,16 @@ __device__ __forceinline__ void transform_queries(const float* __restrict__ q, c
 // ---- factored gather: byte-indexed centroid-pair table -------------------------------------------------------------
 
 // Entry e (the 2b-bit code of two consecutive coordinates, low coordinate in the low bits) holds (c[e & (L-1)],
-// c[e >> b]).  Tables of 64 or more entries are replicated REPS times, entry-major, so that lane l reads copy
-// l % REPS and a warp's 32 lookups touch every bank at most twice (the minimum for 64-bit loads).
+// c[e >> b]).  The table is replicated once per lane, entry-major with a 256-byte entry stride: lane l reads copy
+// l at byte offset e * 256 + 8 l, so a warp's 32 lookups never share a bank with a different address beyond the
+// two wavefronts a 64-bit warp load needs, and the offset of a pair is one byte permute of the packed code word
+// (entry index into byte 1, the lane's copy offset into byte 0).
 template <int BITS>
 struct PairTable {
   static constexpr int L = 1 << BITS;
   static constexpr int E = L * L;
-  static constexpr int REPS = E >= 64 ? 16 : 1;
+  static constexpr int REPS = 32;
   static constexpr int FLOATS = E * REPS * 2;
-  static constexpr int SHIFT = REPS == 16 ? 7 : 3;  // log2 bytes per entry (all copies)
 };
 
 template <int BITS>
@@ -122,10 +123,16 @@ __device__ __forceinline__ void build_pair_table(const float* __restrict__ cent,
   }
 }
 
-// Byte offset of this lane's copy of entry `field` in the pair table.
+// Byte offset of this lane's copy of pair i (coordinates 2i, 2i+1) of a packed slice.  repw = 8 * lane.
 template <int BITS>
-__device__ __forceinline__ uint32_t pair_off(uint32_t field, uint32_t rep_off) {
-  return (field << PairTable<BITS>::SHIFT) | rep_off;
+__device__ __forceinline__ uint32_t pair_addr(uint64_t bits, int i, uint32_t repw) {
+  if constexpr (BITS == 4) {
+    const uint32_t w = i < 4 ? static_cast<uint32_t>(bits) : static_cast<uint32_t>(bits >> 32);
+    return __byte_perm(w, repw, 0x5504u | (static_cast<uint32_t>(i & 3) << 4));
+  } else {
+    constexpr uint32_t MASK = (1u << (2 * BITS)) - 1u;
+    return ((static_cast<uint32_t>(bits >> (2 * BITS * i)) & MASK) << 8) | repw;
+  }
 }
 
 // The J*b bits of coordinates [J*sl, J*sl + J) of one packed row held in shared memory, as a 64-bit value.
@@ -150,14 +157,12 @@ __device__ __forceinline__ uint64_t load_slice(const uint8_t* row, int sl) {
 template <int BITS, int J, int HG>
 __device__ __forceinline__ void factored_slice(uint64_t bits, const uint8_t* tab, uint32_t rep_off,
                                                const float2 (&qp)[HG][J / 2], float (&acc)[HG]) {
-  constexpr uint32_t MASK = (1u << (2 * BITS)) - 1u;
   float2 a[HG];
 #pragma unroll
   for (int h = 0; h < HG; ++h) a[h] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < J / 2; ++i) {
-    const uint32_t field = static_cast<uint32_t>(bits >> (2 * BITS * i)) & MASK;
-    const float2 c = *reinterpret_cast<const float2*>(tab + pair_off<BITS>(field, rep_off));
+    const float2 c = *reinterpret_cast<const float2*>(tab + pair_addr<BITS>(bits, i, rep_off));
 #pragma unroll
     for (int h = 0; h < HG; ++h) a[h] = fma2(qp[h][i], c, a[h]);
   }
@@ -167,12 +172,15 @@ __device__ __forceinline__ void factored_slice(uint64_t bits, const uint8_t* tab
 
 // ---- shared-memory plan of the decode kernels ---------------------------------------------------------------------
 
-constexpr int kTT = 256;     // tokens per tile
-constexpr int kStages = 2;   // cp.async pipeline depth
+constexpr int kTT = 256;     // tokens per tile of the scorer
+constexpr int kStages = 2;   // cp.async pipeline depth of the scorer
 
+// Decode tiles are 128 tokens (one key-phase round): two stages of quantized keys and values plus the pair table
+// leave room for two blocks per SM; fp16 values take three stages and one block per SM.
 template <int D, int BITS, int G, bool VQ, bool DENSE>
 struct DecPlan {
-  static constexpr int TT = DENSE ? 128 : kTT;            // tokens per tile (fp16 keys: half, to fit two stages)
+  static constexpr int TT = 128;
+  static constexpr int NST = (!VQ && !DENSE) ? 3 : 2;     // cp.async pipeline depth
   static constexpr int L = 1 << BITS;
   static constexpr int R = D * BITS / 8;
   static constexpr int KROW = DENSE ? 2 * D : R;          // bytes per key row in the stage
@@ -192,35 +200,39 @@ struct DecPlan {
   static constexpr int REDUCE = NG * G * D;               // final cross-group sum (reuses the stages)
   // byte offsets
   static constexpr size_t OFF_STAGE = 0;
-  static constexpr size_t STAGES_BYTES = (size_t)kStages * STAGE;
+  static constexpr size_t STAGES_BYTES = (size_t)NST * STAGE;
   static constexpr size_t OFF_TAB = ((STAGES_BYTES > REDUCE * 4 ? STAGES_BYTES : REDUCE * 4) + 15) / 16 * 16;
   static constexpr size_t OFF_QS = OFF_TAB + (size_t)TAB * 4;
-  // raw scores and weights are indexed by thread (thread t owns token t of a tile), so size them by the block
-  static_assert(TT <= kDecThreads, "one thread per token of a tile");
-  static constexpr size_t OFF_SS = OFF_QS + (size_t)G * D * 4;                    // raw scores [threads][G]
-  static constexpr size_t OFF_PS = OFF_SS + (size_t)kDecThreads * G * 4;         // weights [threads][G] float2
-  static constexpr size_t OFF_RED = OFF_PS + (size_t)kDecThreads * G * 8;
+  static constexpr size_t OFF_PS = OFF_QS + (size_t)G * D * 4;          // weights [TT][G] float2
+  static constexpr size_t OFF_RED = OFF_PS + (size_t)TT * G * 8;
   static constexpr size_t OFF_CENT = OFF_RED + (size_t)kDecWarps * G * 4;
   static constexpr size_t bytes = OFF_CENT + 16 * 4;
 };
 
 // ---- the partial kernel ------------------------------------------------------------------------------------------
 //
-// Per tile of kTT tokens (double-buffered cp.async staging of key codes and values; norms prefetched to registers):
-//   key phase   -- 8 lanes per token, each lane owns D/8 coordinates and the matching row factors in registers;
-//                  a round covers 4 tokens per lane group; the 8 partial sums of a token are combined by a
-//                  select-free butterfly (lane sl processes token k ^ (sl >> 1) at step k);
-//   softmax     -- thread t owns token t: z = norm * raw score, block max per head, running max/sum update;
-//   value phase -- thread (vg, vc) accumulates coordinates [8vc, 8vc+8) over tokens vg, vg + NG, ...
+// Per tile of TT = 128 tokens (cp.async staging of key codes and values, norms prefetched to registers), each warp
+// w owns tokens [16w, 16w + 16) of the tile end to end, so the softmax state is warp-local:
+//   key phase   -- 8 lanes per token, each lane owning D/8 coordinates and the matching row factors in registers;
+//                  a lane group of 8 scores 4 tokens; the 8 partial sums of a token are combined by a select-free
+//                  butterfly (lane sl processes token k ^ (sl >> 1) at step k), after which lanes 2m, 2m+1 hold
+//                  token m of the group;
+//   softmax     -- the warp's running max per head is updated from its 16 new scores (shuffles over the warp); the
+//                  weights p (times the value norm for quantized values) go to shared memory for the warp only;
+//   value phase -- the same warp accumulates coordinates [8vc, 8vc+8) of its 16 tokens, D/8 lanes per token row.
+// The warps' (max, sum, accumulator) triples are merged once in the epilogue.
 template <int D, int BITS, int G, bool VQ, bool DENSE>
 __global__ void __launch_bounds__(kDecThreads, (VQ && G <= 4) ? 2 : 1)
 attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
   using P = DecPlan<D, BITS, G, VQ, DENSE>;
   constexpr int J = P::J, HG = P::HG, TPR = P::TPR, NG = P::NG;
+  constexpr int TT = P::TT;
+  constexpr int RPW = kWarp / TPR;          // value rows a warp reads at once
+  constexpr int WT = 16;                    // tokens per warp per tile
+  static_assert(TT == kDecWarps * WT, "each warp owns 16 tokens of a tile");
   extern __shared__ __align__(16) uint8_t smem[];
   float* tab = reinterpret_cast<float*>(smem + P::OFF_TAB);
   float* qs = reinterpret_cast<float*>(smem + P::OFF_QS);
-  float* ss = reinterpret_cast<float*>(smem + P::OFF_SS);
   float2* ps = reinterpret_cast<float2*>(smem + P::OFF_PS);
   float* red = reinterpret_cast<float*>(smem + P::OFF_RED);
   float* cent = reinterpret_cast<float*>(smem + P::OFF_CENT);
@@ -230,7 +242,6 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
   const int len = row_len(a, b);
   const int start = split * a.chunk;
   const int end = min(start + a.chunk, len);
-  constexpr int TT = P::TT;
   const int ntiles = end > start ? (end - start + TT - 1) / TT : 0;
   const size_t kv_row0 = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
   const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
@@ -239,7 +250,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
 
   auto issue_tile = [&](int tile) {
     if (tile < ntiles) {
-      uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % kStages) * P::STAGE;
+      uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % P::NST) * P::STAGE;
       const int t0 = start + tile * TT;
       const int n = min(TT, end - t0);
       block_copy_async<P::KCH>(st, ksrc + (kv_row0 + t0) * P::KROW, n * P::KROW);
@@ -249,7 +260,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
   };
 
   // prologue: start the copies, then build the per-block tables while they fly
-  for (int s = 0; s < kStages - 1; ++s) issue_tile(s);
+  for (int s = 0; s < P::NST - 1; ++s) issue_tile(s);
   if (tid < 16) cent[tid] = a.cb.c[tid];
   if constexpr (DENSE) {
     for (int e = tid; e < G * D; e += kDecThreads) qs[e] = qg[e] * a.mult;  // fp16 keys: untransformed query
@@ -259,18 +270,13 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
   __syncthreads();
   if constexpr (!DENSE) build_pair_table<BITS>(cent, tab);
 
-  // norms of the first tile (thread t owns token t of a tile)
-  float kn_next = 0.f, vn_next = 0.f;
-  if (ntiles > 0 && start + tid < end) {
-    kn_next = DENSE ? 1.f : __half2float(a.knorms[kv_row0 + start + tid]);
-    if constexpr (VQ) vn_next = __half2float(a.vnorms[kv_row0 + start + tid]);
-  }
-
-  // key-phase lane roles
-  const int sl = tid & 7;              // slice of coordinates [J*sl, J*sl + J)
-  const int grp = tid >> 3;            // 32 groups of 8 lanes
-  const int kord = sl >> 1;            // token order xor for the butterfly
-  const uint32_t rep_off = PairTable<BITS>::REPS == 16 ? static_cast<uint32_t>(lane & 15) << 3 : 0u;
+  // key-phase lane roles: the token this lane's pair holds after the butterfly is fixed for every tile
+  const int sl = tid & 7;                            // slice of coordinates [J*sl, J*sl + J)
+  const int kord = sl >> 1;                          // token order xor for the butterfly
+  const int tk = warp * WT + ((tid >> 3) & 3) * 4;   // first token of this lane group
+  const int my_t = tk + kord;                        // token held after the butterfly
+  const bool writer_lo = (sl & 1) == 0;              // the pair's even lane writes heads [0, G/2)
+  const uint32_t rep_off = static_cast<uint32_t>(lane) << 3;
   float2 qp[HG][J / 2];
   if constexpr (P::PASSES == 1) {
 #pragma unroll
@@ -279,132 +285,135 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
       for (int i = 0; i < J / 2; ++i) qp[h][i] = make_float2(qs[h * D + J * sl + 2 * i], qs[h * D + J * sl + 2 * i + 1]);
   }
 
-  // value-phase roles and state
-  const int vg = tid / TPR, vc = tid % TPR;
+  // norms of my token in the first tile
+  float kn_next = 1.f, vn_next = 1.f;
+  if (ntiles > 0 && start + my_t < end) {
+    if constexpr (!DENSE) kn_next = __half2float(a.knorms[kv_row0 + start + my_t]);
+    if constexpr (VQ) vn_next = __half2float(a.vnorms[kv_row0 + start + my_t]);
+  }
+
+  // value-phase roles and state (warp-local)
+  const int vrow = lane / TPR, vc = lane % TPR;
   float2 acc[G][4];
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int c = 0; c < 4; ++c) acc[g][c] = make_float2(0.f, 0.f);
-  float m_run[G], l_run[G];
+  float m_run[G], l_lane[G];
 #pragma unroll
-  for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_run[g] = 0.f; }
+  for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_lane[g] = 0.f; }
 
   for (int tile = 0; tile < ntiles; ++tile) {
     const int t0 = start + tile * TT;
     const int nt = min(TT, end - t0);
-    cp_async_wait<kStages - 2>();
-    __syncthreads();  // S1: this tile's stage is complete, and every thread is done with the previous tile
-    issue_tile(tile + kStages - 1);  // refills the stage the previous tile used
-    const uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % kStages) * P::STAGE;
+    cp_async_wait<P::NST - 2>();
+    __syncthreads();  // this tile's stage is complete, and every thread is done with the previous tile
+    issue_tile(tile + P::NST - 1);  // refills the stage the previous tile used
+    const uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % P::NST) * P::STAGE;
     const float kn_cur = kn_next, vn_cur = vn_next;
-    {
-      const int tn = t0 + TT + tid;  // prefetch the next tile's norms
-      if (tile + 1 < ntiles && tn < end) {
-        kn_next = DENSE ? 1.f : __half2float(a.knorms[kv_row0 + tn]);
-        if constexpr (VQ) vn_next = __half2float(a.vnorms[kv_row0 + tn]);
-      }
+    if (tile + 1 < ntiles && t0 + TT + my_t < end) {  // prefetch my token's norms of the next tile
+      if constexpr (!DENSE) kn_next = __half2float(a.knorms[kv_row0 + t0 + TT + my_t]);
+      if constexpr (VQ) vn_next = __half2float(a.vnorms[kv_row0 + t0 + TT + my_t]);
     }
 
-    // ---- key phase: raw scores into ss[token][g] ----
-#pragma unroll 1
-    for (int round = 0; round < TT / 128; ++round) {
-      const int tbase = round * 128 + grp * 4;
-#pragma unroll
-      for (int pass = 0; pass < P::PASSES; ++pass) {
-        if constexpr (P::PASSES > 1) {
-#pragma unroll
-          for (int h = 0; h < HG; ++h)
-#pragma unroll
-            for (int i = 0; i < J / 2; ++i) {
-              const float* qrow = qs + (pass * HG + h) * D + J * sl + 2 * i;
-              qp[h][i] = make_float2(qrow[0], qrow[1]);
-            }
-        }
-        float v[4][HG];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int tt = tbase + (k ^ kord);
-          if constexpr (DENSE) {
-            // fp16 key slice: J halves at byte offset 2*J*sl
-            const __half2* kh = reinterpret_cast<const __half2*>(st + tt * P::KROW + 2 * J * sl);
-            float2 s2[HG];
-#pragma unroll
-            for (int h = 0; h < HG; ++h) s2[h] = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < J / 2; ++i) {
-              const float2 kf = __half22float2(kh[i]);
-#pragma unroll
-              for (int h = 0; h < HG; ++h) s2[h] = fma2(qp[h][i], kf, s2[h]);
-            }
-#pragma unroll
-            for (int h = 0; h < HG; ++h) v[k][h] = s2[h].x + s2[h].y;
-          } else {
-            const uint64_t bits = load_slice<D, BITS, J>(st + tt * P::KROW, sl);
-            factored_slice<BITS, J, HG>(bits, reinterpret_cast<const uint8_t*>(tab), rep_off, qp, v[k]);
-          }
-        }
-        // butterfly over the 8 lanes of the group: 4 tokens -> lane pair (2m, 2m+1) holds token m
-#pragma unroll
-        for (int h = 0; h < HG; ++h) {
-          v[0][h] += __shfl_xor_sync(0xffffffffu, v[2][h], 4);
-          v[1][h] += __shfl_xor_sync(0xffffffffu, v[3][h], 4);
-          v[0][h] += __shfl_xor_sync(0xffffffffu, v[1][h], 2);
-          v[0][h] += __shfl_xor_sync(0xffffffffu, v[0][h], 1);
-        }
-        if ((sl & 1) == 0) {
-          const int tt = tbase + kord;
-#pragma unroll
-          for (int h = 0; h < HG; ++h) ss[tt * G + pass * HG + h] = v[0][h];
-        }
-      }
-    }
-    __syncthreads();  // S2: raw scores complete
-
-    // ---- softmax: thread tid owns token tid of the tile ----
+    // ---- key phase ----
     float z[G];
 #pragma unroll
-    for (int g = 0; g < G; ++g) z[g] = tid < nt ? ss[tid * G + g] * kn_cur : -INFINITY;
+    for (int pass = 0; pass < P::PASSES; ++pass) {
+      if constexpr (P::PASSES > 1) {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float mx = warp_max(z[g]);
-      if (lane == 0) red[warp * G + g] = mx;
+        for (int h = 0; h < HG; ++h)
+#pragma unroll
+          for (int i = 0; i < J / 2; ++i) {
+            const float* qrow = qs + (pass * HG + h) * D + J * sl + 2 * i;
+            qp[h][i] = make_float2(qrow[0], qrow[1]);
+          }
+      }
+      float v[4][HG];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int tt = tk + (k ^ kord);
+        if constexpr (DENSE) {
+          const __half2* kh = reinterpret_cast<const __half2*>(st + tt * P::KROW + 2 * J * sl);
+          float2 s2[HG];
+#pragma unroll
+          for (int h = 0; h < HG; ++h) s2[h] = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < J / 2; ++i) {
+            const float2 kf = __half22float2(kh[i]);
+#pragma unroll
+            for (int h = 0; h < HG; ++h) s2[h] = fma2(qp[h][i], kf, s2[h]);
+          }
+#pragma unroll
+          for (int h = 0; h < HG; ++h) v[k][h] = s2[h].x + s2[h].y;
+        } else {
+          const uint64_t bits = load_slice<D, BITS, J>(st + tt * P::KROW, sl);
+          factored_slice<BITS, J, HG>(bits, reinterpret_cast<const uint8_t*>(tab), rep_off, qp, v[k]);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        v[0][h] += __shfl_xor_sync(0xffffffffu, v[2][h], 4);
+        v[1][h] += __shfl_xor_sync(0xffffffffu, v[3][h], 4);
+        v[0][h] += __shfl_xor_sync(0xffffffffu, v[1][h], 2);
+        v[0][h] += __shfl_xor_sync(0xffffffffu, v[0][h], 1);
+        z[pass * HG + h] = v[0][h];
+      }
     }
-    __syncthreads();  // S3
-    const float vscale = VQ ? vn_cur : 1.f;
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float mt = red[g];
-#pragma unroll
-      for (int w2 = 1; w2 < kDecWarps; ++w2) mt = fmaxf(mt, red[w2 * G + g]);
-      const float m_new = fmaxf(m_run[g], mt);
-      const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run[g] - m_new);
-      const float p = (z[g] == -INFINITY) ? 0.f : exp2f(z[g] - m_new);
-      l_run[g] = l_run[g] * alpha + p;
-      const float pv = p * vscale;
-      ps[tid * G + g] = make_float2(pv, pv);
-#pragma unroll
-      for (int c = 0; c < 4; ++c) { acc[g][c].x *= alpha; acc[g][c].y *= alpha; }
-      m_run[g] = m_new;
-    }
-    __syncthreads();  // S4: weights complete
 
-    // ---- value phase ----
+    // ---- warp-local online softmax over this warp's 16 tokens ----
+    const bool valid = my_t < nt;
+    bool grew = false;
+    float alpha[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      z[g] = valid ? z[g] * kn_cur : -INFINITY;
+      float mx = z[g];
+#pragma unroll
+      for (int msk = 2; msk < 32; msk <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, msk));
+      const float m_new = fmaxf(m_run[g], mx);
+      alpha[g] = (m_new == -INFINITY) ? 1.f : exp2f(m_run[g] - m_new);
+      const float p = valid ? exp2f(z[g] - m_new) : 0.f;
+      l_lane[g] = l_lane[g] * alpha[g] + (writer_lo ? p : 0.f);
+      grew |= m_new != m_run[g];
+      m_run[g] = m_new;
+      z[g] = p * (VQ ? vn_cur : 1.f);
+    }
+    {
+      float2* row = ps + static_cast<size_t>(my_t) * G;
+      constexpr int HALF = G > 1 ? G / 2 : 1;
+      if (G > 1 || writer_lo) {
+#pragma unroll
+        for (int h = 0; h < HALF; ++h) {
+          const int g = (writer_lo ? 0 : HALF) + h;
+          row[g] = make_float2(z[g], z[g]);
+        }
+      }
+    }
+    if (grew) {  // warp-uniform
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) { acc[g][c].x *= alpha[g]; acc[g][c].y *= alpha[g]; }
+    }
+    __syncwarp();
+
+    // ---- value phase: this warp's 16 tokens ----
     const uint8_t* vst = st + P::STAGE_K;
-    for (int tt = vg; tt < nt; tt += NG) {
+#pragma unroll 2
+    for (int i = 0; i < WT / RPW; ++i) {
+      const int tt = warp * WT + vrow + RPW * i;
+      if (tt >= nt) break;
       float2 pw[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) pw[g] = ps[tt * G + g];
       float2 val[4];
       if constexpr (VQ) {
         const uint64_t bits = load_slice<D, BITS, 8>(vst + tt * P::VROW, vc);
-        constexpr uint32_t MASK = (1u << (2 * BITS)) - 1u;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t field = static_cast<uint32_t>(bits >> (2 * BITS * i)) & MASK;
-          val[i] = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(tab) +
-                                                    pair_off<BITS>(field, rep_off));
-        }
+        for (int c = 0; c < 4; ++c)
+          val[c] = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(tab) +
+                                                    pair_addr<BITS>(bits, c, rep_off));
       } else {
         const uint4 u = *reinterpret_cast<const uint4*>(vst + tt * P::VROW + 16 * vc);
         val[0] = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
@@ -419,20 +428,38 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
     }
   }
   cp_async_wait<0>();
-  __syncthreads();  // every stage is idle: reuse it for the cross-group sum
+  __syncthreads();  // every stage is idle: reuse it for the cross-warp merge
 
-  // ---- epilogue ----
+  // ---- epilogue: merge the warps' (max, sum, accumulator) ----
   float* region = reinterpret_cast<float*>(smem + P::OFF_STAGE);
+  if (lane == 0) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) red[warp * G + g] = m_run[g];
+  }
+  __syncthreads();
+  float scl[G], Mblk[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
-    const float s = warp_sum(l_run[g]);
-    if (lane == 0) red[warp * G + g] = s;
+    float M = red[g];
+#pragma unroll
+    for (int w2 = 1; w2 < kDecWarps; ++w2) M = fmaxf(M, red[w2 * G + g]);
+    scl[g] = (m_run[g] == -INFINITY) ? 0.f : exp2f(m_run[g] - M);
+    const float l = warp_sum(l_lane[g]) * scl[g];
+    l_lane[g] = l;  // this warp's rescaled sum (uniform over the warp)
+    Mblk[g] = M;
   }
+  __syncthreads();  // red is rewritten below
+  if (lane == 0) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) red[warp * G + g] = l_lane[g];
+  }
+  const int vg = warp * RPW + vrow;  // value group: one per (warp, row slot)
 #pragma unroll
   for (int g = 0; g < G; ++g)
 #pragma unroll
     for (int c = 0; c < 4; ++c)
-      *reinterpret_cast<float2*>(region + (vg * G + g) * D + vc * 8 + 2 * c) = acc[g][c];
+      *reinterpret_cast<float2*>(region + (vg * G + g) * D + vc * 8 + 2 * c) =
+          make_float2(acc[g][c].x * scl[g], acc[g][c].y * scl[g]);
   __syncthreads();
   const size_t part0 = (static_cast<size_t>(b) * a.Hq + hk * G) * a.splits + split;  // head g adds g * splits
   for (int e = tid; e < G * D; e += kDecThreads) {
@@ -446,10 +473,10 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
     float s = 0.f;
 #pragma unroll
     for (int w2 = 0; w2 < kDecWarps; ++w2) s += red[w2 * G + tid];
-    float mv = m_run[0];  // uniform across the block; pick head tid without dynamic register indexing
+    float mv = Mblk[0];  // the block max (uniform); pick head tid without dynamic register indexing
 #pragma unroll
     for (int g = 1; g < G; ++g)
-      if (g == tid) mv = m_run[g];
+      if (g == tid) mv = Mblk[g];
     a.ws_l[part0 + static_cast<size_t>(tid) * a.splits] = s;
     a.ws_m[part0 + static_cast<size_t>(tid) * a.splits] = mv;
   }
@@ -626,27 +653,49 @@ __global__ void __launch_bounds__(kDecThreads) score_kernel(const __grid_constan
   } else {
     build_pair_table<BITS>(cent, tab);
     const int sl = tid & 7, grp = tid >> 3, kord = sl >> 1;
-    const uint32_t rep_off = PairTable<BITS>::REPS == 16 ? static_cast<uint32_t>(lane & 15) << 3 : 0u;
+    const uint32_t rep_off = static_cast<uint32_t>(lane) << 3;
     float2 qp[HG][J / 2];
+    if constexpr (P::PASSES == 1) {
+#pragma unroll
+      for (int h = 0; h < HG; ++h)
+#pragma unroll
+        for (int i = 0; i < J / 2; ++i) qp[h][i] = make_float2(qs[h * D + J * sl + 2 * i], qs[h * D + J * sl + 2 * i + 1]);
+    }
+    constexpr int ROUNDS = kTT / 128;
+    float kn_next[ROUNDS];
+#pragma unroll
+    for (int r = 0; r < ROUNDS; ++r) {
+      const int t = start + r * 128 + grp * 4 + kord;
+      kn_next[r] = (ntiles > 0 && t < vend) ? __half2float(a.knorms[kv_row0 + t]) : 0.f;
+    }
     for (int tile = 0; tile < ntiles; ++tile) {
       const int t0 = start + tile * kTT;
       const int nt = min(kTT, vend - t0);
       cp_async_wait<kStages - 2>();
       __syncthreads();  // tile complete; previous tile's stage free
       issue_tile(tile + kStages - 1);
+      float kn_cur[ROUNDS];
+#pragma unroll
+      for (int r = 0; r < ROUNDS; ++r) {
+        kn_cur[r] = kn_next[r];
+        const int t = t0 + kTT + r * 128 + grp * 4 + kord;  // my token of the next tile
+        if (tile + 1 < ntiles && t < vend) kn_next[r] = __half2float(a.knorms[kv_row0 + t]);
+      }
       const uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % kStages) * P::STAGE;
-#pragma unroll 1
-      for (int round = 0; round < kTT / 128; ++round) {
+#pragma unroll
+      for (int round = 0; round < ROUNDS; ++round) {
         const int tbase = round * 128 + grp * 4;
 #pragma unroll
         for (int pass = 0; pass < P::PASSES; ++pass) {
+          if constexpr (P::PASSES > 1) {
 #pragma unroll
-          for (int h = 0; h < HG; ++h)
+            for (int h = 0; h < HG; ++h)
 #pragma unroll
-            for (int i = 0; i < J / 2; ++i) {
-              const float* qrow = qs + (pass * HG + h) * D + J * sl + 2 * i;
-              qp[h][i] = make_float2(qrow[0], qrow[1]);
-            }
+              for (int i = 0; i < J / 2; ++i) {
+                const float* qrow = qs + (pass * HG + h) * D + J * sl + 2 * i;
+                qp[h][i] = make_float2(qrow[0], qrow[1]);
+              }
+          }
           float v[4][HG];
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -662,7 +711,7 @@ __global__ void __launch_bounds__(kDecThreads) score_kernel(const __grid_constan
           }
           const int tt = tbase + kord;
           if (tt < nt) {
-            const float n = __half2float(a.knorms[kv_row0 + t0 + tt]);
+            const float n = kn_cur[round];
             // lanes 2m and 2m+1 hold the same sums; each writes half of the heads
 #pragma unroll
             for (int h = 0; h < HG; ++h)
