@@ -28,24 +28,34 @@ struct SplitPlan {
   int chunk;  // tokens per split, a multiple of kTile
 };
 
-constexpr int kTile = 256;          // tokens scored per block iteration
+constexpr int kTile = 128;          // tokens per decode tile; chunks are whole tiles
 constexpr int kSmCount = 148;       // B200
-constexpr int kBlocksPerSm = 2;     // resident decode blocks per SM the plan aims to fill twice over
-constexpr int kMinChunk = 1024;     // keep the per-block table build amortised
+constexpr int kResident = 2 * kSmCount;  // decode blocks resident at once (two per SM)
+constexpr int kMinTiles = 4;        // smallest chunk, in tiles, so per-item setup stays amortised
 
+// Choose the split count that minimises the makespan of the persistent decode kernel: the items (one per batch row,
+// KV head and split) are dealt round-robin to kResident blocks, so the time is about ceil(items / kResident) chunks
+// plus a small per-item setup.
 inline SplitPlan plan_splits(int B, int Hkv, int T) {
   SplitPlan p{1, kTile};
   if (T <= 0 || B <= 0 || Hkv <= 0) return p;
   const long units = static_cast<long>(B) * Hkv;
-  const long target = 2L * kSmCount * kBlocksPerSm;
-  long s = (target + units - 1) / units;
-  const long max_s = (T + kMinChunk - 1) / kMinChunk;
-  if (s > max_s) s = max_s;
-  if (s < 1) s = 1;
-  long chunk = (T + s - 1) / s;
-  chunk = (chunk + kTile - 1) / kTile * kTile;
-  p.chunk = static_cast<int>(chunk);
-  p.splits = static_cast<int>((T + chunk - 1) / chunk);
+  const long tiles_total = (T + kTile - 1) / kTile;
+  long max_s = tiles_total / kMinTiles;
+  if (max_s < 1) max_s = 1;
+  if (max_s > 4096) max_s = 4096;
+  double best = 1e300;
+  for (long s = 1; s <= max_s; ++s) {
+    const long tiles = (tiles_total + s - 1) / s;
+    const long splits = (tiles_total + tiles - 1) / tiles;
+    const long rounds = (units * splits + kResident - 1) / kResident;
+    const double cost = static_cast<double>(rounds) * (static_cast<double>(tiles) + 0.5);
+    if (cost < best - 1e-9) {
+      best = cost;
+      p.chunk = static_cast<int>(tiles * kTile);
+      p.splits = static_cast<int>(splits);
+    }
+  }
   return p;
 }
 

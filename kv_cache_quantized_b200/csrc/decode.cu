@@ -35,7 +35,9 @@ axr_status launch_attend(const DecodeArgs& a, cudaStream_t st, const char* what)
   auto k1 = attend_partial_kernel<D, BITS, G, VQ, DENSE>;
   axr_status rs = ensure_smem(k1, S::bytes, what);
   if (rs != AXR_OK) return rs;
-  dim3 grid(a.splits, a.Hkv, a.B);
+  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent blocks loop over the items
+  const long resident = static_cast<long>(S::MIN_BLOCKS) * kSmCount;
+  const unsigned grid = static_cast<unsigned>(items < resident ? items : resident);
   k1<<<grid, kDecThreads, S::bytes, st>>>(a);
   attend_reduce_kernel<D, VQ><<<a.B * a.Hq, D, 0, st>>>(a);
   return check_launch(what);

@@ -170,315 +170,370 @@ __device__ __forceinline__ void factored_slice(uint64_t bits, const uint8_t* tab
   for (int h = 0; h < HG; ++h) acc[h] = a[h].x + a[h].y;
 }
 
-// ---- shared-memory plan of the decode kernels ---------------------------------------------------------------------
+// ---- the decode partial kernel: persistent and warp-specialised ---------------------------------------------------
+//
+// A block of 256 threads runs as two roles, one tile of TT = 128 tokens apart, with one block barrier per tile:
+//   scoring warps 0..3 -- hold the query row factors in registers and score the tile's tokens (8 lanes per token,
+//                         each lane owning D/8 coordinates; a lane group of 8 scores 4 tokens per round and combines
+//                         its partial sums with a select-free butterfly: lane sl processes token k ^ (sl >> 1) at step
+//                         k, after which lanes 2m, 2m+1 hold token m); scoring warp w owns tokens [32w, 32w + 32) of
+//                         every tile and keeps the running max and sum of its tokens (online softmax); it writes the
+//                         weights p (times the value norm for quantized values) and its rescale factor to shared
+//                         memory;
+//   value warps 4..7   -- hold the value accumulators and consume the previous tile: value warp 4 + w accumulates the
+//                         tokens of scoring warp w against the same running max, D/8 lanes per token row.
+// Keeping the two register sets in different warps is what lets each role run without spilling.  The roles never
+// wait on each other except at the shared per-tile barrier (bar.sync 1 with all 256 threads, which both roles execute
+// the same number of times).  Blocks are persistent: each loops over (batch, KV head, split) items, and builds the
+// pair table once.
 
 constexpr int kTT = 256;     // tokens per tile of the scorer
 constexpr int kStages = 2;   // cp.async pipeline depth of the scorer
 
-// Decode tiles are 128 tokens (one key-phase round): two stages of quantized keys and values plus the pair table
-// leave room for two blocks per SM; fp16 values take three stages and one block per SM.
 template <int D, int BITS, int G, bool VQ, bool DENSE>
 struct DecPlan {
-  static constexpr int TT = 128;
-  static constexpr int NST = (!VQ && !DENSE) ? 3 : 2;     // cp.async pipeline depth
+  static constexpr int TT = 128;                          // tokens per tile
+  static constexpr int KW = 4;                            // scoring warps; value warps follow them
+  static constexpr int RT = 128;                          // role threads
+  static constexpr int WT = TT / KW;                      // tokens per scoring warp per tile
   static constexpr int L = 1 << BITS;
   static constexpr int R = D * BITS / 8;
-  static constexpr int KROW = DENSE ? 2 * D : R;          // bytes per key row in the stage
+  static constexpr int KROW = DENSE ? 2 * D : R;          // bytes per key row
   static constexpr int VROW = VQ ? R : 2 * D;             // bytes per value row
-  static constexpr int KCH = (KROW % 16 == 0) ? 16 : 8;   // cp.async chunk for key rows
+  static constexpr int KCH = (KROW % 16 == 0) ? 16 : 8;   // cp.async chunk sizes
   static constexpr int VCH = (VROW % 16 == 0) ? 16 : 8;
   static constexpr int STAGE_K = TT * KROW;
   static constexpr int STAGE_V = TT * VROW;
-  static constexpr int STAGE = STAGE_K + STAGE_V;
-  static constexpr int LPT = 8;                           // key-phase lanes per token
-  static constexpr int J = D / LPT;                       // coordinates per lane
-  static constexpr int HG = G < 4 ? G : 4;                // heads per key-phase pass
+  static constexpr int J = D / 8;                         // key coordinates per lane
+  static constexpr int HG = G < 4 ? G : 4;                // heads per scoring pass
   static constexpr int PASSES = G / HG;
-  static constexpr int TPR = D / 8;                       // value-phase threads per token row (8 coordinates each)
-  static constexpr int NG = kDecThreads / TPR;            // value-phase token groups
+  static constexpr int TPR = D / 8;                       // value lanes per token row (8 coordinates each)
+  static constexpr int RPW = kWarp / TPR;                 // value rows per warp step
+  static constexpr int NVG = KW * RPW;                    // value lane groups, summed at the end
   static constexpr int TAB = DENSE ? 0 : PairTable<BITS>::FLOATS;
-  static constexpr int REDUCE = NG * G * D;               // final cross-group sum (reuses the stages)
-  // byte offsets
-  static constexpr size_t OFF_STAGE = 0;
-  static constexpr size_t STAGES_BYTES = (size_t)NST * STAGE;
-  static constexpr size_t OFF_TAB = ((STAGES_BYTES > REDUCE * 4 ? STAGES_BYTES : REDUCE * 4) + 15) / 16 * 16;
-  static constexpr size_t OFF_QS = OFF_TAB + (size_t)TAB * 4;
-  static constexpr size_t OFF_PS = OFF_QS + (size_t)G * D * 4;          // weights [TT][G] float2
-  static constexpr size_t OFF_RED = OFF_PS + (size_t)TT * G * 8;
-  static constexpr size_t OFF_CENT = OFF_RED + (size_t)kDecWarps * G * 4;
+  static constexpr size_t OFF_K = 0;                                         // [2][STAGE_K]
+  static constexpr size_t OFF_V = OFF_K + 2 * (size_t)STAGE_K;               // [2][STAGE_V]
+  static constexpr size_t STAGES_END = OFF_V + 2 * (size_t)STAGE_V;
+  static constexpr size_t REDUCE_BYTES = (size_t)NVG * G * D * 4;            // final sum, reuses the stages
+  static constexpr size_t OFF_TAB = ((STAGES_END > REDUCE_BYTES ? STAGES_END : REDUCE_BYTES) + 15) / 16 * 16;
+  static constexpr size_t OFF_QS = OFF_TAB + (size_t)TAB * 4;               // [G][D] row factors
+  static constexpr size_t OFF_P = OFF_QS + (size_t)G * D * 4;               // [2][TT][G] float2 weights
+  static constexpr size_t OFF_AL = OFF_P + 2 * (size_t)TT * G * 8;          // [2][KW][G] rescale factors
+  static constexpr size_t OFF_GR = OFF_AL + 2 * (size_t)KW * G * 4;         // [2][KW] rescale flags
+  static constexpr size_t OFF_RM = OFF_GR + 2 * (size_t)KW * 4;             // [KW][G] running max
+  static constexpr size_t OFF_RL = OFF_RM + (size_t)KW * G * 4;             // [KW][G] running sum
+  static constexpr size_t OFF_CENT = OFF_RL + (size_t)KW * G * 4;
   static constexpr size_t bytes = OFF_CENT + 16 * 4;
+  static constexpr int MIN_BLOCKS = bytes <= 110 * 1024 ? 2 : 1;
 };
 
-// ---- the partial kernel ------------------------------------------------------------------------------------------
-//
-// Per tile of TT = 128 tokens (cp.async staging of key codes and values, norms prefetched to registers), each warp
-// w owns tokens [16w, 16w + 16) of the tile end to end, so the softmax state is warp-local:
-//   key phase   -- 8 lanes per token, each lane owning D/8 coordinates and the matching row factors in registers;
-//                  a lane group of 8 scores 4 tokens; the 8 partial sums of a token are combined by a select-free
-//                  butterfly (lane sl processes token k ^ (sl >> 1) at step k), after which lanes 2m, 2m+1 hold
-//                  token m of the group;
-//   softmax     -- the warp's running max per head is updated from its 16 new scores (shuffles over the warp); the
-//                  weights p (times the value norm for quantized values) go to shared memory for the warp only;
-//   value phase -- the same warp accumulates coordinates [8vc, 8vc+8) of its 16 tokens, D/8 lanes per token row.
-// The warps' (max, sum, accumulator) triples are merged once in the epilogue.
+__device__ __forceinline__ void roles_sync() { asm volatile("bar.sync 1, 256;\n" ::: "memory"); }
+
+// Copy `bytes` (a multiple of CH) from global to shared with the 128 threads of one role.
+template <int CH>
+__device__ __forceinline__ void role_copy_async(uint8_t* dst, const uint8_t* src, int bytes, int rtid) {
+  for (int o = rtid * CH; o < bytes; o += 128 * CH) cp_async<CH>(dst + o, src + o);
+}
+
 template <int D, int BITS, int G, bool VQ, bool DENSE>
-__global__ void __launch_bounds__(kDecThreads, (VQ && G <= 4) ? 2 : 1)
+__global__ void __launch_bounds__(kDecThreads, DecPlan<D, BITS, G, VQ, DENSE>::MIN_BLOCKS)
 attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
   using P = DecPlan<D, BITS, G, VQ, DENSE>;
-  constexpr int J = P::J, HG = P::HG, TPR = P::TPR, NG = P::NG;
-  constexpr int TT = P::TT;
-  constexpr int RPW = kWarp / TPR;          // value rows a warp reads at once
-  constexpr int WT = 16;                    // tokens per warp per tile
-  static_assert(TT == kDecWarps * WT, "each warp owns 16 tokens of a tile");
+  constexpr int J = P::J, HG = P::HG, TT = P::TT, WT = P::WT, KW = P::KW, RPW = P::RPW, TPR = P::TPR;
   extern __shared__ __align__(16) uint8_t smem[];
   float* tab = reinterpret_cast<float*>(smem + P::OFF_TAB);
   float* qs = reinterpret_cast<float*>(smem + P::OFF_QS);
-  float2* ps = reinterpret_cast<float2*>(smem + P::OFF_PS);
-  float* red = reinterpret_cast<float*>(smem + P::OFF_RED);
+  float2* pbuf = reinterpret_cast<float2*>(smem + P::OFF_P);
+  float* alpha_s = reinterpret_cast<float*>(smem + P::OFF_AL);
+  int* grew_s = reinterpret_cast<int*>(smem + P::OFF_GR);
+  float* red_m = reinterpret_cast<float*>(smem + P::OFF_RM);
+  float* red_l = reinterpret_cast<float*>(smem + P::OFF_RL);
   float* cent = reinterpret_cast<float*>(smem + P::OFF_CENT);
+  float* region = reinterpret_cast<float*>(smem);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = blockIdx.z, hk = blockIdx.y, split = blockIdx.x;
-  const int len = row_len(a, b);
-  const int start = split * a.chunk;
-  const int end = min(start + a.chunk, len);
-  const int ntiles = end > start ? (end - start + TT - 1) / TT : 0;
-  const size_t kv_row0 = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
-  const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
-  const uint8_t* ksrc = DENSE ? reinterpret_cast<const uint8_t*>(a.kdense) : a.kcodes;
-  const uint8_t* vsrc = static_cast<const uint8_t*>(a.v);
+  const bool scorer = warp < KW;
+  const int rtid = scorer ? tid : tid - P::RT;  // thread index within the role
 
-  auto issue_tile = [&](int tile) {
-    if (tile < ntiles) {
-      uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % P::NST) * P::STAGE;
-      const int t0 = start + tile * TT;
-      const int n = min(TT, end - t0);
-      block_copy_async<P::KCH>(st, ksrc + (kv_row0 + t0) * P::KROW, n * P::KROW);
-      block_copy_async<P::VCH>(st + P::STAGE_K, vsrc + (kv_row0 + t0) * P::VROW, n * P::VROW);
-    }
-    cp_async_commit();
-  };
-
-  // prologue: start the copies, then build the per-block tables while they fly
-  for (int s = 0; s < P::NST - 1; ++s) issue_tile(s);
   if (tid < 16) cent[tid] = a.cb.c[tid];
-  if constexpr (DENSE) {
-    for (int e = tid; e < G * D; e += kDecThreads) qs[e] = qg[e] * a.mult;  // fp16 keys: untransformed query
-  } else {
-    transform_queries<D, G>(qg, a.signs, a.mult, qs);
-  }
   __syncthreads();
   if constexpr (!DENSE) build_pair_table<BITS>(cent, tab);
 
-  // key-phase lane roles: the token this lane's pair holds after the butterfly is fixed for every tile
-  const int sl = tid & 7;                            // slice of coordinates [J*sl, J*sl + J)
-  const int kord = sl >> 1;                          // token order xor for the butterfly
-  const int tk = warp * WT + ((tid >> 3) & 3) * 4;   // first token of this lane group
-  const int my_t = tk + kord;                        // token held after the butterfly
-  const bool writer_lo = (sl & 1) == 0;              // the pair's even lane writes heads [0, G/2)
-  const uint32_t rep_off = static_cast<uint32_t>(lane) << 3;
-  float2 qp[HG][J / 2];
-  if constexpr (P::PASSES == 1) {
-#pragma unroll
-    for (int h = 0; h < HG; ++h)
-#pragma unroll
-      for (int i = 0; i < J / 2; ++i) qp[h][i] = make_float2(qs[h * D + J * sl + 2 * i], qs[h * D + J * sl + 2 * i + 1]);
-  }
+  const int items = a.B * a.Hkv * a.splits;
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    const int split = item % a.splits;
+    const int hk = (item / a.splits) % a.Hkv;
+    const int b = item / (a.splits * a.Hkv);
+    const int len = row_len(a, b);
+    const int start = split * a.chunk;
+    const int end = min(start + a.chunk, len);
+    const int ntiles = end > start ? (end - start + TT - 1) / TT : 0;
+    const size_t kv_row0 = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
+    const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
 
-  // norms of my token in the first tile
-  float kn_next = 1.f, vn_next = 1.f;
-  if (ntiles > 0 && start + my_t < end) {
-    if constexpr (!DENSE) kn_next = __half2float(a.knorms[kv_row0 + start + my_t]);
-    if constexpr (VQ) vn_next = __half2float(a.vnorms[kv_row0 + start + my_t]);
-  }
-
-  // value-phase roles and state (warp-local)
-  const int vrow = lane / TPR, vc = lane % TPR;
-  float2 acc[G][4];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[g][c] = make_float2(0.f, 0.f);
-  float m_run[G], l_lane[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_lane[g] = 0.f; }
-
-  for (int tile = 0; tile < ntiles; ++tile) {
-    const int t0 = start + tile * TT;
-    const int nt = min(TT, end - t0);
-    cp_async_wait<P::NST - 2>();
-    __syncthreads();  // this tile's stage is complete, and every thread is done with the previous tile
-    issue_tile(tile + P::NST - 1);  // refills the stage the previous tile used
-    const uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % P::NST) * P::STAGE;
-    const float kn_cur = kn_next, vn_cur = vn_next;
-    if (tile + 1 < ntiles && t0 + TT + my_t < end) {  // prefetch my token's norms of the next tile
-      if constexpr (!DENSE) kn_next = __half2float(a.knorms[kv_row0 + t0 + TT + my_t]);
-      if constexpr (VQ) vn_next = __half2float(a.vnorms[kv_row0 + t0 + TT + my_t]);
+    __syncthreads();  // the previous item is finished with the row factors, the stages and the merge region
+    if constexpr (DENSE) {
+      for (int e = tid; e < G * D; e += kDecThreads) qs[e] = qg[e] * a.mult;  // fp16 keys: untransformed query
+    } else {
+      transform_queries<D, G>(qg, a.signs, a.mult, qs);
     }
+    __syncthreads();
 
-    // ---- key phase ----
-    float z[G];
-#pragma unroll
-    for (int pass = 0; pass < P::PASSES; ++pass) {
-      if constexpr (P::PASSES > 1) {
+    if (scorer) {
+      // ================================= scoring role =================================
+      const int sl = tid & 7, kord = sl >> 1;
+      const int tk0 = warp * WT + ((tid >> 3) & 3) * 4;  // first token of this lane group, round 0
+      const bool writer_lo = (sl & 1) == 0;
+      const uint32_t rep_off = static_cast<uint32_t>(lane) << 3;
+      const uint8_t* ksrc = DENSE ? reinterpret_cast<const uint8_t*>(a.kdense) : a.kcodes;
+      float2 qp[HG][J / 2];
+      if constexpr (P::PASSES == 1) {
 #pragma unroll
         for (int h = 0; h < HG; ++h)
 #pragma unroll
-          for (int i = 0; i < J / 2; ++i) {
-            const float* qrow = qs + (pass * HG + h) * D + J * sl + 2 * i;
-            qp[h][i] = make_float2(qrow[0], qrow[1]);
-          }
+          for (int i = 0; i < J / 2; ++i)
+            qp[h][i] = make_float2(qs[h * D + J * sl + 2 * i], qs[h * D + J * sl + 2 * i + 1]);
       }
-      float v[4][HG];
+      float m_run[G], l_lane[G];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int tt = tk + (k ^ kord);
-        if constexpr (DENSE) {
-          const __half2* kh = reinterpret_cast<const __half2*>(st + tt * P::KROW + 2 * J * sl);
-          float2 s2[HG];
+      for (int g = 0; g < G; ++g) { m_run[g] = -INFINITY; l_lane[g] = 0.f; }
+      float kn_next[2], vn_next[2];
 #pragma unroll
-          for (int h = 0; h < HG; ++h) s2[h] = make_float2(0.f, 0.f);
+      for (int r = 0; r < 2; ++r) {
+        const int t = start + tk0 + 16 * r + kord;
+        kn_next[r] = (!DENSE && ntiles > 0 && t < end) ? __half2float(a.knorms[kv_row0 + t]) : 1.f;
+        vn_next[r] = (VQ && ntiles > 0 && t < end) ? __half2float(a.vnorms[kv_row0 + t]) : 1.f;
+      }
+      auto issue_k = [&](int tile) {
+        if (tile < ntiles) {
+          const int t0 = start + tile * TT;
+          role_copy_async<P::KCH>(smem + P::OFF_K + (tile & 1) * P::STAGE_K, ksrc + (kv_row0 + t0) * P::KROW,
+                                  min(TT, end - t0) * P::KROW, rtid);
+        }
+        cp_async_commit();
+      };
+      issue_k(0);
+      for (int it = 0; it <= ntiles; ++it) {
+        cp_async_wait<0>();
+        roles_sync();
+        issue_k(it + 1);
+        if (it == ntiles) continue;
+        const int t0 = start + it * TT;
+        const int nt = min(TT, end - t0);
+        const uint8_t* st = smem + P::OFF_K + (it & 1) * P::STAGE_K;
+        float kn_cur[2], vn_cur[2];
 #pragma unroll
-          for (int i = 0; i < J / 2; ++i) {
-            const float2 kf = __half22float2(kh[i]);
+        for (int r = 0; r < 2; ++r) {
+          kn_cur[r] = kn_next[r];
+          vn_cur[r] = vn_next[r];
+          const int t = t0 + TT + tk0 + 16 * r + kord;  // my tokens of the next tile
+          if (it + 1 < ntiles && t < end) {
+            if constexpr (!DENSE) kn_next[r] = __half2float(a.knorms[kv_row0 + t]);
+            if constexpr (VQ) vn_next[r] = __half2float(a.vnorms[kv_row0 + t]);
+          }
+        }
+        float z[2][G];
 #pragma unroll
-            for (int h = 0; h < HG; ++h) s2[h] = fma2(qp[h][i], kf, s2[h]);
+        for (int r = 0; r < 2; ++r) {
+          const int tk = tk0 + 16 * r;
+#pragma unroll
+          for (int pass = 0; pass < P::PASSES; ++pass) {
+            if constexpr (P::PASSES > 1) {
+#pragma unroll
+              for (int h = 0; h < HG; ++h)
+#pragma unroll
+                for (int i = 0; i < J / 2; ++i) {
+                  const float* qrow = qs + (pass * HG + h) * D + J * sl + 2 * i;
+                  qp[h][i] = make_float2(qrow[0], qrow[1]);
+                }
+            }
+            float v[4][HG];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int tt = tk + (k ^ kord);
+              if constexpr (DENSE) {
+                const __half2* kh = reinterpret_cast<const __half2*>(st + tt * P::KROW + 2 * J * sl);
+                float2 s2[HG];
+#pragma unroll
+                for (int h = 0; h < HG; ++h) s2[h] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < J / 2; ++i) {
+                  const float2 kf = __half22float2(kh[i]);
+#pragma unroll
+                  for (int h = 0; h < HG; ++h) s2[h] = fma2(qp[h][i], kf, s2[h]);
+                }
+#pragma unroll
+                for (int h = 0; h < HG; ++h) v[k][h] = s2[h].x + s2[h].y;
+              } else {
+                const uint64_t bits = load_slice<D, BITS, J>(st + tt * P::KROW, sl);
+                factored_slice<BITS, J, HG>(bits, reinterpret_cast<const uint8_t*>(tab), rep_off, qp, v[k]);
+              }
+            }
+#pragma unroll
+            for (int h = 0; h < HG; ++h) {
+              v[0][h] += __shfl_xor_sync(0xffffffffu, v[2][h], 4);
+              v[1][h] += __shfl_xor_sync(0xffffffffu, v[3][h], 4);
+              v[0][h] += __shfl_xor_sync(0xffffffffu, v[1][h], 2);
+              v[0][h] += __shfl_xor_sync(0xffffffffu, v[0][h], 1);
+              z[r][pass * HG + h] = v[0][h];
+            }
+          }
+        }
+        // online softmax over this warp's 32 tokens of the tile
+        bool grew = false;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float mx = -INFINITY;
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const bool valid = tk0 + 16 * r + kord < nt;
+            z[r][g] = valid ? z[r][g] * kn_cur[r] : -INFINITY;
+            mx = fmaxf(mx, z[r][g]);
           }
 #pragma unroll
-          for (int h = 0; h < HG; ++h) v[k][h] = s2[h].x + s2[h].y;
-        } else {
-          const uint64_t bits = load_slice<D, BITS, J>(st + tt * P::KROW, sl);
-          factored_slice<BITS, J, HG>(bits, reinterpret_cast<const uint8_t*>(tab), rep_off, qp, v[k]);
+          for (int msk = 2; msk < 32; msk <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, msk));
+          const float m_new = fmaxf(m_run[g], mx);
+          const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run[g] - m_new);
+          float psum = 0.f;
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            const float p = (z[r][g] == -INFINITY) ? 0.f : exp2f(z[r][g] - m_new);
+            psum += p;
+            z[r][g] = p * (VQ ? vn_cur[r] : 1.f);
+          }
+          l_lane[g] = l_lane[g] * alpha + (writer_lo ? psum : 0.f);
+          grew |= m_new != m_run[g];
+          m_run[g] = m_new;
+          if (lane == 0) alpha_s[((it & 1) * KW + warp) * G + g] = alpha;
+        }
+        if (lane == 0) grew_s[(it & 1) * KW + warp] = grew ? 1 : 0;
+        constexpr int HALF = G > 1 ? G / 2 : 1;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          float2* row = pbuf + (static_cast<size_t>(it & 1) * TT + tk0 + 16 * r + kord) * G;
+          if (G > 1 || writer_lo) {
+#pragma unroll
+            for (int h = 0; h < HALF; ++h) {
+              const int g = (writer_lo ? 0 : HALF) + h;
+              row[g] = make_float2(z[r][g], z[r][g]);
+            }
+          }
         }
       }
+      cp_async_wait<0>();
+      // merge, step 1: publish this warp's running max
+      if (lane == 0) {
 #pragma unroll
-      for (int h = 0; h < HG; ++h) {
-        v[0][h] += __shfl_xor_sync(0xffffffffu, v[2][h], 4);
-        v[1][h] += __shfl_xor_sync(0xffffffffu, v[3][h], 4);
-        v[0][h] += __shfl_xor_sync(0xffffffffu, v[1][h], 2);
-        v[0][h] += __shfl_xor_sync(0xffffffffu, v[0][h], 1);
-        z[pass * HG + h] = v[0][h];
+        for (int g = 0; g < G; ++g) red_m[warp * G + g] = m_run[g];
       }
-    }
-
-    // ---- warp-local online softmax over this warp's 16 tokens ----
-    const bool valid = my_t < nt;
-    bool grew = false;
-    float alpha[G];
+      roles_sync();
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      z[g] = valid ? z[g] * kn_cur : -INFINITY;
-      float mx = z[g];
+      for (int g = 0; g < G; ++g) {
+        float M = red_m[g];
 #pragma unroll
-      for (int msk = 2; msk < 32; msk <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, msk));
-      const float m_new = fmaxf(m_run[g], mx);
-      alpha[g] = (m_new == -INFINITY) ? 1.f : exp2f(m_run[g] - m_new);
-      const float p = valid ? exp2f(z[g] - m_new) : 0.f;
-      l_lane[g] = l_lane[g] * alpha[g] + (writer_lo ? p : 0.f);
-      grew |= m_new != m_run[g];
-      m_run[g] = m_new;
-      z[g] = p * (VQ ? vn_cur : 1.f);
-    }
-    {
-      float2* row = ps + static_cast<size_t>(my_t) * G;
-      constexpr int HALF = G > 1 ? G / 2 : 1;
-      if (G > 1 || writer_lo) {
-#pragma unroll
-        for (int h = 0; h < HALF; ++h) {
-          const int g = (writer_lo ? 0 : HALF) + h;
-          row[g] = make_float2(z[g], z[g]);
-        }
+        for (int w2 = 1; w2 < KW; ++w2) M = fmaxf(M, red_m[w2 * G + g]);
+        const float scl = (m_run[g] == -INFINITY) ? 0.f : exp2f(m_run[g] - M);
+        const float l = warp_sum(l_lane[g]) * scl;
+        if (lane == 0) red_l[warp * G + g] = l;
       }
-    }
-    if (grew) {  // warp-uniform
+    } else {
+      // ================================= value role =================================
+      const int vw = warp - KW;
+      const int vrow = lane / TPR, vc = lane % TPR;
+      const uint32_t rep_off = static_cast<uint32_t>(lane) << 3;
+      const uint8_t* vsrc = static_cast<const uint8_t*>(a.v);
+      float2 acc[G][4];
 #pragma unroll
       for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) { acc[g][c].x *= alpha[g]; acc[g][c].y *= alpha[g]; }
-    }
-    __syncwarp();
-
-    // ---- value phase: this warp's 16 tokens ----
-    const uint8_t* vst = st + P::STAGE_K;
-#pragma unroll 2
-    for (int i = 0; i < WT / RPW; ++i) {
-      const int tt = warp * WT + vrow + RPW * i;
-      if (tt >= nt) break;
-      float2 pw[G];
+        for (int c = 0; c < 4; ++c) acc[g][c] = make_float2(0.f, 0.f);
+      auto issue_v = [&](int tile) {
+        if (tile < ntiles) {
+          const int t0 = start + tile * TT;
+          role_copy_async<P::VCH>(smem + P::OFF_V + (tile & 1) * P::STAGE_V, vsrc + (kv_row0 + t0) * P::VROW,
+                                  min(TT, end - t0) * P::VROW, rtid);
+        }
+        cp_async_commit();
+      };
+      for (int it = 0; it <= ntiles; ++it) {
+        cp_async_wait<0>();
+        roles_sync();
+        issue_v(it);
+        if (it == 0) continue;
+        const int j = it - 1;  // the tile scored in the previous step
+        const int nt = min(TT, end - (start + j * TT));
+        const int pb = j & 1;
+        if (grew_s[pb * KW + vw]) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) pw[g] = ps[tt * G + g];
-      float2 val[4];
-      if constexpr (VQ) {
-        const uint64_t bits = load_slice<D, BITS, 8>(vst + tt * P::VROW, vc);
+          for (int g = 0; g < G; ++g) {
+            const float al = alpha_s[(pb * KW + vw) * G + g];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) { acc[g][c].x *= al; acc[g][c].y *= al; }
+          }
+        }
+        const uint8_t* vst = smem + P::OFF_V + pb * P::STAGE_V;
+        const float2* prow = pbuf + static_cast<size_t>(pb) * TT * G;
+#pragma unroll 2
+        for (int i = 0; i < WT / RPW; ++i) {
+          const int tt = vw * WT + vrow + RPW * i;
+          if (tt >= nt) break;
+          float2 pw[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) pw[g] = prow[tt * G + g];
+          float2 val[4];
+          if constexpr (VQ) {
+            const uint64_t bits = load_slice<D, BITS, 8>(vst + tt * P::VROW, vc);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              val[c] = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(tab) +
+                                                        pair_addr<BITS>(bits, c, rep_off));
+          } else {
+            const uint4 u = *reinterpret_cast<const uint4*>(vst + tt * P::VROW + 16 * vc);
+            val[0] = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+            val[1] = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+            val[2] = __half22float2(*reinterpret_cast<const __half2*>(&u.z));
+            val[3] = __half22float2(*reinterpret_cast<const __half2*>(&u.w));
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[g][c] = fma2(pw[g], val[c], acc[g][c]);
+        }
+      }
+      cp_async_wait<0>();
+      roles_sync();  // merge, step 1 (the scoring warps publish their running max)
+      const int vg = vw * RPW + vrow;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float M = red_m[g];
+#pragma unroll
+        for (int w2 = 1; w2 < KW; ++w2) M = fmaxf(M, red_m[w2 * G + g]);
+        const float mw = red_m[vw * G + g];
+        const float scl = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
 #pragma unroll
         for (int c = 0; c < 4; ++c)
-          val[c] = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(tab) +
-                                                    pair_addr<BITS>(bits, c, rep_off));
-      } else {
-        const uint4 u = *reinterpret_cast<const uint4*>(vst + tt * P::VROW + 16 * vc);
-        val[0] = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
-        val[1] = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
-        val[2] = __half22float2(*reinterpret_cast<const __half2*>(&u.z));
-        val[3] = __half22float2(*reinterpret_cast<const __half2*>(&u.w));
+          *reinterpret_cast<float2*>(region + (vg * G + g) * D + vc * 8 + 2 * c) =
+              make_float2(acc[g][c].x * scl, acc[g][c].y * scl);
       }
-#pragma unroll
-      for (int g = 0; g < G; ++g)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[g][c] = fma2(pw[g], val[c], acc[g][c]);
     }
-  }
-  cp_async_wait<0>();
-  __syncthreads();  // every stage is idle: reuse it for the cross-warp merge
-
-  // ---- epilogue: merge the warps' (max, sum, accumulator) ----
-  float* region = reinterpret_cast<float*>(smem + P::OFF_STAGE);
-  if (lane == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) red[warp * G + g] = m_run[g];
-  }
-  __syncthreads();
-  float scl[G], Mblk[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    float M = red[g];
-#pragma unroll
-    for (int w2 = 1; w2 < kDecWarps; ++w2) M = fmaxf(M, red[w2 * G + g]);
-    scl[g] = (m_run[g] == -INFINITY) ? 0.f : exp2f(m_run[g] - M);
-    const float l = warp_sum(l_lane[g]) * scl[g];
-    l_lane[g] = l;  // this warp's rescaled sum (uniform over the warp)
-    Mblk[g] = M;
-  }
-  __syncthreads();  // red is rewritten below
-  if (lane == 0) {
-#pragma unroll
-    for (int g = 0; g < G; ++g) red[warp * G + g] = l_lane[g];
-  }
-  const int vg = warp * RPW + vrow;  // value group: one per (warp, row slot)
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int c = 0; c < 4; ++c)
-      *reinterpret_cast<float2*>(region + (vg * G + g) * D + vc * 8 + 2 * c) =
-          make_float2(acc[g][c].x * scl[g], acc[g][c].y * scl[g]);
-  __syncthreads();
-  const size_t part0 = (static_cast<size_t>(b) * a.Hq + hk * G) * a.splits + split;  // head g adds g * splits
-  for (int e = tid; e < G * D; e += kDecThreads) {
-    const int g = e / D, j = e % D;
-    float s = 0.f;
+    __syncthreads();  // merge, step 2: every value group and every warp sum is in shared memory
+    const size_t part0 = (static_cast<size_t>(b) * a.Hq + hk * G) * a.splits + split;  // head g adds g * splits
+    for (int e = tid; e < G * D; e += kDecThreads) {
+      const int g = e / D, jj = e % D;
+      float s = 0.f;
 #pragma unroll 4
-    for (int r = 0; r < NG; ++r) s += region[(r * G + g) * D + j];
-    a.ws_o[(part0 + static_cast<size_t>(g) * a.splits) * D + j] = s;
-  }
-  if (tid < G) {
-    float s = 0.f;
+      for (int r = 0; r < P::NVG; ++r) s += region[(r * G + g) * D + jj];
+      a.ws_o[(part0 + static_cast<size_t>(g) * a.splits) * D + jj] = s;
+    }
+    if (tid < G) {
+      float M = red_m[tid], s = 0.f;
 #pragma unroll
-    for (int w2 = 0; w2 < kDecWarps; ++w2) s += red[w2 * G + tid];
-    float mv = Mblk[0];  // the block max (uniform); pick head tid without dynamic register indexing
+      for (int w2 = 1; w2 < KW; ++w2) M = fmaxf(M, red_m[w2 * G + tid]);
 #pragma unroll
-    for (int g = 1; g < G; ++g)
-      if (g == tid) mv = Mblk[g];
-    a.ws_l[part0 + static_cast<size_t>(tid) * a.splits] = s;
-    a.ws_m[part0 + static_cast<size_t>(tid) * a.splits] = mv;
+      for (int w2 = 0; w2 < KW; ++w2) s += red_l[w2 * G + tid];
+      a.ws_l[part0 + static_cast<size_t>(tid) * a.splits] = s;
+      a.ws_m[part0 + static_cast<size_t>(tid) * a.splits] = M;
+    }
   }
 }
 
