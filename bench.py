@@ -277,7 +277,7 @@ def run_axr(args, w):
     scorer = {}
     if not args.no_scorer:
         sc_out = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
-        for mode in ("factored", "table"):
+        for mode in ("tensor", "factored", "table"):
             ops.set_gather(mode)
             for _ in range(3):
                 ops.score(q, kc, kn, signs, bits, scale=1.0 / math.sqrt(d), out=sc_out)
@@ -292,7 +292,7 @@ def run_axr(args, w):
             ms = float(np.mean([a_.elapsed_time(b2) for a_, b2 in evs]))
             sbytes = (R + 2 + 4 * w.G) * B * Hkv * T
             scorer[mode] = {"ms": ms, "achieved_gbs": sbytes / (ms / 1e3) / 1e9, "algorithmic_bytes": sbytes}
-        ops.set_gather("factored")
+        ops.set_gather("tensor")
         del sc_out
 
     # max over ranks

@@ -104,16 +104,21 @@ AXR_API axr_status axr_score(const float* q, const uint8_t* kcodes, const uint16
                      float* scores, void* stream);
 
 /*
- * Table read mode of axr_score (process-wide; default AXR_GATHER_FACTORED).  Both modes compute the same table
- * entries LUT[j][k] = scale * q~_j * c_k (AXELRAM Key Points, 2nd item) and agree to fp32 rounding:
+ * Table read mode of axr_score (process-wide; default AXR_GATHER_TENSOR).  Every mode computes the same table
+ * entries LUT[j][k] = scale * q~_j * c_k (AXELRAM Key Points, 2nd item) summed at each token's indices, and they agree
+ * to within the score tolerance:
  *   AXR_GATHER_TABLE     the d x 2^b table (G heads wide) is materialised in shared memory and gathered entry by
  *                        entry, one thread per token;
  *   AXR_GATHER_FACTORED  the table is held factored -- row factor q~_j in registers, column factor c_k gathered two
  *                        coordinates at a time from a byte-indexed pair table -- and each entry is formed by the
- *                        packed FMA that accumulates it; on B200 this takes half the shared-memory wavefronts.
+ *                        packed fp32 FMA that accumulates it; half the shared-memory wavefronts of TABLE;
+ *   AXR_GATHER_TENSOR    the same factored table on the tensor cores: each token's gathered column factors (split
+ *                        into hi and lo fp16 planes, about 22 bits) form a row of an MMA operand in tensor memory,
+ *                        the row factors (split the same way) the other operand, and tcgen05.mma accumulates the
+ *                        G sums per token in fp32.
  * axr_attend_decode always reads the table in factored form.  Errors: AXR_EINVAL for an unknown mode.
  */
-typedef enum axr_gather { AXR_GATHER_FACTORED = 0, AXR_GATHER_TABLE = 1 } axr_gather;
+typedef enum axr_gather { AXR_GATHER_FACTORED = 0, AXR_GATHER_TABLE = 1, AXR_GATHER_TENSOR = 2 } axr_gather;
 AXR_API axr_status axr_set_gather(axr_gather mode);
 AXR_API axr_gather axr_get_gather(void);
 

@@ -19,6 +19,7 @@ constexpr int kMaxLevels = 16;  // b <= 4
 struct Codebook {
   float c[kMaxLevels];
   float tau[kMaxLevels];
+  float gamma[kMaxLevels];  // N(0,1)-scale centroids gamma_k = sqrt(d) * c_k, fp32
 };
 
 // ---- host-side status plumbing (defined in api.cu) ----

@@ -80,6 +80,7 @@ const Entry* entry_for(int d, int bits) {
     e.t[m - 1] = 0.0;  // exact by symmetry
     for (int k = 0; k < axr::kMaxLevels; ++k) {
       e.dev.c[k] = k < L ? static_cast<float>(e.c[k]) : 0.0f;
+      e.dev.gamma[k] = k < L ? static_cast<float>(e.c[k] * std::sqrt(static_cast<double>(d))) : 0.0f;
       // thresholds in N(0,1) units for the writer (see axr::Codebook)
       e.dev.tau[k] = k < L - 1 ? static_cast<float>(e.t[k] * std::sqrt(static_cast<double>(d))) : INFINITY;
     }

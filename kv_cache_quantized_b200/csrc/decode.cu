@@ -43,7 +43,19 @@ axr_status launch_attend(const DecodeArgs& a, cudaStream_t st, const char* what)
   return check_launch(what);
 }
 
-std::atomic<int> g_gather{kGatherFactored};
+std::atomic<int> g_gather{kGatherTensor};
+
+template <int D, int BITS, int G>
+axr_status launch_score_tc(const DecodeArgs& a, cudaStream_t st) {
+  using S = ScoreTcPlan<D, BITS, G>;
+  auto k = score_tc_kernel<D, BITS, G>;
+  axr_status rs = ensure_smem(k, S::bytes, "axr_score");
+  if (rs != AXR_OK) return rs;
+  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;
+  const long resident = 2L * kSmCount;
+  k<<<static_cast<unsigned>(items < resident ? items : resident), tc::kM, S::bytes, st>>>(a);
+  return check_launch("axr_score");
+}
 
 template <int D, int BITS, int G, int MODE>
 axr_status launch_score_mode(const DecodeArgs& a, cudaStream_t st) {
@@ -58,8 +70,10 @@ axr_status launch_score_mode(const DecodeArgs& a, cudaStream_t st) {
 
 template <int D, int BITS, int G>
 axr_status launch_score(const DecodeArgs& a, cudaStream_t st) {
-  return g_gather.load() == kGatherTable ? launch_score_mode<D, BITS, G, kGatherTable>(a, st)
-                                         : launch_score_mode<D, BITS, G, kGatherFactored>(a, st);
+  const int mode = g_gather.load();
+  if (mode == kGatherTable) return launch_score_mode<D, BITS, G, kGatherTable>(a, st);
+  if (mode == kGatherFactored) return launch_score_mode<D, BITS, G, kGatherFactored>(a, st);
+  return launch_score_tc<D, BITS, G>(a, st);
 }
 
 template <int D, int BITS>
@@ -236,12 +250,15 @@ extern "C" axr_status axr_dense_decode(const float* q, const uint16_t* k, const 
 
 extern "C" axr_status axr_set_gather(axr_gather mode) {
   using namespace axr;
-  if (mode != AXR_GATHER_FACTORED && mode != AXR_GATHER_TABLE)
-    return set_error(AXR_EINVAL, "axr_set_gather: unknown mode %d", (int)mode);
-  g_gather.store(mode == AXR_GATHER_TABLE ? kGatherTable : kGatherFactored);
+  if (mode == AXR_GATHER_FACTORED) g_gather.store(kGatherFactored);
+  else if (mode == AXR_GATHER_TABLE) g_gather.store(kGatherTable);
+  else if (mode == AXR_GATHER_TENSOR) g_gather.store(kGatherTensor);
+  else return set_error(AXR_EINVAL, "axr_set_gather: unknown mode %d", (int)mode);
   return set_error(AXR_OK, "");
 }
 
 extern "C" axr_gather axr_get_gather(void) {
-  return axr::g_gather.load() == axr::kGatherTable ? AXR_GATHER_TABLE : AXR_GATHER_FACTORED;
+  const int m = axr::g_gather.load();
+  return m == axr::kGatherTable ? AXR_GATHER_TABLE : m == axr::kGatherFactored ? AXR_GATHER_FACTORED
+                                                                                : AXR_GATHER_TENSOR;
 }

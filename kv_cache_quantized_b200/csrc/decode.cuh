@@ -18,6 +18,7 @@
 #pragma once
 
 #include "axr_host.h"
+#include "tc.cuh"
 
 namespace axr {
 
@@ -25,7 +26,7 @@ constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / kWarp;
 constexpr float kLog2e = 1.4426950408889634f;
 
-enum Gather { kGatherFactored = 0, kGatherTable = 1 };
+enum Gather { kGatherFactored = 0, kGatherTable = 1, kGatherTensor = 2 };
 
 struct DecodeArgs {
   const float* q;            // [B, Hq, D]
@@ -85,7 +86,7 @@ __device__ __forceinline__ void transform_queries(const float* __restrict__ q, c
   constexpr int VPL = WarpVec<D>::VPL;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float norm = mult * rsqrtf(static_cast<float>(D));
-  for (int g = warp; g < G; g += kDecWarps) {
+  for (int g = warp; g < G; g += blockDim.x / kWarp) {
     float v[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
@@ -105,17 +106,27 @@ __device__ __forceinline__ void transform_queries(const float* __restrict__ q, c
 // l at byte offset e * 256 + 8 l, so a warp's 32 lookups never share a bank with a different address beyond the
 // two wavefronts a 64-bit warp load needs, and the offset of a pair is one byte permute of the packed code word
 // (entry index into byte 1, the lane's copy offset into byte 0).
-template <int BITS>
+//
+// With 16 copies (REPS = 16, 128-byte entry stride) lanes l and l + 16 share a copy; they sit in different halves
+// of the warp's 64-bit request, so the request still takes its two wavefronts, at half the shared memory, but the
+// offset then needs a shift and a mask instead of one byte permute.
+template <int BITS, int REPS_ = 32>
 struct PairTable {
   static constexpr int L = 1 << BITS;
   static constexpr int E = L * L;
-  static constexpr int REPS = 32;
+  static constexpr int REPS = REPS_;
+  static constexpr int SHIFT = REPS == 32 ? 8 : 7;   // log2 of the entry stride in bytes
   static constexpr int FLOATS = E * REPS * 2;
 };
 
-template <int BITS>
+template <int BITS, int REPS = 32>
+__device__ __forceinline__ uint32_t rep_offset(int lane) {
+  return static_cast<uint32_t>(lane & (REPS - 1)) << 3;
+}
+
+template <int BITS, int REPS = 32>
 __device__ __forceinline__ void build_pair_table(const float* __restrict__ cent, float* __restrict__ tab) {
-  using P = PairTable<BITS>;
+  using P = PairTable<BITS, REPS>;
   for (int i = threadIdx.x; i < P::E * P::REPS; i += kDecThreads) {
     const int e = i / P::REPS;
     tab[2 * i] = cent[e & (P::L - 1)];
@@ -123,15 +134,15 @@ __device__ __forceinline__ void build_pair_table(const float* __restrict__ cent,
   }
 }
 
-// Byte offset of this lane's copy of pair i (coordinates 2i, 2i+1) of a packed slice.  repw = 8 * lane.
-template <int BITS>
+// Byte offset of this lane's copy of pair i (coordinates 2i, 2i+1) of a packed slice; repw = rep_offset(lane).
+template <int BITS, int REPS = 32>
 __device__ __forceinline__ uint32_t pair_addr(uint64_t bits, int i, uint32_t repw) {
-  if constexpr (BITS == 4) {
+  if constexpr (BITS == 4 && REPS == 32) {
     const uint32_t w = i < 4 ? static_cast<uint32_t>(bits) : static_cast<uint32_t>(bits >> 32);
     return __byte_perm(w, repw, 0x5504u | (static_cast<uint32_t>(i & 3) << 4));
   } else {
     constexpr uint32_t MASK = (1u << (2 * BITS)) - 1u;
-    return ((static_cast<uint32_t>(bits >> (2 * BITS * i)) & MASK) << 8) | repw;
+    return ((static_cast<uint32_t>(bits >> (2 * BITS * i)) & MASK) << PairTable<BITS, REPS>::SHIFT) | repw;
   }
 }
 
@@ -154,7 +165,7 @@ __device__ __forceinline__ uint64_t load_slice(const uint8_t* row, int sl) {
 
 // Partial dot products of one token's slice with the HG heads' row factors: acc[h] = sum over the slice's coordinate
 // pairs of (q~_{h,2i}, q~_{h,2i+1}) . (c, c') -- the packed FMA keeps even and odd coordinates in the two halves.
-template <int BITS, int J, int HG>
+template <int BITS, int J, int HG, int REPS = 32>
 __device__ __forceinline__ void factored_slice(uint64_t bits, const uint8_t* tab, uint32_t rep_off,
                                                const float2 (&qp)[HG][J / 2], float (&acc)[HG]) {
   float2 a[HG];
@@ -162,7 +173,7 @@ __device__ __forceinline__ void factored_slice(uint64_t bits, const uint8_t* tab
   for (int h = 0; h < HG; ++h) a[h] = make_float2(0.f, 0.f);
 #pragma unroll
   for (int i = 0; i < J / 2; ++i) {
-    const float2 c = *reinterpret_cast<const float2*>(tab + pair_addr<BITS>(bits, i, rep_off));
+    const float2 c = *reinterpret_cast<const float2*>(tab + pair_addr<BITS, REPS>(bits, i, rep_off));
 #pragma unroll
     for (int h = 0; h < HG; ++h) a[h] = fma2(qp[h][i], c, a[h]);
   }
@@ -187,8 +198,9 @@ __device__ __forceinline__ void factored_slice(uint64_t bits, const uint8_t* tab
 // the same number of times).  Blocks are persistent: each loops over (batch, KV head, split) items, and builds the
 // pair table once.
 
-constexpr int kTT = 256;     // tokens per tile of the scorer
-constexpr int kStages = 2;   // cp.async pipeline depth of the scorer
+constexpr int kTT = 128;     // tokens per tile of the scorer
+constexpr int kStages = 3;   // cp.async pipeline depth (two tiles in flight while one is processed)
+constexpr int kDecReps = 16; // pair-table copies in the decode kernel
 
 template <int D, int BITS, int G, bool VQ, bool DENSE>
 struct DecPlan {
@@ -210,10 +222,10 @@ struct DecPlan {
   static constexpr int TPR = D / 8;                       // value lanes per token row (8 coordinates each)
   static constexpr int RPW = kWarp / TPR;                 // value rows per warp step
   static constexpr int NVG = KW * RPW;                    // value lane groups, summed at the end
-  static constexpr int TAB = DENSE ? 0 : PairTable<BITS>::FLOATS;
-  static constexpr size_t OFF_K = 0;                                         // [2][STAGE_K]
-  static constexpr size_t OFF_V = OFF_K + 2 * (size_t)STAGE_K;               // [2][STAGE_V]
-  static constexpr size_t STAGES_END = OFF_V + 2 * (size_t)STAGE_V;
+  static constexpr int TAB = DENSE ? 0 : PairTable<BITS, kDecReps>::FLOATS;
+  static constexpr size_t OFF_K = 0;                                         // [kStages][STAGE_K]
+  static constexpr size_t OFF_V = OFF_K + kStages * (size_t)STAGE_K;         // [kStages][STAGE_V]
+  static constexpr size_t STAGES_END = OFF_V + kStages * (size_t)STAGE_V;
   static constexpr size_t REDUCE_BYTES = (size_t)NVG * G * D * 4;            // final sum, reuses the stages
   static constexpr size_t OFF_TAB = ((STAGES_END > REDUCE_BYTES ? STAGES_END : REDUCE_BYTES) + 15) / 16 * 16;
   static constexpr size_t OFF_QS = OFF_TAB + (size_t)TAB * 4;               // [G][D] row factors
@@ -257,7 +269,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
 
   if (tid < 16) cent[tid] = a.cb.c[tid];
   __syncthreads();
-  if constexpr (!DENSE) build_pair_table<BITS>(cent, tab);
+  if constexpr (!DENSE) build_pair_table<BITS, kDecReps>(cent, tab);
 
   const int items = a.B * a.Hkv * a.splits;
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
@@ -284,7 +296,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
       const int sl = tid & 7, kord = sl >> 1;
       const int tk0 = warp * WT + ((tid >> 3) & 3) * 4;  // first token of this lane group, round 0
       const bool writer_lo = (sl & 1) == 0;
-      const uint32_t rep_off = static_cast<uint32_t>(lane) << 3;
+      const uint32_t rep_off = rep_offset<BITS, kDecReps>(lane);
       const uint8_t* ksrc = DENSE ? reinterpret_cast<const uint8_t*>(a.kdense) : a.kcodes;
       float2 qp[HG][J / 2];
       if constexpr (P::PASSES == 1) {
@@ -307,20 +319,21 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
       auto issue_k = [&](int tile) {
         if (tile < ntiles) {
           const int t0 = start + tile * TT;
-          role_copy_async<P::KCH>(smem + P::OFF_K + (tile & 1) * P::STAGE_K, ksrc + (kv_row0 + t0) * P::KROW,
-                                  min(TT, end - t0) * P::KROW, rtid);
+          role_copy_async<P::KCH>(smem + P::OFF_K + (tile % kStages) * P::STAGE_K,
+                                  ksrc + (kv_row0 + t0) * P::KROW, min(TT, end - t0) * P::KROW, rtid);
         }
         cp_async_commit();
       };
       issue_k(0);
+      issue_k(1);
       for (int it = 0; it <= ntiles; ++it) {
-        cp_async_wait<0>();
+        cp_async_wait<1>();  // tile it has landed; tile it + 1 may still be in flight
         roles_sync();
-        issue_k(it + 1);
+        issue_k(it + 2);     // into the stage tile it - 1 used
         if (it == ntiles) continue;
         const int t0 = start + it * TT;
         const int nt = min(TT, end - t0);
-        const uint8_t* st = smem + P::OFF_K + (it & 1) * P::STAGE_K;
+        const uint8_t* st = smem + P::OFF_K + (it % kStages) * P::STAGE_K;
         float kn_cur[2], vn_cur[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
@@ -366,7 +379,8 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
                 for (int h = 0; h < HG; ++h) v[k][h] = s2[h].x + s2[h].y;
               } else {
                 const uint64_t bits = load_slice<D, BITS, J>(st + tt * P::KROW, sl);
-                factored_slice<BITS, J, HG>(bits, reinterpret_cast<const uint8_t*>(tab), rep_off, qp, v[k]);
+                factored_slice<BITS, J, HG, kDecReps>(bits, reinterpret_cast<const uint8_t*>(tab), rep_off, qp,
+                                                      v[k]);
               }
             }
 #pragma unroll
@@ -440,7 +454,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
       // ================================= value role =================================
       const int vw = warp - KW;
       const int vrow = lane / TPR, vc = lane % TPR;
-      const uint32_t rep_off = static_cast<uint32_t>(lane) << 3;
+      const uint32_t rep_off = rep_offset<BITS, kDecReps>(lane);
       const uint8_t* vsrc = static_cast<const uint8_t*>(a.v);
       float2 acc[G][4];
 #pragma unroll
@@ -450,15 +464,16 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
       auto issue_v = [&](int tile) {
         if (tile < ntiles) {
           const int t0 = start + tile * TT;
-          role_copy_async<P::VCH>(smem + P::OFF_V + (tile & 1) * P::STAGE_V, vsrc + (kv_row0 + t0) * P::VROW,
-                                  min(TT, end - t0) * P::VROW, rtid);
+          role_copy_async<P::VCH>(smem + P::OFF_V + (tile % kStages) * P::STAGE_V,
+                                  vsrc + (kv_row0 + t0) * P::VROW, min(TT, end - t0) * P::VROW, rtid);
         }
         cp_async_commit();
       };
+      issue_v(0);
       for (int it = 0; it <= ntiles; ++it) {
-        cp_async_wait<0>();
+        cp_async_wait<1>();  // tile it - 1 has landed; tile it may still be in flight
         roles_sync();
-        issue_v(it);
+        issue_v(it + 1);     // into the stage tile it - 2 used
         if (it == 0) continue;
         const int j = it - 1;  // the tile scored in the previous step
         const int nt = min(TT, end - (start + j * TT));
@@ -471,7 +486,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
             for (int c = 0; c < 4; ++c) { acc[g][c].x *= al; acc[g][c].y *= al; }
           }
         }
-        const uint8_t* vst = smem + P::OFF_V + pb * P::STAGE_V;
+        const uint8_t* vst = smem + P::OFF_V + (j % kStages) * P::STAGE_V;
         const float2* prow = pbuf + static_cast<size_t>(pb) * TT * G;
 #pragma unroll 2
         for (int i = 0; i < WT / RPW; ++i) {
@@ -486,7 +501,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
 #pragma unroll
             for (int c = 0; c < 4; ++c)
               val[c] = *reinterpret_cast<const float2*>(reinterpret_cast<const uint8_t*>(tab) +
-                                                        pair_addr<BITS>(bits, c, rep_off));
+                                                        pair_addr<BITS, kDecReps>(bits, c, rep_off));
           } else {
             const uint4 u = *reinterpret_cast<const uint4*>(vst + tt * P::VROW + 16 * vc);
             val[0] = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
@@ -777,6 +792,188 @@ __global__ void __launch_bounds__(kDecThreads) score_kernel(const __grid_constan
       }
     }
     cp_async_wait<0>();
+  }
+}
+
+// ---- scores on the tensor cores ------------------------------------------------------------------------------------
+//
+// Persistent blocks of 128 threads; thread r owns token r of each 128-token tile and TMEM lane r.  Per tile: the
+// thread dequantizes its row's centroid pairs (hi and lo fp16 planes) into TMEM, one thread issues the d/8 MMAs
+// against the query's hi/lo planes in shared memory, and every thread reads back its token's accumulator columns.
+// Key codes are staged by cp.async four tiles deep (three in flight).
+// Staging layout for one-thread-per-row reads: the 16-byte chunk c of row t sits at chunk position c ^ f(t), so
+// that the 8 threads of a quarter warp reading chunk c of 8 consecutive rows hit 8 different bank groups.
+// Rows of 64 bytes use f(t) = (t >> 1) & 3, rows of 32 bytes f(t) = (t >> 2) & 1; other rows are unswizzled.
+template <int R>
+__device__ __forceinline__ int stage_swizzle(int o) {
+  if constexpr (R == 64) {
+    const int t = o >> 6, c = (o >> 4) & 3;
+    return (t << 6) | ((c ^ ((t >> 1) & 3)) << 4) | (o & 15);
+  } else if constexpr (R == 32) {
+    const int t = o >> 5, c = (o >> 4) & 1;
+    return (t << 5) | ((c ^ ((t >> 2) & 1)) << 4) | (o & 15);
+  } else {
+    return o;
+  }
+}
+
+template <int R>
+__device__ __forceinline__ void load_swizzled_row(const uint8_t* stage, int t, uint32_t* w) {
+  if constexpr (R % 16 == 0) {
+#pragma unroll
+    for (int c = 0; c < R / 16; ++c) {
+      const uint4 u = *reinterpret_cast<const uint4*>(stage + stage_swizzle<R>(t * R + c * 16));
+      w[4 * c] = u.x; w[4 * c + 1] = u.y; w[4 * c + 2] = u.z; w[4 * c + 3] = u.w;
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < R / 8; ++c) {
+      const uint2 u = *reinterpret_cast<const uint2*>(stage + t * R + c * 8);
+      w[2 * c] = u.x; w[2 * c + 1] = u.y;
+    }
+  }
+}
+
+template <int D, int BITS, int G>
+struct ScoreTcPlan {
+  static constexpr int TT = tc::kM;
+  static constexpr int R = D * BITS / 8;
+  static constexpr int KCH = (R % 16 == 0) ? 16 : 8;
+  static constexpr int NST = 4;
+  static constexpr int STAGE = TT * R;
+  static constexpr size_t OFF_STAGE = 0;
+  static constexpr size_t OFF_TAB = ((size_t)NST * STAGE + 255) / 256 * 256;
+  static constexpr size_t OFF_B = OFF_TAB + tc::PairTable16<BITS>::BYTES;
+  static constexpr size_t OFF_QS = OFF_B + tc::Layout<D>::B_BYTES;
+  static constexpr size_t OFF_SC = OFF_QS + (size_t)G * D * 4;     // scale[8], inv_scale[8]
+  static constexpr size_t OFF_CENT = OFF_SC + 16 * 4;
+  static constexpr size_t OFF_MBAR = OFF_CENT + 16 * 4;             // 8-byte aligned
+  static constexpr size_t OFF_TMEM = OFF_MBAR + 8;    // TMEM base address, then the failure flag
+  static constexpr size_t bytes = OFF_TMEM + 16;
+};
+
+template <int D, int BITS, int G>
+__global__ void __launch_bounds__(tc::kM, 2) score_tc_kernel(const __grid_constant__ DecodeArgs a) {
+  using P = ScoreTcPlan<D, BITS, G>;
+  using LY = tc::Layout<D>;
+  constexpr int R = P::R, TT = P::TT, NST = P::NST;
+  static_assert(G <= tc::kN / 2, "two accumulator columns per head");
+  extern __shared__ __align__(16) uint8_t smem[];
+  const uint8_t* tab = smem + P::OFF_TAB;
+  __half* bs = reinterpret_cast<__half*>(smem + P::OFF_B);
+  float* qs = reinterpret_cast<float*>(smem + P::OFF_QS);
+  float* scale_s = reinterpret_cast<float*>(smem + P::OFF_SC);
+  float* inv_s = scale_s + 8;
+  float* cent = reinterpret_cast<float*>(smem + P::OFF_CENT);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + P::OFF_MBAR);
+  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(smem + P::OFF_TMEM);
+  volatile int* failed = reinterpret_cast<volatile int*>(smem + P::OFF_TMEM + 4);
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid < 16) cent[tid] = a.cb.gamma[tid];
+  if (warp == 0) tc::tmem_alloc(tmem_s, LY::NCOLS);
+  if (tid == 0) {
+    tc::mbar_init(mbar, 1);
+    *failed = 0;
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_s;
+  const uint32_t tlane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+  tc::build_table<BITS>(cent, reinterpret_cast<uint2*>(smem + P::OFF_TAB));
+  const uint32_t repw = static_cast<uint32_t>(lane) << 3;
+  const uint32_t b_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(bs));
+  const float rd = rsqrtf(static_cast<float>(D));
+  uint32_t phase = 0;
+
+  const int items = a.B * a.Hkv * a.splits;
+  for (int item = blockIdx.x; item < items; item += gridDim.x) {
+    const int split = item % a.splits;
+    const int hk = (item / a.splits) % a.Hkv;
+    const int b = item / (a.splits * a.Hkv);
+    const int len = row_len(a, b);
+    const int start = split * a.chunk;
+    const int end = min(start + a.chunk, a.T);
+    const int vend = min(end, len);
+    const int ntiles = vend > start ? (vend - start + TT - 1) / TT : 0;
+    const size_t kv_row0 = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
+    float* out = a.scores + (static_cast<size_t>(b) * a.Hq + hk * G) * a.T;
+
+    __syncthreads();  // the previous item is done with the row factors, B and the stages
+    if (*failed) break;  // block-uniform: read after the barrier
+    transform_queries<D, G>(a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D, a.signs, a.mult, qs);
+    __syncthreads();
+    tc::build_b<D, G>(qs, bs, inv_s, scale_s);
+    tc::fence_async_smem();  // B is read by the tensor cores (async proxy)
+    for (int t = max(start, len) + tid; t < end; t += TT)
+#pragma unroll
+      for (int g = 0; g < G; ++g) out[static_cast<size_t>(g) * a.T + t] = -INFINITY;
+
+    auto issue_tile = [&](int tile) {
+      if (tile < ntiles) {
+        const int t0 = start + tile * TT;
+        uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % NST) * P::STAGE;
+        const uint8_t* src = a.kcodes + (kv_row0 + t0) * R;
+        const int bytes = min(TT, vend - t0) * R;
+        for (int o = tid * P::KCH; o < bytes; o += TT * P::KCH) cp_async<P::KCH>(st + stage_swizzle<R>(o), src + o);
+      }
+      cp_async_commit();
+    };
+    for (int s = 0; s < NST - 1; ++s) issue_tile(s);
+    float kn_next = (ntiles > 0 && start + tid < vend) ? __half2float(a.knorms[kv_row0 + start + tid]) : 0.f;
+
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int t0 = start + tile * TT;
+      const int nt = min(TT, vend - t0);
+      cp_async_wait<NST - 2>();
+      __syncthreads();  // this tile has landed everywhere; the previous tile's stage and accumulator reads are done
+      if (*failed) break;  // block-uniform: read after the barrier
+      issue_tile(tile + NST - 1);
+      const float kn_cur = kn_next;
+      if (tile + 1 < ntiles && t0 + TT + tid < vend) kn_next = __half2float(a.knorms[kv_row0 + t0 + TT + tid]);
+      {
+        // every lane stores a row (the store is warp-collective); rows past the tile end use all-zero codes
+        uint32_t w[R / 4 + 1];
+        load_swizzled_row<R>(smem + P::OFF_STAGE + static_cast<size_t>(tile % NST) * P::STAGE, tid, w);
+        if (tid >= nt) {
+#pragma unroll
+          for (int i = 0; i < R / 4; ++i) w[i] = 0u;
+        }
+        w[R / 4] = 0u;
+        tc::store_row<D, BITS>(w, tab, repw, tlane);
+      }
+      tc::wait_st();
+      tc::fence_before();
+      __syncthreads();  // every row of A is in tensor memory
+      if (tid == 0) {
+        tc::fence_after();
+        tc::issue_mma<D>(tmem, b_saddr, mbar);
+      }
+      const bool ok = tc::mbar_wait(mbar, phase);
+      if (!ok) *failed = 1;
+      phase ^= 1u;
+      tc::fence_after();
+      uint32_t dacc[16];
+      tc::ld_x16(tlane + LY::DCOL, dacc);
+      tc::wait_ld();
+      tc::fence_before();
+      if (tid < nt) {
+        const float f = kn_cur * rd;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float sc = (__uint_as_float(dacc[2 * g]) + __uint_as_float(dacc[2 * g + 1])) * inv_s[g] * f;
+          out[static_cast<size_t>(g) * a.T + t0 + tid] = ok ? sc : __int_as_float(0x7fc00000);
+        }
+      }
+    }
+    cp_async_wait<0>();
+  }
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after();
+    tc::tmem_dealloc(tmem, LY::NCOLS);
   }
 }
 

@@ -126,14 +126,18 @@ def score(q, kcodes, knorms, signs, bits, scale=1.0, seq_lens=None, T=None, out=
     return out
 
 
+GATHER_MODES = {"tensor": _abi.GATHER_TENSOR, "factored": _abi.GATHER_FACTORED, "table": _abi.GATHER_TABLE}
+
+
 def set_gather(mode: str) -> None:
-    """Table read mode of score(): "factored" (default) or "table" (the materialised table, gathered per entry)."""
-    code = {"factored": _abi.GATHER_FACTORED, "table": _abi.GATHER_TABLE}[mode]
-    _abi.check(_abi.lib().axr_set_gather(code), "axr_set_gather")
+    """Table read mode of score(): "tensor" (default: tensor cores), "factored" (packed fp32 FMAs) or "table"
+    (the materialised table, gathered per entry)."""
+    _abi.check(_abi.lib().axr_set_gather(GATHER_MODES[mode]), "axr_set_gather")
 
 
 def get_gather() -> str:
-    return "table" if _abi.lib().axr_get_gather() == _abi.GATHER_TABLE else "factored"
+    code = _abi.lib().axr_get_gather()
+    return {v: k for k, v in GATHER_MODES.items()}[code]
 
 
 def attend_workspace_bytes(B, Hq, Hkv, T, d) -> int:

@@ -44,8 +44,20 @@ SMALL += [(128, 3, g, vq) for g in (1, 2, 8) for vq in (False, True)]
 SMALL += [(64, 4, g, False) for g in (1, 2, 8)]
 
 
-@pytest.mark.parametrize("d,bits,G", sorted({(d, b, g) for d, b, g, _ in SMALL}))
-def test_score_matches_oracle(d, bits, G):
+SCORE_CASES = [(d, b, g, "tensor") for d, b, g in sorted({(d, b, g) for d, b, g, _ in SMALL})]
+SCORE_CASES += [(d, b, g, m) for m in ("factored", "table") for d, b, g in [(128, 4, 4), (64, 3, 4), (128, 2, 8),
+                                                                             (128, 1, 1)]]
+
+
+@pytest.fixture
+def gather_mode(request):
+    ops.set_gather(request.param)
+    yield request.param
+    ops.set_gather("tensor")
+
+
+@pytest.mark.parametrize("d,bits,G,gather_mode", SCORE_CASES, indirect=["gather_mode"])
+def test_score_matches_oracle(d, bits, G, gather_mode):
     B, Hkv, T, Tcap = 2, 2, 2500, 2560
     Hq = G * Hkv
     k, v, s, kc, kn, _, _ = oracle_cache(B, Hkv, T, d, bits, 300 + d + bits + G, False)
