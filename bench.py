@@ -296,10 +296,8 @@ def run_axr(args, w):
         del sc_out
 
     # max over ranks
-    t = torch.tensor([step_ms, e2e_ms, float(np.mean(attend_ms))], device=dev, dtype=torch.float64)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    step_ms, e2e_ms, attend_avg_ms = t.tolist()
+    from kv_cache_quantized_b200 import dist as D
+    step_ms, e2e_ms, attend_avg_ms = D.max_over_ranks([step_ms, e2e_ms, float(np.mean(attend_ms))], device=dev)
     if ws > 1:
         dist.destroy_process_group()
     if rank != 0:
