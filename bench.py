@@ -292,7 +292,7 @@ def run_axr(args, w):
             ms = float(np.mean([a_.elapsed_time(b2) for a_, b2 in evs]))
             sbytes = (R + 2 + 4 * w.G) * B * Hkv * T
             scorer[mode] = {"ms": ms, "achieved_gbs": sbytes / (ms / 1e3) / 1e9, "algorithmic_bytes": sbytes}
-        ops.set_gather("tensor")
+        ops.set_gather("factored")
         del sc_out
 
     # max over ranks

@@ -104,7 +104,7 @@ AXR_API axr_status axr_score(const float* q, const uint8_t* kcodes, const uint16
                      float* scores, void* stream);
 
 /*
- * Table read mode of axr_score (process-wide; default AXR_GATHER_TENSOR).  Every mode computes the same table
+ * Table read mode of axr_score (process-wide; default AXR_GATHER_FACTORED, the fastest on B200).  Every mode computes the same table
  * entries LUT[j][k] = scale * q~_j * c_k (AXELRAM Key Points, 2nd item) summed at each token's indices, and they agree
  * to within the score tolerance:
  *   AXR_GATHER_TABLE     the d x 2^b table (G heads wide) is materialised in shared memory and gathered entry by

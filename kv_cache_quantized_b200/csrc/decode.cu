@@ -3,6 +3,7 @@
 #include <cmath>
 
 #include "decode.cuh"
+#include "score_tc.cuh"
 
 namespace axr {
 namespace {
@@ -43,17 +44,18 @@ axr_status launch_attend(const DecodeArgs& a, cudaStream_t st, const char* what)
   return check_launch(what);
 }
 
-std::atomic<int> g_gather{kGatherTensor};
+std::atomic<int> g_gather{kGatherFactored};
 
 template <int D, int BITS, int G>
 axr_status launch_score_tc(const DecodeArgs& a, cudaStream_t st) {
-  using S = ScoreTcPlan<D, BITS, G>;
+  using S = TcScorePlan<D, BITS, G>;
   auto k = score_tc_kernel<D, BITS, G>;
-  axr_status rs = ensure_smem(k, S::bytes, "axr_score");
+  axr_status rs = ensure_smem(k, S::launch_bytes, "axr_score");
   if (rs != AXR_OK) return rs;
-  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;
-  const long resident = 2L * kSmCount;
-  k<<<static_cast<unsigned>(items < resident ? items : resident), tc::kM, S::bytes, st>>>(a);
+  // one persistent CTA per SM, each taking a contiguous share of the tiles (at most as many CTAs as tiles)
+  const long tiles = static_cast<long>(a.B) * a.Hkv * ((a.T + kTile - 1) / kTile);
+  const unsigned grid = static_cast<unsigned>(tiles < kSmCount ? tiles : kSmCount);
+  k<<<grid, S::THREADS, S::launch_bytes, st>>>(a);
   return check_launch("axr_score");
 }
 

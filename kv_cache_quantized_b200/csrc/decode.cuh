@@ -795,12 +795,8 @@ __global__ void __launch_bounds__(kDecThreads) score_kernel(const __grid_constan
   }
 }
 
-// ---- scores on the tensor cores ------------------------------------------------------------------------------------
+// ---- staging layout for one-thread-per-row reads ---------------------------------------------------------------
 //
-// Persistent blocks of 128 threads; thread r owns token r of each 128-token tile and TMEM lane r.  Per tile: the
-// thread dequantizes its row's centroid pairs (hi and lo fp16 planes) into TMEM, one thread issues the d/8 MMAs
-// against the query's hi/lo planes in shared memory, and every thread reads back its token's accumulator columns.
-// Key codes are staged by cp.async four tiles deep (three in flight).
 // Staging layout for one-thread-per-row reads: the 16-byte chunk c of row t sits at chunk position c ^ f(t), so
 // that the 8 threads of a quarter warp reading chunk c of 8 consecutive rows hit 8 different bank groups.
 // Rows of 64 bytes use f(t) = (t >> 1) & 3, rows of 32 bytes f(t) = (t >> 2) & 1; other rows are unswizzled.
@@ -831,149 +827,6 @@ __device__ __forceinline__ void load_swizzled_row(const uint8_t* stage, int t, u
       const uint2 u = *reinterpret_cast<const uint2*>(stage + t * R + c * 8);
       w[2 * c] = u.x; w[2 * c + 1] = u.y;
     }
-  }
-}
-
-template <int D, int BITS, int G>
-struct ScoreTcPlan {
-  static constexpr int TT = tc::kM;
-  static constexpr int R = D * BITS / 8;
-  static constexpr int KCH = (R % 16 == 0) ? 16 : 8;
-  static constexpr int NST = 4;
-  static constexpr int STAGE = TT * R;
-  static constexpr size_t OFF_STAGE = 0;
-  static constexpr size_t OFF_TAB = ((size_t)NST * STAGE + 255) / 256 * 256;
-  static constexpr size_t OFF_B = OFF_TAB + tc::PairTable16<BITS>::BYTES;
-  static constexpr size_t OFF_QS = OFF_B + tc::Layout<D>::B_BYTES;
-  static constexpr size_t OFF_SC = OFF_QS + (size_t)G * D * 4;     // scale[8], inv_scale[8]
-  static constexpr size_t OFF_CENT = OFF_SC + 16 * 4;
-  static constexpr size_t OFF_MBAR = OFF_CENT + 16 * 4;             // 8-byte aligned
-  static constexpr size_t OFF_TMEM = OFF_MBAR + 8;    // TMEM base address, then the failure flag
-  static constexpr size_t bytes = OFF_TMEM + 16;
-};
-
-template <int D, int BITS, int G>
-__global__ void __launch_bounds__(tc::kM, 2) score_tc_kernel(const __grid_constant__ DecodeArgs a) {
-  using P = ScoreTcPlan<D, BITS, G>;
-  using LY = tc::Layout<D>;
-  constexpr int R = P::R, TT = P::TT, NST = P::NST;
-  static_assert(G <= tc::kN / 2, "two accumulator columns per head");
-  extern __shared__ __align__(16) uint8_t smem[];
-  const uint8_t* tab = smem + P::OFF_TAB;
-  __half* bs = reinterpret_cast<__half*>(smem + P::OFF_B);
-  float* qs = reinterpret_cast<float*>(smem + P::OFF_QS);
-  float* scale_s = reinterpret_cast<float*>(smem + P::OFF_SC);
-  float* inv_s = scale_s + 8;
-  float* cent = reinterpret_cast<float*>(smem + P::OFF_CENT);
-  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + P::OFF_MBAR);
-  uint32_t* tmem_s = reinterpret_cast<uint32_t*>(smem + P::OFF_TMEM);
-  volatile int* failed = reinterpret_cast<volatile int*>(smem + P::OFF_TMEM + 4);
-
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < 16) cent[tid] = a.cb.gamma[tid];
-  if (warp == 0) tc::tmem_alloc(tmem_s, LY::NCOLS);
-  if (tid == 0) {
-    tc::mbar_init(mbar, 1);
-    *failed = 0;
-  }
-  tc::fence_before();
-  __syncthreads();
-  tc::fence_after();
-  const uint32_t tmem = *tmem_s;
-  const uint32_t tlane = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-  tc::build_table<BITS>(cent, reinterpret_cast<uint2*>(smem + P::OFF_TAB));
-  const uint32_t repw = static_cast<uint32_t>(lane) << 3;
-  const uint32_t b_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(bs));
-  const float rd = rsqrtf(static_cast<float>(D));
-  uint32_t phase = 0;
-
-  const int items = a.B * a.Hkv * a.splits;
-  for (int item = blockIdx.x; item < items; item += gridDim.x) {
-    const int split = item % a.splits;
-    const int hk = (item / a.splits) % a.Hkv;
-    const int b = item / (a.splits * a.Hkv);
-    const int len = row_len(a, b);
-    const int start = split * a.chunk;
-    const int end = min(start + a.chunk, a.T);
-    const int vend = min(end, len);
-    const int ntiles = vend > start ? (vend - start + TT - 1) / TT : 0;
-    const size_t kv_row0 = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
-    float* out = a.scores + (static_cast<size_t>(b) * a.Hq + hk * G) * a.T;
-
-    __syncthreads();  // the previous item is done with the row factors, B and the stages
-    if (*failed) break;  // block-uniform: read after the barrier
-    transform_queries<D, G>(a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D, a.signs, a.mult, qs);
-    __syncthreads();
-    tc::build_b<D, G>(qs, bs, inv_s, scale_s);
-    tc::fence_async_smem();  // B is read by the tensor cores (async proxy)
-    for (int t = max(start, len) + tid; t < end; t += TT)
-#pragma unroll
-      for (int g = 0; g < G; ++g) out[static_cast<size_t>(g) * a.T + t] = -INFINITY;
-
-    auto issue_tile = [&](int tile) {
-      if (tile < ntiles) {
-        const int t0 = start + tile * TT;
-        uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % NST) * P::STAGE;
-        const uint8_t* src = a.kcodes + (kv_row0 + t0) * R;
-        const int bytes = min(TT, vend - t0) * R;
-        for (int o = tid * P::KCH; o < bytes; o += TT * P::KCH) cp_async<P::KCH>(st + stage_swizzle<R>(o), src + o);
-      }
-      cp_async_commit();
-    };
-    for (int s = 0; s < NST - 1; ++s) issue_tile(s);
-    float kn_next = (ntiles > 0 && start + tid < vend) ? __half2float(a.knorms[kv_row0 + start + tid]) : 0.f;
-
-    for (int tile = 0; tile < ntiles; ++tile) {
-      const int t0 = start + tile * TT;
-      const int nt = min(TT, vend - t0);
-      cp_async_wait<NST - 2>();
-      __syncthreads();  // this tile has landed everywhere; the previous tile's stage and accumulator reads are done
-      if (*failed) break;  // block-uniform: read after the barrier
-      issue_tile(tile + NST - 1);
-      const float kn_cur = kn_next;
-      if (tile + 1 < ntiles && t0 + TT + tid < vend) kn_next = __half2float(a.knorms[kv_row0 + t0 + TT + tid]);
-      {
-        // every lane stores a row (the store is warp-collective); rows past the tile end use all-zero codes
-        uint32_t w[R / 4 + 1];
-        load_swizzled_row<R>(smem + P::OFF_STAGE + static_cast<size_t>(tile % NST) * P::STAGE, tid, w);
-        if (tid >= nt) {
-#pragma unroll
-          for (int i = 0; i < R / 4; ++i) w[i] = 0u;
-        }
-        w[R / 4] = 0u;
-        tc::store_row<D, BITS>(w, tab, repw, tlane);
-      }
-      tc::wait_st();
-      tc::fence_before();
-      __syncthreads();  // every row of A is in tensor memory
-      if (tid == 0) {
-        tc::fence_after();
-        tc::issue_mma<D>(tmem, b_saddr, mbar);
-      }
-      const bool ok = tc::mbar_wait(mbar, phase);
-      if (!ok) *failed = 1;
-      phase ^= 1u;
-      tc::fence_after();
-      uint32_t dacc[16];
-      tc::ld_x16(tlane + LY::DCOL, dacc);
-      tc::wait_ld();
-      tc::fence_before();
-      if (tid < nt) {
-        const float f = kn_cur * rd;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float sc = (__uint_as_float(dacc[2 * g]) + __uint_as_float(dacc[2 * g + 1])) * inv_s[g] * f;
-          out[static_cast<size_t>(g) * a.T + t0 + tid] = ok ? sc : __int_as_float(0x7fc00000);
-        }
-      }
-    }
-    cp_async_wait<0>();
-  }
-  tc::fence_before();
-  __syncthreads();
-  if (warp == 0) {
-    tc::fence_after();
-    tc::tmem_dealloc(tmem, LY::NCOLS);
   }
 }
 

@@ -73,6 +73,27 @@ __device__ __forceinline__ void ld_x16(uint32_t taddr, uint32_t (&d)[16]) {
       : "memory");
 }
 
+__device__ __forceinline__ void st_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* mbar) {
+  const uint32_t mb = static_cast<uint32_t>(__cvta_generic_to_shared(mbar));
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(mb) : "memory");
+}
+
+// The mbarrier counts one arrival once every cp.async this thread issued so far has landed (the arrival is part of
+// the barrier's expected count: no pending-count increment).
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* mbar) {
+  const uint32_t mb = static_cast<uint32_t>(__cvta_generic_to_shared(mbar));
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(mb) : "memory");
+}
+
 // Instruction descriptor of kind::f16: fp16 A and B (K-major), fp32 accumulator, M = 128, N = 16.
 __host__ __device__ constexpr uint32_t idesc_f16_m128_n16() {
   return (1u << 4) | (static_cast<uint32_t>(kN >> 3) << 17) | (static_cast<uint32_t>(kM >> 4) << 24);
@@ -84,8 +105,10 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t sbo) {
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
 }
 
+// The d/8 MMAs of one tile: D (TMEM, fp32, N columns at d_taddr) = A (TMEM, hi/lo planes from column a_taddr) x B
+// (shared memory at b_saddr), committed to mbar once they have all completed.
 template <int D>
-__device__ __forceinline__ void issue_mma(uint32_t tmem, uint32_t b_saddr, uint64_t* mbar) {
+__device__ __forceinline__ void issue_mma(uint32_t a_taddr, uint32_t d_taddr, uint32_t b_saddr, uint64_t* mbar) {
   using LY = Layout<D>;
   const uint32_t idesc = idesc_f16_m128_n16();
 #pragma unroll
@@ -94,8 +117,8 @@ __device__ __forceinline__ void issue_mma(uint32_t tmem, uint32_t b_saddr, uint6
     const uint32_t acc = s > 0 ? 1u : 0u;
     asm volatile(
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem + LY::DCOL),
-        "r"(tmem + static_cast<uint32_t>(s * 8)), "l"(desc), "r"(idesc), "r"(acc)
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_taddr),
+        "r"(a_taddr + static_cast<uint32_t>(s * 8)), "l"(desc), "r"(idesc), "r"(acc)
         : "memory");
   }
   const uint32_t mb = static_cast<uint32_t>(__cvta_generic_to_shared(mbar));
@@ -157,64 +180,49 @@ __device__ __forceinline__ uint32_t pair_off(const uint32_t* w, int i, uint32_t 
   }
 }
 
-// B operand from the fp32 row factors qs [G][D] (already scaled): per head a power-of-two range scale so that the
-// hi/lo split keeps its precision; inv_scale[h] undoes it.  Uses all threads of the block; ends without a barrier.
-template <int D, int G>
-__device__ __forceinline__ void build_b(const float* __restrict__ qs, __half* __restrict__ bs,
-                                        float* __restrict__ inv_scale, float* __restrict__ scale_s) {
-  using LY = Layout<D>;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // per-head max |q~| -> scale 2^(14 - exponent)
-  for (int g = warp; g < G; g += blockDim.x / 32) {
-    float m = 0.f;
-    for (int j = lane; j < D; j += 32) m = fmaxf(m, fabsf(qs[g * D + j]));
-    m = warp_max(m);
-    if (lane == 0) {
-      int e = 0;
-      frexpf(m, &e);  // m = f * 2^e, f in [0.5, 1)
-      const float s = m > 0.f ? ldexpf(1.f, 14 - e) : 1.f;
-      scale_s[g] = s;
-      inv_scale[g] = 1.f / s;
-    }
+// Power-of-two range scale of one head's query operand: 2^(14 - e) with |mult| * ||q|| in [2^(e-1), 2^e).  Every
+// |q~_j| is at most |mult| * ||q|| (the transform is orthonormal), so the scaled factors stay below 2^14 in fp16
+// while keeping fp16's relative precision; the epilogue divides it out.  Computed by a whole warp from the query in
+// global memory, identically wherever it is needed.
+template <int D>
+__device__ __forceinline__ float head_scale(const float* __restrict__ qh, float mult) {
+  const int lane = threadIdx.x & 31;
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < (D + 31) / 32; ++i) {
+    const int j = lane + 32 * i;
+    const float x = j < D ? qh[j] : 0.f;
+    ss = fmaf(x, x, ss);
   }
-  __syncthreads();
+  const float m = sqrtf(warp_sum(ss)) * fabsf(mult);
+  if (!(m > 0.f) || !isfinite(m)) return 1.f;
+  int e = 0;
+  frexpf(m, &e);
+  return ldexpf(1.f, 14 - e);
+}
+
+// B operand from the fp32 row factors qs [G][D] (already multiplied by mult) and the head scales: column 2h holds
+// hi(s_h q~_h) against both A planes, column 2h+1 holds lo(s_h q~_h) against the hi plane only.  One warp.
+template <int D, int G>
+__device__ __forceinline__ void build_b(const float* __restrict__ qs, const float (&scale)[G],
+                                        __half* __restrict__ bs) {
+  using LY = Layout<D>;
+  const int lane = threadIdx.x & 31;
   constexpr int K = 2 * D;
-  for (int idx = tid; idx < kN * K; idx += blockDim.x) {
+  for (int idx = lane; idx < kN * K; idx += 32) {
     const int n = idx / K, k = idx % K;
     const int h = n >> 1;
     float v = 0.f;
-    if (h < G) {
-      const float q = qs[h * D + (k % D)] * scale_s[h];
-      const float qh = __half2float(__float2half_rn(q));
-      v = (n & 1) ? (k < D ? q - qh : 0.f) : qh;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (g == h) {
+        const float q = qs[g * D + (k % D)] * scale[g];
+        const float qh = __half2float(__float2half_rn(q));
+        v = (n & 1) ? (k < D ? q - qh : 0.f) : qh;
+      }
     }
     const int off = (n >> 3) * (LY::SBO / 2) + (k >> 3) * 64 + (n & 7) * 8 + (k & 7);
     bs[off] = __float2half_rn(v);
-  }
-}
-
-// Dequantize one token row (packed codes in w) into the two TMEM planes of this thread's lane.  tcgen05.st is a
-// warp-collective (.sync.aligned) instruction: every lane of the warp must call this, with some row of codes.
-template <int D, int BITS>
-__device__ __forceinline__ void store_row(const uint32_t* w, const uint8_t* tab, uint32_t repw, uint32_t tlane) {
-  constexpr int PAIRS = D / 2;
-  constexpr int CH = PAIRS < 32 ? PAIRS : 32;
-#pragma unroll
-  for (int c0 = 0; c0 < PAIRS; c0 += 32) {
-    uint32_t hi[32], lo[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      if (i < CH) {
-        const uint2 e = *reinterpret_cast<const uint2*>(tab + pair_off<BITS>(w, c0 + i, repw));
-        hi[i] = e.x;
-        lo[i] = e.y;
-      } else {
-        hi[i] = 0u;
-        lo[i] = 0u;
-      }
-    }
-    st_x32(tlane + static_cast<uint32_t>(c0), hi);
-    st_x32(tlane + static_cast<uint32_t>(PAIRS + c0), lo);
   }
 }
 

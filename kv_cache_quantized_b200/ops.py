@@ -130,7 +130,7 @@ GATHER_MODES = {"tensor": _abi.GATHER_TENSOR, "factored": _abi.GATHER_FACTORED, 
 
 
 def set_gather(mode: str) -> None:
-    """Table read mode of score(): "tensor" (default: tensor cores), "factored" (packed fp32 FMAs) or "table"
+    """Table read mode of score(): "factored" (default: packed fp32 FMAs), "tensor" (tensor cores) or "table"
     (the materialised table, gathered per entry)."""
     _abi.check(_abi.lib().axr_set_gather(GATHER_MODES[mode]), "axr_set_gather")
 

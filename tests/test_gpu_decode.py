@@ -53,7 +53,7 @@ SCORE_CASES += [(d, b, g, m) for m in ("factored", "table") for d, b, g in [(128
 def gather_mode(request):
     ops.set_gather(request.param)
     yield request.param
-    ops.set_gather("tensor")
+    ops.set_gather("factored")
 
 
 @pytest.mark.parametrize("d,bits,G,gather_mode", SCORE_CASES, indirect=["gather_mode"])
