@@ -55,7 +55,9 @@ typedef enum axr_status {
 } axr_status;
 
 typedef enum axr_dtype { AXR_F32 = 0, AXR_F16 = 1 } axr_dtype;
-typedef enum axr_vkind { AXR_V_F16 = 0, AXR_V_QUANT = 1 } axr_vkind;
+/* Value storage for axr_attend_decode: fp16 rows, quantized rows (the keys' layout), or quantized and tiled
+ * (axr_write_values_tiled's layout, d = 128). */
+typedef enum axr_vkind { AXR_V_F16 = 0, AXR_V_QUANT = 1, AXR_V_QUANT_TILED = 2 } axr_vkind;
 
 /* Thread-local message for the last non-OK status returned on this thread (empty string if none). */
 AXR_API const char* axr_last_error(void);
@@ -88,6 +90,25 @@ AXR_API axr_status axr_codebook(int d, int bits, double* centroids, double* thre
  */
 AXR_API axr_status axr_write_keys(const void* x, axr_dtype x_dtype, int64_t n_vec, int d, int bits, const int8_t* signs,
                           const int64_t* dst_rows, uint8_t* codes, uint16_t* norms, void* stream);
+
+/*
+ * axr_write_values_tiled -- the write path of axr_write_keys (same transform, norm, codebook and tie rule) with the
+ * codes stored for the tensor-core value product: the cache is cut into tiles of 128 tokens and within a tile each
+ * coordinate's 128 codes form one LSB-first bitstream, token o at bits [o*b, o*b + b).  The pages fix no layout
+ * (AXELRAM Key Points, 2nd item, quantizes the cache once; the values are quantized the same way); this one lets
+ * the read path gather two tokens' values of a coordinate with one lookup.
+ *   x         [dev] [n_vec, d] of x_dtype, contiguous rows;  signs [dev] [d] int8;
+ *   dst_rows  [dev] [n_vec] int64 destination rows r = (b*Hkv + h)*Tcap + t, distinct, or NULL for rows 0..n_vec-1;
+ *   Tcap      tokens per (batch, KV head) in the cache, a positive multiple of 128;
+ *   codes     [dev] out, [B*Hkv][Tcap/128][d][16*b] bytes (4-byte aligned);  norms [dev] out, fp16 per row r.
+ * With dst_rows NULL and n_vec a multiple of 128 whole tiles are written with plain stores; otherwise each code is
+ * replaced in place with word atomics (other tokens of the tile keep theirs).
+ * Errors: AXR_EINVAL (null pointer, n_vec < 0, bad dtype, Tcap, misalignment), AXR_EUNSUPPORTED (d != 128, b),
+ * AXR_ECUDA.  n_vec == 0 is a no-op.
+ */
+AXR_API axr_status axr_write_values_tiled(const void* x, axr_dtype x_dtype, int64_t n_vec, int d, int bits,
+                                          const int8_t* signs, const int64_t* dst_rows, int Tcap, uint8_t* codes,
+                                          uint16_t* norms, void* stream);
 
 /*
  * axr_score -- read-path scores (AXELRAM Key Points, 1st and 2nd items; Abstract: scores straight from the indices
@@ -131,9 +152,12 @@ AXR_API size_t axr_attend_workspace_bytes(int B, int Hq, int Hkv, int T, int d);
  * `scale`, typically 1/sqrt(d)), an online softmax per split of the token axis, the value product, and a merge of
  * the splits.  Values are fp16 (AXR_V_F16: out = sum_t p_t v_t) or quantized like the keys with the same signs
  * (AXR_V_QUANT: the weighted sum is formed in the rotated domain and mapped back once, out = s .* H (sum_t p_t
- * n^V_t c[idx^V_t])).  The softmax, the value product and the split merge are not on the pages (an SRAM macro only
- * scores); they are the standard definitions.  A batch row with len_b = 0 gets out = 0.
- *   v [dev] fp16 values or value codes;  vnorms [dev] value norms (AXR_V_QUANT) or NULL (AXR_V_F16);
+ * n^V_t c[idx^V_t])).  AXR_V_QUANT_TILED takes the value codes in axr_write_values_tiled's layout (d = 128, Tcap
+ * a multiple of 128) and forms the value product on the tensor cores: per 128-token tile an M = 128 (coordinates) x
+ * N = 16 (heads) x K = 128 (tokens) MMA of the fp16 value centroids with the fp16 weights p_t n^V_t, accumulated in
+ * fp32.  The softmax, the value product and the split merge are not on the pages (an SRAM macro only scores); they
+ * are the standard definitions.  A batch row with len_b = 0 gets out = 0.
+ *   v [dev] fp16 values or value codes;  vnorms [dev] value norms (quantized kinds) or NULL (AXR_V_F16);
  *   out [dev] [B, Hq, d] f32;  workspace [dev] >= axr_attend_workspace_bytes(B, Hq, Hkv, T, d) bytes, 16-aligned.
  * Errors: as axr_score, plus AXR_EWORKSPACE.
  */

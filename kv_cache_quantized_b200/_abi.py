@@ -14,7 +14,7 @@ LIB_PATH = os.path.join(_HERE, "libaxr.so")
 
 STATUS = {0: "AXR_OK", 1: "AXR_EINVAL", 2: "AXR_EUNSUPPORTED", 3: "AXR_ECUDA", 4: "AXR_EWORKSPACE"}
 F32, F16 = 0, 1
-V_F16, V_QUANT = 0, 1
+V_F16, V_QUANT, V_QUANT_TILED = 0, 1, 2
 GATHER_FACTORED, GATHER_TABLE, GATHER_TENSOR = 0, 1, 2
 
 _p = ctypes.c_void_p
@@ -28,6 +28,7 @@ SIGNATURES = {
     "axr_version": (_i, []),
     "axr_codebook": (_i, [_i, _i, _p, _p]),
     "axr_write_keys": (_i, [_p, _i, _i64, _i, _i, _p, _p, _p, _p, _p]),
+    "axr_write_values_tiled": (_i, [_p, _i, _i64, _i, _i, _p, _p, _i, _p, _p, _p]),
     "axr_score": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p]),
     "axr_attend_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "axr_attend_decode": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p, _sz, _p]),

@@ -4,6 +4,7 @@
 
 #include "decode.cuh"
 #include "score_tc.cuh"
+#include "attend_tcv.cuh"
 
 namespace axr {
 namespace {
@@ -42,6 +43,40 @@ axr_status launch_attend(const DecodeArgs& a, cudaStream_t st, const char* what)
   k1<<<grid, kDecThreads, S::bytes, st>>>(a);
   attend_reduce_kernel<D, VQ><<<a.B * a.Hq, D, 0, st>>>(a);
   return check_launch(what);
+}
+
+template <int BITS, int G>
+axr_status launch_attend_tcv(const DecodeArgs& a, cudaStream_t st) {
+  using S = TcaPlan<BITS, G>;
+  auto k1 = attend_tcv_kernel<BITS, G>;
+  axr_status rs = ensure_smem(k1, S::bytes, "axr_attend_decode");
+  if (rs != AXR_OK) return rs;
+  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent: one CTA per SM
+  const unsigned grid = static_cast<unsigned>(items < kSmCount ? items : kSmCount);
+  k1<<<grid, S::THREADS, S::bytes, st>>>(a);
+  attend_reduce_kernel<128, true><<<a.B * a.Hq, 128, 0, st>>>(a);
+  return check_launch("axr_attend_decode");
+}
+
+template <int BITS>
+axr_status attend_tcv_g(int G, const DecodeArgs& a, cudaStream_t st) {
+  switch (G) {
+    case 1: return launch_attend_tcv<BITS, 1>(a, st);
+    case 2: return launch_attend_tcv<BITS, 2>(a, st);
+    case 4: return launch_attend_tcv<BITS, 4>(a, st);
+    case 8: return launch_attend_tcv<BITS, 8>(a, st);
+  }
+  return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: G=%d", G);
+}
+
+axr_status attend_tcv_bits(int bits, int G, const DecodeArgs& a, cudaStream_t st) {
+  switch (bits) {
+    case 1: return attend_tcv_g<1>(G, a, st);
+    case 2: return attend_tcv_g<2>(G, a, st);
+    case 3: return attend_tcv_g<3>(G, a, st);
+    case 4: return attend_tcv_g<4>(G, a, st);
+  }
+  return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: bits=%d", bits);
 }
 
 std::atomic<int> g_gather{kGatherFactored};
@@ -200,9 +235,14 @@ extern "C" axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, c
   axr_status st = check_decode_sizes(w, B, Hq, Hkv, T, Tcap, d);
   if (st != AXR_OK) return st;
   if (bits < 1 || bits > 4) return set_error(AXR_EUNSUPPORTED, "%s: bits=%d outside 1..4", w, bits);
-  if (vkind != AXR_V_F16 && vkind != AXR_V_QUANT) return set_error(AXR_EINVAL, "%s: bad vkind", w);
+  if (vkind != AXR_V_F16 && vkind != AXR_V_QUANT && vkind != AXR_V_QUANT_TILED)
+    return set_error(AXR_EINVAL, "%s: bad vkind", w);
+  if (vkind == AXR_V_QUANT_TILED && d != 128)
+    return set_error(AXR_EUNSUPPORTED, "%s: tiled values need d = 128 (d=%d)", w, d);
+  if (vkind == AXR_V_QUANT_TILED && Tcap % 128)
+    return set_error(AXR_EINVAL, "%s: tiled values need Tcap a multiple of 128 (Tcap=%d)", w, Tcap);
   if (B == 0) return set_error(AXR_OK, "");
-  if (!q || !kcodes || !knorms || !signs || !v || !out || (vkind == AXR_V_QUANT && !vnorms))
+  if (!q || !kcodes || !knorms || !signs || !v || !out || (vkind != AXR_V_F16 && !vnorms))
     return set_error(AXR_EINVAL, "%s: null pointer", w);
   if (!aligned(q, 16) || !aligned(kcodes, 16) || !aligned(knorms, 4) || !aligned(out, 16) || !aligned(v, 16) ||
       (vnorms && !aligned(vnorms, 4)) || (seq_lens && !aligned(seq_lens, 4)))
@@ -220,6 +260,7 @@ extern "C" axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, c
   a.kcodes = kcodes; a.knorms = reinterpret_cast<const __half*>(knorms); a.signs = signs; a.out = out;
   a.v = v; a.vnorms = reinterpret_cast<const __half*>(vnorms); a.cb = *cb;
   const int G = Hq / Hkv;
+  if (vkind == AXR_V_QUANT_TILED) return attend_tcv_bits(bits, G, a, as_stream(stream));
   const bool vq = vkind == AXR_V_QUANT;
   return d == 64 ? attend_bits<64>(bits, G, vq, a, as_stream(stream))
                  : attend_bits<128>(bits, G, vq, a, as_stream(stream));

@@ -133,8 +133,7 @@ struct TcScorePlan {
   static constexpr size_t OFF_STAGE = 0;
   static constexpr size_t OFF_TAB = ((size_t)NS * STAGE + 1023) / 1024 * 1024;
   static constexpr size_t OFF_B = OFF_TAB + ((size_t)tc::PairTable16<BITS>::BYTES + 1023) / 1024 * 1024;
-  static constexpr size_t OFF_QS = OFF_B + 2 * (size_t)B_BYTES;       // [G][D] row factors (B build scratch)
-  static constexpr size_t OFF_CENT = OFF_QS + (size_t)G * D * 4;
+  static constexpr size_t OFF_CENT = OFF_B + 2 * (size_t)B_BYTES;
   static constexpr size_t OFF_MBAR = OFF_CENT + 16 * 4;               // a_full, mma_done, d_empty, code_full, b_full
   static constexpr int NMBAR = 3 * NB + NS + 2;
   static constexpr size_t OFF_MISC = OFF_MBAR + (size_t)NMBAR * 8;    // TMEM base, failure flag
@@ -148,10 +147,9 @@ __global__ void __launch_bounds__(TcScorePlan<D, BITS, G>::THREADS, 1)
 score_tc_kernel(const __grid_constant__ DecodeArgs a) {
   using P = TcScorePlan<D, BITS, G>;
   constexpr int R = P::R, TT = P::TT, NB = P::NB, NS = P::NS, LA = P::LA, PG = P::PG;
-  extern __shared__ __align__(1024) uint8_t smem[];
+  extern __shared__ __align__(16) uint8_t smem[];
   uint8_t* stage = smem + P::OFF_STAGE;
   const uint8_t* tab = smem + P::OFF_TAB;
-  float* qs = reinterpret_cast<float*>(smem + P::OFF_QS);
   float* cent = reinterpret_cast<float*>(smem + P::OFF_CENT);
   uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + P::OFF_MBAR);
   uint64_t* a_full = mbar;
@@ -194,6 +192,9 @@ score_tc_kernel(const __grid_constant__ DecodeArgs a) {
   tc::fence_after();
   const uint32_t tmem = *tmem_s;
   tc::build_table<BITS>(cent, reinterpret_cast<uint2*>(smem + P::OFF_TAB));
+  for (int i = tid; i < 2 * P::B_BYTES / 4; i += P::THREADS)  // entries the row builder never writes stay 0
+    reinterpret_cast<uint32_t*>(smem + P::OFF_B)[i] = 0u;
+  tc::fence_async_smem();
   __syncthreads();
 
   if (warp < P::GW) {
@@ -289,13 +290,8 @@ score_tc_kernel(const __grid_constant__ DecodeArgs a) {
     const bool builder = warp == P::EW0;
     // B of row (b, hk) into slot `slot`, by the builder warp alone (no cross-warp barrier)
     auto build_row_b = [&](int b, int hk, int slot) {
-      const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
-      transform_queries_role<D, G>(qg, a.signs, a.mult, qs, 0, 1);
-      float scl[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) scl[g] = tc::head_scale<D>(qg + g * D, a.mult);
-      __syncwarp();
-      tc::build_b<D, G>(qs, scl, reinterpret_cast<__half*>(smem + P::OFF_B + slot * P::B_BYTES));
+      tc::build_b_warp<D, G>(a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D, a.signs, a.mult,
+                             reinterpret_cast<__half*>(smem + P::OFF_B + slot * P::B_BYTES));
       tc::fence_async_smem();  // B is read by the tensor cores (async proxy)
       __syncwarp();
       if (lane == 0) tc::mbar_arrive(b_full + slot);

@@ -19,6 +19,8 @@
 
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "axr_common.cuh"
 
 namespace axr {
@@ -180,6 +182,10 @@ __device__ __forceinline__ uint32_t pair_off(const uint32_t* w, int i, uint32_t 
   }
 }
 
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 // Power-of-two range scale of one head's query operand: 2^(14 - e) with |mult| * ||q|| in [2^(e-1), 2^e).  Every
 // |q~_j| is at most |mult| * ||q|| (the transform is orthonormal), so the scaled factors stay below 2^14 in fp16
 // while keeping fp16's relative precision; the epilogue divides it out.  Computed by a whole warp from the query in
@@ -201,28 +207,46 @@ __device__ __forceinline__ float head_scale(const float* __restrict__ qh, float 
   return ldexpf(1.f, 14 - e);
 }
 
-// B operand from the fp32 row factors qs [G][D] (already multiplied by mult) and the head scales: column 2h holds
-// hi(s_h q~_h) against both A planes, column 2h+1 holds lo(s_h q~_h) against the hi plane only.  One warp.
+// B operand of the G heads of one KV head, built by one warp from the raw queries: q~_h = mult * H (s .* q_h) in
+// registers (lane l holds coordinates 4l .. 4l + 3 for d = 128), scaled by head_scale, split into hi/lo fp16.
+// Column 2h holds hi against both A planes, column 2h+1 holds lo against the hi plane; every other entry of the
+// operand is zero and is written once (zero_b) -- only the 3 G d live entries are stored per row.
+template <int D>
+__device__ __forceinline__ int b_off(int n, int k) {  // K-major, no-swizzle canonical layout, in halves
+  return (n >> 3) * (Layout<D>::SBO / 2) + (k >> 3) * 64 + (n & 7) * 8 + (k & 7);
+}
+
 template <int D, int G>
-__device__ __forceinline__ void build_b(const float* __restrict__ qs, const float (&scale)[G],
-                                        __half* __restrict__ bs) {
-  using LY = Layout<D>;
+__device__ __forceinline__ void build_b_warp(const float* __restrict__ qg, const int8_t* __restrict__ signs,
+                                             float mult, __half* __restrict__ bs) {
+  constexpr int VPL = D / 32;  // coordinates per lane, consecutive: they share one 16-byte core-matrix row
+  static_assert(VPL == 2 || VPL == 4, "d = 64 or 128");
+  using Vec = typename std::conditional<VPL == 4, uint2, uint32_t>::type;
   const int lane = threadIdx.x & 31;
-  constexpr int K = 2 * D;
-  for (int idx = lane; idx < kN * K; idx += 32) {
-    const int n = idx / K, k = idx % K;
-    const int h = n >> 1;
-    float v = 0.f;
+  const float norm = mult * rsqrtf(static_cast<float>(D));
+  float sg[VPL];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      if (g == h) {
-        const float q = qs[g * D + (k % D)] * scale[g];
-        const float qh = __half2float(__float2half_rn(q));
-        v = (n & 1) ? (k < D ? q - qh : 0.f) : qh;
-      }
+  for (int i = 0; i < VPL; ++i) sg[i] = signs[VPL * lane + i] < 0 ? -1.f : 1.f;
+#pragma unroll
+  for (int h = 0; h < G; ++h) {
+    float v[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) v[i] = qg[h * D + VPL * lane + i] * sg[i];
+    fwht_warp<D>(v, lane);
+    const float sc = head_scale<D>(qg + h * D, mult);
+    uint32_t hw[VPL / 2], lw[VPL / 2];
+#pragma unroll
+    for (int i = 0; i < VPL; i += 2) {
+      const float q0 = v[i] * norm * sc, q1 = v[i + 1] * norm * sc;
+      const __half h0 = __float2half_rn(q0), h1 = __float2half_rn(q1);
+      const __half2 hh = __halves2half2(h0, h1);
+      const __half2 ll = __halves2half2(__float2half_rn(q0 - __half2float(h0)), __float2half_rn(q1 - __half2float(h1)));
+      hw[i / 2] = *reinterpret_cast<const uint32_t*>(&hh);
+      lw[i / 2] = *reinterpret_cast<const uint32_t*>(&ll);
     }
-    const int off = (n >> 3) * (LY::SBO / 2) + (k >> 3) * 64 + (n & 7) * 8 + (k & 7);
-    bs[off] = __float2half_rn(v);
+    *reinterpret_cast<Vec*>(bs + b_off<D>(2 * h, VPL * lane)) = *reinterpret_cast<const Vec*>(hw);
+    *reinterpret_cast<Vec*>(bs + b_off<D>(2 * h, D + VPL * lane)) = *reinterpret_cast<const Vec*>(hw);
+    *reinterpret_cast<Vec*>(bs + b_off<D>(2 * h + 1, VPL * lane)) = *reinterpret_cast<const Vec*>(lw);
   }
 }
 

@@ -88,6 +88,57 @@ def write_keys(x: torch.Tensor, signs: torch.Tensor, bits: int, codes: torch.Ten
     return codes, norms
 
 
+TILE = 128  # tokens per tile of the tiled value layout
+
+
+def tiled_shape(B, Hkv, Tcap, d, bits):
+    """Shape of value codes in the tiled layout: [B, Hkv, Tcap/128, d, 16*b] uint8."""
+    if Tcap % TILE:
+        raise ValueError("the tiled layout needs Tcap to be a multiple of 128")
+    return (B, Hkv, Tcap // TILE, d, TILE * bits // 8)
+
+
+def write_values_tiled(x: torch.Tensor, signs: torch.Tensor, bits: int, codes: torch.Tensor | None = None,
+                       norms: torch.Tensor | None = None, dst_rows: torch.Tensor | None = None, Tcap: int | None = None):
+    """Quantize value vectors like write_keys, storing the codes tiled for the tensor-core value product.
+
+    Without dst_rows x is the whole cache [B, Hkv, Tcap, d] (Tcap a multiple of 128) and (codes [B, Hkv, Tcap/128,
+    d, 16*b], norms [B, Hkv, Tcap]) are returned.  With dst_rows (int64, rows (b*Hkv + h)*Tcap + t) the vectors x
+    [n, d] are written into the given codes/norms in place.
+    """
+    _need_cuda("x", x)
+    _need_cuda("signs", signs, torch.int8)
+    if x.dtype not in (torch.float16, torch.float32):
+        raise TypeError("x must be float16 or float32")
+    d = x.shape[-1]
+    n_vec = x.numel() // d if d else 0
+    if dst_rows is None:
+        if x.dim() != 4:
+            raise ValueError("x must be [B, Hkv, Tcap, d] without dst_rows")
+        B, Hkv, Tc, _ = x.shape
+        Tcap = Tc
+        if codes is None:
+            codes = torch.empty(tiled_shape(B, Hkv, Tcap, d, bits), dtype=torch.uint8, device=x.device)
+        if norms is None:
+            norms = torch.empty((B, Hkv, Tcap), dtype=torch.float16, device=x.device)
+    else:
+        _need_cuda("dst_rows", dst_rows, torch.int64)
+        if codes is None or norms is None:
+            raise ValueError("dst_rows needs the destination codes and norms buffers")
+        if dst_rows.numel() != n_vec:
+            raise ValueError("dst_rows must hold one row index per vector")
+        if codes.dim() != 5:
+            raise ValueError("codes must be [B, Hkv, Tcap/128, d, 16*b]")
+        Tcap = codes.shape[2] * TILE
+    _need_cuda("codes", codes, torch.uint8)
+    _need_cuda("norms", norms, torch.float16)
+    dt = _abi.F16 if x.dtype == torch.float16 else _abi.F32
+    st = _abi.lib().axr_write_values_tiled(_ptr(x), dt, n_vec, d, bits, _ptr(signs), _ptr(dst_rows), int(Tcap),
+                                           _ptr(codes), _ptr(norms), _stream())
+    _abi.check(st, "axr_write_values_tiled")
+    return codes, norms
+
+
 def _cache_dims(q, kcodes, knorms, d, bits, T):
     _need_cuda("q", q, torch.float32)
     _need_cuda("kcodes", kcodes, torch.uint8)
@@ -154,7 +205,8 @@ def _workspace(nbytes, device, ws):
 def attend_decode(q, kcodes, knorms, signs, bits, v=None, vcodes=None, vnorms=None, scale=None, seq_lens=None,
                   T=None, out=None, workspace=None):
     """One decode step over a quantized key cache.  Values: v (float16 [B,Hkv,Tcap,d]) or vcodes/vnorms (quantized
-    like the keys with the same signs).  Returns out [B, Hq, d] float32."""
+    like the keys with the same signs, in the keys' row layout or -- 5-D -- in write_values_tiled's layout, which
+    runs the value product on the tensor cores).  Returns out [B, Hq, d] float32."""
     d = q.shape[-1]
     B, Hq, Hkv, Tcap, T = _cache_dims(q, kcodes, knorms, d, bits, T)
     _need_cuda("signs", signs, torch.int8)
@@ -169,9 +221,17 @@ def attend_decode(q, kcodes, knorms, signs, bits, v=None, vcodes=None, vnorms=No
     else:
         _need_cuda("vcodes", vcodes, torch.uint8)
         _need_cuda("vnorms", vnorms, torch.float16)
-        if vcodes.shape != kcodes.shape or vnorms.shape != knorms.shape:
-            raise ValueError("vcodes/vnorms must have the key cache's shapes")
-        vkind, vptr, vnptr = _abi.V_QUANT, _ptr(vcodes), _ptr(vnorms)
+        if vnorms.shape != knorms.shape:
+            raise ValueError("vnorms must have the key norms' shape")
+        if vcodes.dim() == 5:  # tiled layout (write_values_tiled)
+            if tuple(vcodes.shape) != tiled_shape(B, Hkv, Tcap, d, bits):
+                raise ValueError("tiled vcodes must be [B, Hkv, Tcap/128, d, 16*b]")
+            vkind = _abi.V_QUANT_TILED
+        else:
+            if vcodes.shape != kcodes.shape:
+                raise ValueError("vcodes must have the key cache's shape")
+            vkind = _abi.V_QUANT
+        vptr, vnptr = _ptr(vcodes), _ptr(vnorms)
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)

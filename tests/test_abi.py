@@ -79,6 +79,28 @@ def test_write_argument_errors(L):
     assert L.axr_write_keys(None, 0, 0, 128, 4, None, None, None, None, None) == 0  # empty is a no-op
 
 
+def test_write_tiled_argument_errors(L):
+    W = L.axr_write_values_tiled
+    assert W(FAKE, 0, -1, 128, 4, FAKE, None, 256, FAKE, FAKE, None) == 1     # n_vec < 0
+    assert W(FAKE, 0, 128, 64, 4, FAKE, None, 256, FAKE, FAKE, None) == 2     # tiles are built for d = 128
+    assert W(FAKE, 0, 128, 128, 0, FAKE, None, 256, FAKE, FAKE, None) == 2
+    assert W(FAKE, 0, 128, 128, 4, FAKE, None, 200, FAKE, FAKE, None) == 1    # Tcap not a multiple of 128
+    assert W(FAKE, 0, 128, 128, 4, FAKE, None, 0, FAKE, FAKE, None) == 1
+    assert W(None, 0, 128, 128, 4, FAKE, None, 256, FAKE, FAKE, None) == 1
+    assert W(FAKE, 0, 128, 128, 4, FAKE, None, 256, FAKE + 2, FAKE, None) == 1  # codes need 4-byte alignment
+    assert W(None, 0, 0, 128, 4, None, None, 256, None, None, None) == 0       # empty is a no-op
+
+
+def test_attend_tiled_argument_errors(L):
+    call = lambda d=128, Tcap=256, vn=FAKE: L.axr_attend_decode(FAKE, FAKE, FAKE, 2, FAKE, vn, None, 2, 8, 2, 200,
+                                                               Tcap, d, 4, FAKE, 0.1, FAKE, FAKE, 1 << 20, None)
+    assert call(d=64, Tcap=256) == 2   # tiled values: d = 128 only
+    assert call(Tcap=320) == 1         # Tcap a multiple of 128
+    assert call(vn=None) == 1          # value norms required
+    assert L.axr_attend_decode(FAKE, FAKE, FAKE, 3, FAKE, FAKE, None, 2, 8, 2, 200, 256, 128, 4, FAKE, 0.1, FAKE,
+                               FAKE, 1 << 20, None) == 1  # unknown vkind
+
+
 def test_score_argument_errors(L):
     args = lambda **kw: dict(dict(q=FAKE, kc=FAKE, kn=FAKE, sl=None, B=2, Hq=8, Hkv=2, T=10, Tcap=16, d=128,
                                   bits=4, s=FAKE, scale=1.0, out=FAKE), **kw)
