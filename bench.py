@@ -190,8 +190,11 @@ def run_axr(args, w):
         k = W.lognormal_rows_device((B, Hkv, T, d), seed, dev)
     v = (W.lognormal_rows_device if w.v_quant else W.normal_device)((B, Hkv, T, d), seed + 2, dev)
     kc, kn = ops.write_keys(k, signs, bits)
+    vt = vtn = None
     if w.v_quant:
         vc, vn = ops.write_keys(v, signs, bits)
+        if not args.no_variants and d == 128:  # the tiled value layout, for the variants below
+            vt, vtn = ops.write_values_tiled(v, signs, bits)
         del v
         v = None
     del k
@@ -273,11 +276,37 @@ def run_axr(args, w):
     h2d = q_h.numel() * 4 + k_h.numel() * 2 + v_h.numel() * 2
     d2h = o_h.numel() * 4
 
-    # the scorer alone (axr_score) on the same cache, both table read modes, L2 flushed before each call
+    def time_calls(fn):  # mean ms per call, L2 flushed before each call, outside the events
+        for _ in range(3):
+            fn()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        for a_, b2 in evs:
+            flush.zero_()
+            a_.record(stream)
+            fn()
+            b2.record(stream)
+        torch.cuda.synchronize()
+        return float(np.mean([a_.elapsed_time(b2) for a_, b2 in evs]))
+
+    # attend_decode over the tiled value layout (same cache contents): value product as warp-level MMAs, and the
+    # tcgen05 kernel (key scores and value product from tensor memory)
+    variants = {}
+    if vt is not None:
+        ab = _bytes_per_key_head(w) * B * Hkv * T
+        for name, mode in (("tiled_values_mma", "mma"), ("tiled_values_tcgen05", "tensor")):
+            ops.set_gather(mode)
+            ms = time_calls(lambda: ops.attend_decode(q, kc, kn, signs, bits, vcodes=vt, vnorms=vtn, out=out,
+                                                      workspace=wsp))
+            variants[name] = {"ms": ms, "achieved_gbs": ab / (ms / 1e3) / 1e9, "algorithmic_bytes": ab}
+        ops.set_gather("mma")
+        variants["rows"] = {"ms": float(np.mean(attend_ms)),
+                            "achieved_gbs": ab / (float(np.mean(attend_ms)) / 1e3) / 1e9, "algorithmic_bytes": ab}
+
+    # the scorer alone (axr_score) on the same cache, every table read mode, L2 flushed before each call
     scorer = {}
     if not args.no_scorer:
         sc_out = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
-        for mode in ("tensor", "factored", "table"):
+        for mode in ("mma", "tensor", "factored", "table"):
             ops.set_gather(mode)
             for _ in range(3):
                 ops.score(q, kc, kn, signs, bits, scale=1.0 / math.sqrt(d), out=sc_out)
@@ -292,7 +321,7 @@ def run_axr(args, w):
             ms = float(np.mean([a_.elapsed_time(b2) for a_, b2 in evs]))
             sbytes = (R + 2 + 4 * w.G) * B * Hkv * T
             scorer[mode] = {"ms": ms, "achieved_gbs": sbytes / (ms / 1e3) / 1e9, "algorithmic_bytes": sbytes}
-        ops.set_gather("factored")
+        ops.set_gather("mma")
         del sc_out
 
     # max over ranks
@@ -323,6 +352,7 @@ def run_axr(args, w):
         "e2e": {"value": key_heads / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "scorer": {m: dict(v_, frac=v_["achieved_gbs"] / _peaks()[0]) for m, v_ in scorer.items()},
+        "attend_variants": {m: dict(v_, frac=v_["achieved_gbs"] / _peaks()[0]) for m, v_ in variants.items()},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -363,6 +393,7 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch size (small ncu cases)")
     ap.add_argument("--no-scorer", action="store_true", help="skip the separate axr_score measurement")
+    ap.add_argument("--no-variants", action="store_true", help="skip the tiled-value attend variants")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

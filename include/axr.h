@@ -125,7 +125,7 @@ AXR_API axr_status axr_score(const float* q, const uint8_t* kcodes, const uint16
                      float* scores, void* stream);
 
 /*
- * Table read mode of axr_score (process-wide; default AXR_GATHER_FACTORED, the fastest on B200).  Every mode computes the same table
+ * Table read mode of axr_score (process-wide; default AXR_GATHER_MMA, the fastest on B200).  Every mode computes the same table
  * entries LUT[j][k] = scale * q~_j * c_k (AXELRAM Key Points, 2nd item) summed at each token's indices, and they agree
  * to within the score tolerance:
  *   AXR_GATHER_TABLE     the d x 2^b table (G heads wide) is materialised in shared memory and gathered entry by
@@ -136,10 +136,18 @@ AXR_API axr_status axr_score(const float* q, const uint8_t* kcodes, const uint16
  *   AXR_GATHER_TENSOR    the same factored table on the tensor cores: each token's gathered column factors (split
  *                        into hi and lo fp16 planes, about 22 bits) form a row of an MMA operand in tensor memory,
  *                        the row factors (split the same way) the other operand, and tcgen05.mma accumulates the
- *                        G sums per token in fp32.
- * axr_attend_decode always reads the table in factored form.  Errors: AXR_EINVAL for an unknown mode.
+ *                        G sums per token in fp32;
+ *   AXR_GATHER_MMA       the same hi/lo operands as warp-level MMAs (mma.sync, operands in registers): one table
+ *                        lookup gives a token's hi and lo registers for two coordinates.
+ * axr_attend_decode reads the key table in factored form; with tiled values the value product runs as warp-level
+ * MMAs, or, in AXR_GATHER_TENSOR mode, both products run as tcgen05 MMAs.  Errors: AXR_EINVAL for an unknown mode.
  */
-typedef enum axr_gather { AXR_GATHER_FACTORED = 0, AXR_GATHER_TABLE = 1, AXR_GATHER_TENSOR = 2 } axr_gather;
+typedef enum axr_gather {
+  AXR_GATHER_FACTORED = 0,
+  AXR_GATHER_TABLE = 1,
+  AXR_GATHER_TENSOR = 2,
+  AXR_GATHER_MMA = 3
+} axr_gather;
 AXR_API axr_status axr_set_gather(axr_gather mode);
 AXR_API axr_gather axr_get_gather(void);
 

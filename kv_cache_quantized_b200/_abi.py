@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libaxr.so")
 STATUS = {0: "AXR_OK", 1: "AXR_EINVAL", 2: "AXR_EUNSUPPORTED", 3: "AXR_ECUDA", 4: "AXR_EWORKSPACE"}
 F32, F16 = 0, 1
 V_F16, V_QUANT, V_QUANT_TILED = 0, 1, 2
-GATHER_FACTORED, GATHER_TABLE, GATHER_TENSOR = 0, 1, 2
+GATHER_FACTORED, GATHER_TABLE, GATHER_TENSOR, GATHER_MMA = 0, 1, 2, 3
 
 _p = ctypes.c_void_p
 _i = ctypes.c_int

@@ -5,6 +5,8 @@
 #include "decode.cuh"
 #include "score_tc.cuh"
 #include "attend_tcv.cuh"
+#include "attend_mma.cuh"
+#include "score_mma.cuh"
 
 namespace axr {
 namespace {
@@ -58,15 +60,40 @@ axr_status launch_attend_tcv(const DecodeArgs& a, cudaStream_t st) {
   return check_launch("axr_attend_decode");
 }
 
+template <int BITS, int G>
+axr_status launch_attend_mma(const DecodeArgs& a, cudaStream_t st) {
+  using S = MmaPlan<BITS, G>;
+  auto k1 = attend_mma_kernel<BITS, G>;
+  axr_status rs = ensure_smem(k1, S::bytes, "axr_attend_decode");
+  if (rs != AXR_OK) return rs;
+  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent blocks loop over the items
+  const long resident = static_cast<long>(S::MIN_BLOCKS) * kSmCount;
+  k1<<<static_cast<unsigned>(items < resident ? items : resident), kDecThreads, S::bytes, st>>>(a);
+  attend_reduce_kernel<128, true><<<a.B * a.Hq, 128, 0, st>>>(a);
+  return check_launch("axr_attend_decode");
+}
+
+template <int BITS, int G>
+axr_status launch_attend_tiled(const DecodeArgs& a, cudaStream_t st);
+
 template <int BITS>
 axr_status attend_tcv_g(int G, const DecodeArgs& a, cudaStream_t st) {
   switch (G) {
-    case 1: return launch_attend_tcv<BITS, 1>(a, st);
-    case 2: return launch_attend_tcv<BITS, 2>(a, st);
-    case 4: return launch_attend_tcv<BITS, 4>(a, st);
-    case 8: return launch_attend_tcv<BITS, 8>(a, st);
+    case 1: return launch_attend_tiled<BITS, 1>(a, st);
+    case 2: return launch_attend_tiled<BITS, 2>(a, st);
+    case 4: return launch_attend_tiled<BITS, 4>(a, st);
+    case 8: return launch_attend_tiled<BITS, 8>(a, st);
   }
   return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: G=%d", G);
+}
+
+std::atomic<int> g_gather{kGatherMma};
+
+// Tiled values: the tensor-core (tcgen05) kernel in AXR_GATHER_TENSOR mode, else warp-level MMAs for the values.
+template <int BITS, int G>
+axr_status launch_attend_tiled(const DecodeArgs& a, cudaStream_t st) {
+  if (g_gather.load() == kGatherTensor) return launch_attend_tcv<BITS, G>(a, st);
+  return launch_attend_mma<BITS, G>(a, st);
 }
 
 axr_status attend_tcv_bits(int bits, int G, const DecodeArgs& a, cudaStream_t st) {
@@ -79,7 +106,6 @@ axr_status attend_tcv_bits(int bits, int G, const DecodeArgs& a, cudaStream_t st
   return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: bits=%d", bits);
 }
 
-std::atomic<int> g_gather{kGatherFactored};
 
 template <int D, int BITS, int G>
 axr_status launch_score_tc(const DecodeArgs& a, cudaStream_t st) {
@@ -106,8 +132,21 @@ axr_status launch_score_mode(const DecodeArgs& a, cudaStream_t st) {
 }
 
 template <int D, int BITS, int G>
+axr_status launch_score_mma(const DecodeArgs& a, cudaStream_t st) {
+  using S = ScoreMmaPlan<D, BITS, G>;
+  auto k = score_mma_kernel<D, BITS, G>;
+  axr_status rs = ensure_smem(k, S::bytes, "axr_score");
+  if (rs != AXR_OK) return rs;
+  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent: two blocks per SM
+  const long resident = 2L * kSmCount;
+  k<<<static_cast<unsigned>(items < resident ? items : resident), S::THREADS, S::bytes, st>>>(a);
+  return check_launch("axr_score");
+}
+
+template <int D, int BITS, int G>
 axr_status launch_score(const DecodeArgs& a, cudaStream_t st) {
   const int mode = g_gather.load();
+  if (mode == kGatherMma) return launch_score_mma<D, BITS, G>(a, st);
   if (mode == kGatherTable) return launch_score_mode<D, BITS, G, kGatherTable>(a, st);
   if (mode == kGatherFactored) return launch_score_mode<D, BITS, G, kGatherFactored>(a, st);
   return launch_score_tc<D, BITS, G>(a, st);
@@ -296,12 +335,15 @@ extern "C" axr_status axr_set_gather(axr_gather mode) {
   if (mode == AXR_GATHER_FACTORED) g_gather.store(kGatherFactored);
   else if (mode == AXR_GATHER_TABLE) g_gather.store(kGatherTable);
   else if (mode == AXR_GATHER_TENSOR) g_gather.store(kGatherTensor);
+  else if (mode == AXR_GATHER_MMA) g_gather.store(kGatherMma);
   else return set_error(AXR_EINVAL, "axr_set_gather: unknown mode %d", (int)mode);
   return set_error(AXR_OK, "");
 }
 
 extern "C" axr_gather axr_get_gather(void) {
   const int m = axr::g_gather.load();
-  return m == axr::kGatherTable ? AXR_GATHER_TABLE : m == axr::kGatherFactored ? AXR_GATHER_FACTORED
-                                                                                : AXR_GATHER_TENSOR;
+  return m == axr::kGatherTable      ? AXR_GATHER_TABLE
+         : m == axr::kGatherFactored ? AXR_GATHER_FACTORED
+         : m == axr::kGatherMma      ? AXR_GATHER_MMA
+                                     : AXR_GATHER_TENSOR;
 }

@@ -26,7 +26,7 @@ constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / kWarp;
 constexpr float kLog2e = 1.4426950408889634f;
 
-enum Gather { kGatherFactored = 0, kGatherTable = 1, kGatherTensor = 2 };
+enum Gather { kGatherFactored = 0, kGatherTable = 1, kGatherTensor = 2, kGatherMma = 3 };
 
 struct DecodeArgs {
   const float* q;            // [B, Hq, D]
@@ -168,17 +168,22 @@ __device__ __forceinline__ uint64_t load_slice(const uint8_t* row, int sl) {
 template <int BITS, int J, int HG, int REPS = 32>
 __device__ __forceinline__ void factored_slice(uint64_t bits, const uint8_t* tab, uint32_t rep_off,
                                                const float2 (&qp)[HG][J / 2], float (&acc)[HG]) {
-  float2 a[HG];
+  // two accumulators per head (even and odd pairs) halve the dependent FMA chain
+  float2 a[2][HG];
 #pragma unroll
-  for (int h = 0; h < HG; ++h) a[h] = make_float2(0.f, 0.f);
+  for (int h = 0; h < HG; ++h) a[0][h] = a[1][h] = make_float2(0.f, 0.f);
+  float2 c[J / 2];
 #pragma unroll
-  for (int i = 0; i < J / 2; ++i) {
-    const float2 c = *reinterpret_cast<const float2*>(tab + pair_addr<BITS, REPS>(bits, i, rep_off));
+  for (int i = 0; i < J / 2; ++i) c[i] = *reinterpret_cast<const float2*>(tab + pair_addr<BITS, REPS>(bits, i, rep_off));
 #pragma unroll
-    for (int h = 0; h < HG; ++h) a[h] = fma2(qp[h][i], c, a[h]);
+  for (int i = 0; i < J / 2; ++i)
+#pragma unroll
+    for (int h = 0; h < HG; ++h) a[i & 1][h] = fma2(qp[h][i], c[i], a[i & 1][h]);
+#pragma unroll
+  for (int h = 0; h < HG; ++h) {
+    const float2 t = add2(a[0][h], a[1][h]);
+    acc[h] = t.x + t.y;
   }
-#pragma unroll
-  for (int h = 0; h < HG; ++h) acc[h] = a[h].x + a[h].y;
 }
 
 // ---- the decode partial kernel: persistent and warp-specialised ---------------------------------------------------

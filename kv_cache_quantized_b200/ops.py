@@ -177,12 +177,13 @@ def score(q, kcodes, knorms, signs, bits, scale=1.0, seq_lens=None, T=None, out=
     return out
 
 
-GATHER_MODES = {"tensor": _abi.GATHER_TENSOR, "factored": _abi.GATHER_FACTORED, "table": _abi.GATHER_TABLE}
+GATHER_MODES = {"tensor": _abi.GATHER_TENSOR, "factored": _abi.GATHER_FACTORED, "table": _abi.GATHER_TABLE,
+                "mma": _abi.GATHER_MMA}
 
 
 def set_gather(mode: str) -> None:
-    """Table read mode of score(): "factored" (default: packed fp32 FMAs), "tensor" (tensor cores) or "table"
-    (the materialised table, gathered per entry)."""
+    """Table read mode of score(): "mma" (default: warp-level MMAs on hi/lo fp16 operands), "factored" (packed fp32
+    FMAs), "tensor" (tcgen05 MMAs from tensor memory) or "table" (the materialised table, gathered per entry)."""
     _abi.check(_abi.lib().axr_set_gather(GATHER_MODES[mode]), "axr_set_gather")
 
 

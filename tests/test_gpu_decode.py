@@ -44,7 +44,7 @@ SMALL += [(128, 3, g, vq) for g in (1, 2, 8) for vq in (False, True)]
 SMALL += [(64, 4, g, False) for g in (1, 2, 8)]
 
 
-SCORE_CASES = [(d, b, g, "tensor") for d, b, g in sorted({(d, b, g) for d, b, g, _ in SMALL})]
+SCORE_CASES = [(d, b, g, m) for m in ("tensor", "mma") for d, b, g in sorted({(d, b, g) for d, b, g, _ in SMALL})]
 SCORE_CASES += [(d, b, g, m) for m in ("factored", "table") for d, b, g in [(128, 4, 4), (64, 3, 4), (128, 2, 8),
                                                                              (128, 1, 1)]]
 
@@ -53,7 +53,7 @@ SCORE_CASES += [(d, b, g, m) for m in ("factored", "table") for d, b, g in [(128
 def gather_mode(request):
     ops.set_gather(request.param)
     yield request.param
-    ops.set_gather("factored")
+    ops.set_gather("mma")
 
 
 @pytest.mark.parametrize("d,bits,G,gather_mode", SCORE_CASES, indirect=["gather_mode"])
