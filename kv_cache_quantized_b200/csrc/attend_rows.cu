@@ -1,0 +1,51 @@
+// Launcher of the row-layout decode kernel with MMA key scores (attend_rows.cuh).
+#include "attend_rows.cuh"
+#include "launch.h"
+
+namespace axr {
+namespace {
+
+template <int D, int BITS, int G, bool VQ>
+axr_status launch(const DecodeArgs& a, cudaStream_t st) {
+  using S = RowsPlan<D, BITS, G, VQ>;
+  auto k1 = attend_rows_kernel<D, BITS, G, VQ>;
+  axr_status rs = ensure_smem(k1, S::bytes, "axr_attend_decode");
+  if (rs != AXR_OK) return rs;
+  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent blocks loop over the items
+  const long resident = static_cast<long>(S::MIN_BLOCKS) * kSmCount;
+  k1<<<static_cast<unsigned>(items < resident ? items : resident), kDecThreads, S::bytes, st>>>(a);
+  attend_reduce_kernel<D, VQ><<<a.B * a.Hq, D, 0, st>>>(a);
+  return check_launch("axr_attend_decode");
+}
+
+template <int D, int BITS>
+axr_status by_g(int G, bool vq, const DecodeArgs& a, cudaStream_t st) {
+  switch (G) {
+    case 1: return vq ? launch<D, BITS, 1, true>(a, st) : launch<D, BITS, 1, false>(a, st);
+    case 2: return vq ? launch<D, BITS, 2, true>(a, st) : launch<D, BITS, 2, false>(a, st);
+    case 4: return vq ? launch<D, BITS, 4, true>(a, st) : launch<D, BITS, 4, false>(a, st);
+    case 8: return vq ? launch<D, BITS, 8, true>(a, st) : launch<D, BITS, 8, false>(a, st);
+  }
+  return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: G=%d", G);
+}
+
+template <int D>
+axr_status by_bits(int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st) {
+  switch (bits) {
+    case 1: return by_g<D, 1>(G, vq, a, st);
+    case 2: return by_g<D, 2>(G, vq, a, st);
+    case 3: return by_g<D, 3>(G, vq, a, st);
+    case 4: return by_g<D, 4>(G, vq, a, st);
+  }
+  return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: bits=%d", bits);
+}
+
+}  // namespace
+
+axr_status attend_rows_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st) {
+  if (d == 64) return by_bits<64>(bits, G, vq, a, st);
+  if (d == 128) return by_bits<128>(bits, G, vq, a, st);
+  return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: d=%d", d);
+}
+
+}  // namespace axr

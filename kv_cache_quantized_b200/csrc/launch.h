@@ -1,0 +1,37 @@
+// Host launchers of the decode kernel families.  Each family is compiled in a translation unit of its own (they
+// hold many template instances) and exposes one dispatcher over its runtime sizes; decode.cu validates the
+// arguments and picks the family.
+#pragma once
+
+#include "decode.cuh"
+
+namespace axr {
+
+// Raise the dynamic shared-memory limit of `kernel` to `bytes` when it is above the default 48 KB.
+template <typename K>
+axr_status ensure_smem(K kernel, size_t bytes, const char* what) {
+  if (bytes > 48 * 1024) {  // idempotent, and per device: set before every launch
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e != cudaSuccess) return set_error(AXR_ECUDA, "%s: cudaFuncSetAttribute: %s", what, cudaGetErrorString(e));
+  }
+  return AXR_OK;
+}
+
+// Row-layout cache, quantized keys scored through warp-level MMAs (attend_rows.cu); vq: values quantized.
+axr_status attend_rows_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st);
+
+// Row-layout cache on CUDA cores (attend_partial.cu): quantized keys through the factored gather, or fp16 keys
+// (dense; bits ignored).
+axr_status attend_partial_launch(int d, int bits, int G, bool vq, bool dense, const DecodeArgs& a, cudaStream_t st,
+                                 const char* what);
+
+// Tiled value layout, d = 128 (attend_tiled.cu): tcgen05 kernel if tensor, else warp-level MMAs.
+axr_status attend_tiled_launch(int bits, int G, bool tensor, const DecodeArgs& a, cudaStream_t st);
+
+// Scores only (score.cu): mode is one of kGatherTable, kGatherFactored, kGatherMma.
+axr_status score_launch(int d, int bits, int G, int mode, const DecodeArgs& a, cudaStream_t st);
+
+// Scores only on the tcgen05 tensor cores (score_tc.cu).
+axr_status score_tc_launch(int d, int bits, int G, const DecodeArgs& a, cudaStream_t st);
+
+}  // namespace axr

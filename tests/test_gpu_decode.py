@@ -49,6 +49,13 @@ SCORE_CASES += [(d, b, g, m) for m in ("factored", "table") for d, b, g in [(128
                                                                              (128, 1, 1)]]
 
 
+# the attend kernels follow the gather mode: "mma" (the default) scores keys through warp-level MMAs, "factored" on
+# CUDA cores
+ATTEND_CASES = [(d, b, g, vq, "mma") for d, b, g, vq in SMALL]
+ATTEND_CASES += [(d, b, g, vq, "factored") for d, b, g, vq in [(128, 4, 4, True), (128, 4, 4, False), (64, 3, 4, True),
+                                                                (128, 2, 8, False), (128, 1, 1, True)]]
+
+
 @pytest.fixture
 def gather_mode(request):
     ops.set_gather(request.param)
@@ -76,8 +83,8 @@ def test_score_matches_oracle(d, bits, G, gather_mode):
             assert np.all(np.isneginf(out[b, h, Tb:]))
 
 
-@pytest.mark.parametrize("d,bits,G,vq", SMALL)
-def test_attend_matches_oracle(d, bits, G, vq):
+@pytest.mark.parametrize("d,bits,G,vq,gather_mode", ATTEND_CASES, indirect=["gather_mode"])
+def test_attend_matches_oracle(d, bits, G, vq, gather_mode):
     B, Hkv, T, Tcap = 2, 2, 2500, 2600
     Hq = G * Hkv
     k, v, s, kc, kn, vc, vn = oracle_cache(B, Hkv, T, d, bits, 500 + d + bits + G, vq)
@@ -96,8 +103,9 @@ def test_attend_matches_oracle(d, bits, G, vq):
     parity.check_outputs(out.cpu().numpy(), want)
 
 
+@pytest.mark.parametrize("gather_mode", ["mma", "factored"], indirect=True)
 @pytest.mark.parametrize("vq", [False, True])
-def test_attend_edge_cases(vq):
+def test_attend_edge_cases(vq, gather_mode):
     d, bits, Hkv, G = 128, 4, 2, 4
     Hq = Hkv * G
     B, T, Tcap = 4, 300, 320
