@@ -36,6 +36,8 @@ struct RowsPlan {
   static constexpr int KCH = (R % 16 == 0) ? 16 : 8;
   static constexpr int STAGE_K = TT * R;
   static constexpr int STAGE_V = TT * VROW;
+  static constexpr int STAGE_N = 2 * TT * 2;              // key norms, then value norms (fp16)
+  static constexpr int STAGE_ALL = STAGE_K + STAGE_V + STAGE_N;
   static constexpr int NT = MmaB<D, G>::NT;
   static constexpr int TPR = D / 8;                       // fp16 values: value lanes per token row (8 coordinates)
   static constexpr int RPW = kWarp / TPR;                 // fp16 values: value rows per warp step
@@ -43,19 +45,20 @@ struct RowsPlan {
   static constexpr int PST = TT + 8;                      // quantized values: weight row stride (halves), padded
   static constexpr size_t PBUF = VQ ? 2 * 8 * (size_t)PST * 2 : 2 * (size_t)TT * G * 8;
   // everything but the stages
-  static constexpr size_t FIXED = (size_t)HiLoTable16<BITS>::BYTES + (size_t)G * D * 4 + PBUF +
+  static constexpr size_t FIXED = (size_t)HiLoTable16<BITS>::BYTES + (size_t)G * D * 4 + PBUF + 2 * 8 * 8 + 8 +
                                   2 * (size_t)KW * G * 4 + 2 * (size_t)KW * 4 + 2 * (size_t)KW * G * 4 + 16 * 4 + 128;
   static constexpr size_t kTwoBlocks = 112 * 1024;       // per-block budget for two resident blocks per SM
   // pipeline depth: NSTG - 1 tiles in flight per role; four stages where two blocks per SM still fit, else three,
   // and up to six for a single block per SM (fp16 values)
-  static constexpr int NSTG = FIXED + 4 * (size_t)(STAGE_K + STAGE_V) <= kTwoBlocks   ? 4
-                              : FIXED + 3 * (size_t)(STAGE_K + STAGE_V) <= kTwoBlocks ? 3
-                              : FIXED + 6 * (size_t)(STAGE_K + STAGE_V) <= 220 * 1024 ? 6
-                              : FIXED + 5 * (size_t)(STAGE_K + STAGE_V) <= 220 * 1024 ? 5
-                                                                                      : 4;
+  static constexpr int NSTG = FIXED + 4 * (size_t)STAGE_ALL <= kTwoBlocks   ? 4
+                              : FIXED + 3 * (size_t)STAGE_ALL <= kTwoBlocks ? 3
+                              : FIXED + 6 * (size_t)STAGE_ALL <= 220 * 1024 ? 6
+                              : FIXED + 5 * (size_t)STAGE_ALL <= 220 * 1024 ? 5
+                                                                            : 4;
   static constexpr size_t OFF_K = 0;                                         // [NSTG][STAGE_K], rows swizzled
   static constexpr size_t OFF_V = OFF_K + NSTG * (size_t)STAGE_K;            // [NSTG][STAGE_V]
-  static constexpr size_t STAGES_END = OFF_V + NSTG * (size_t)STAGE_V;
+  static constexpr size_t OFF_N = OFF_V + NSTG * (size_t)STAGE_V;            // [NSTG][2][TT] fp16 norms
+  static constexpr size_t STAGES_END = OFF_N + NSTG * (size_t)STAGE_N;
   static constexpr size_t REDUCE_BYTES = (size_t)NVG * G * D * 4;            // final sum, reuses the stages
   static constexpr size_t OFF_TAB = ((STAGES_END > REDUCE_BYTES ? STAGES_END : REDUCE_BYTES) + 127) / 128 * 128;
   static constexpr size_t OFF_QS = OFF_TAB + (size_t)HiLoTable16<BITS>::BYTES;  // [G][D] row factors
@@ -65,7 +68,11 @@ struct RowsPlan {
   static constexpr size_t OFF_RM = OFF_GR + 2 * (size_t)KW * 4;             // [KW][G] running max
   static constexpr size_t OFF_RL = OFF_RM + (size_t)KW * G * 4;             // [KW][G] running sum
   static constexpr size_t OFF_CENT = OFF_RL + (size_t)KW * G * 4;
-  static constexpr size_t bytes = OFF_CENT + 16 * 4;
+  static constexpr size_t OFF_MB = (OFF_CENT + 16 * 4 + 7) / 8 * 8;          // [2][NSTG] stage barriers, flag
+  static constexpr size_t bytes = OFF_MB + 2 * NSTG * 8 + 8;
+  // code and value tiles travel as one bulk copy each when rows are a multiple of 16 bytes (then nothing is
+  // swizzled), else as 8-byte cp.async chunks
+  static constexpr bool BULK = R % 16 == 0 && VROW % 16 == 0;
   static constexpr int MIN_BLOCKS = bytes <= kTwoBlocks ? 2 : 1;
   static_assert(bytes <= 227 * 1024, "shared memory of one block");
 };
@@ -93,9 +100,21 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
   const uint32_t rep16 = static_cast<uint32_t>(lane & 15) << 4;
   const float rd = rsqrtf(static_cast<float>(D));
 
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + P::OFF_MB);  // stage s holds its key tile
+  uint64_t* vfull = kfull + P::NSTG;                                  // stage s holds its value tile
+  volatile int* failed = reinterpret_cast<volatile int*>(kfull + 2 * P::NSTG);
   if (tid < 16) cent[tid] = a.cb.gamma[tid];
+  if (tid == 0) {
+    for (int s = 0; s < 2 * P::NSTG; ++s) tc::mbar_init(kfull + s, 1);
+    *failed = 0;
+  }
   __syncthreads();
   build_hilo_table16<BITS>(cent, smem + P::OFF_TAB);
+  // tiles of earlier items of this block: tile t of an item uses stage (done + t) % NSTG, and its barrier phase of
+  // parity ((done + t) / NSTG) & 1
+  int done = 0;
+  auto stg = [&](int tile) { return (done + tile) % P::NSTG; };
+  auto par = [&](int tile) { return static_cast<uint32_t>(((done + tile) / P::NSTG) & 1); };
 
   const int items = a.B * a.Hkv * a.splits;
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
@@ -109,7 +128,8 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
     const size_t kv_row0 = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
     const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
 
-    __syncthreads();  // the previous item is finished with the row factors, the stages and the merge region
+    fence_proxy_async();  // the merge region's generic writes come before the bulk copies that reuse it
+    __syncthreads();      // the previous item is finished with the row factors, the stages and the merge region
     transform_queries<D, G>(qg, a.signs, a.mult, qs);
     __syncthreads();
 
@@ -127,16 +147,20 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
       float m_run[NT], l_lane[NT];
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) { m_run[nt] = -INFINITY; l_lane[nt] = 0.f; }
-      // raw fp16 norms of token `lane` of the warp's share of a tile (key norm | value norm << 16), loaded one tile
-      // ahead and converted only when used, so that the load latency stays hidden behind a tile of work
-      const unsigned short* kn16 = reinterpret_cast<const unsigned short*>(a.knorms) + kv_row0;
-      const unsigned short* vn16 = VQ ? reinterpret_cast<const unsigned short*>(a.vnorms) + kv_row0 : nullptr;
+      // norms: staged with the codes when both norm rows start 16-byte aligned (cp.async), else raw fp16 values of
+      // token `lane` of the warp's share of a tile (key norm | value norm << 16) loaded one tile ahead into registers
+      // and converted only when used
+      const __half* kn_src = a.knorms + kv_row0;
+      const __half* vn_src = VQ ? a.vnorms + kv_row0 : nullptr;
+      const bool nrm_async = (reinterpret_cast<uintptr_t>(kn_src + start) & 15) == 0 &&
+                             (!VQ || (reinterpret_cast<uintptr_t>(vn_src + start) & 15) == 0);
+      __half* nst = reinterpret_cast<__half*>(smem + P::OFF_N);
       auto load_norms = [&](int tile) -> uint32_t {
         const int t = start + tile * TT + warp * WT + lane;
         uint32_t r = 0x3c00u << 16;  // value norm 1 for fp16 values
-        if (tile < ntiles && t < end) {
-          r = __ldg(kn16 + t);
-          if constexpr (VQ) r |= static_cast<uint32_t>(__ldg(vn16 + t)) << 16;
+        if (!nrm_async && tile < ntiles && t < end) {
+          r = __half_as_ushort(__ldg(kn_src + t));
+          if constexpr (VQ) r |= static_cast<uint32_t>(__half_as_ushort(__ldg(vn_src + t))) << 16;
           else r |= 0x3c00u << 16;
         }
         return r;
@@ -145,10 +169,23 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
       auto issue_k = [&](int tile) {
         if (tile < ntiles) {
           const int t0 = start + tile * TT;
-          const int bytes = min(TT, end - t0) * R;
-          uint8_t* dst = smem + P::OFF_K + (tile % P::NSTG) * P::STAGE_K;
+          const int n = min(TT, end - t0);
+          const int bytes = n * R;
+          uint8_t* dst = smem + P::OFF_K + stg(tile) * P::STAGE_K;
           const uint8_t* src = a.kcodes + (kv_row0 + t0) * R;
-          for (int o = rtid * P::KCH; o < bytes; o += 128 * P::KCH) cp_async<P::KCH>(dst + stage_swizzle<R>(o), src + o);
+          if constexpr (P::BULK) {
+            if (rtid == 0) {
+              mbar_arrive_expect_tx(kfull + stg(tile), bytes);
+              bulk_copy_g2s(dst, src, bytes, kfull + stg(tile));
+            }
+          } else {
+            for (int o = rtid * P::KCH; o < bytes; o += 128 * P::KCH) cp_async<P::KCH>(dst + o, src + o);
+          }
+          if (nrm_async) {
+            __half* nd = nst + stg(tile) * 2 * TT;
+            if (rtid < 16) stage_norms(nd, kn_src + t0, n, rtid);
+            else if (VQ && rtid < 32) stage_norms(nd + TT, vn_src + t0, n, rtid - 16);
+          }
         }
         cp_async_commit();
       };
@@ -160,21 +197,35 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
         if (it == ntiles) continue;
         const int t0 = start + it * TT;
         const int nt_tok = min(TT, end - t0);
-        const uint8_t* st = smem + P::OFF_K + (it % P::NSTG) * P::STAGE_K;
-        const uint32_t nrm = nrm_next;
-        nrm_next = load_norms(it + 1);
+        const uint8_t* st = smem + P::OFF_K + stg(it) * P::STAGE_K;
+        if constexpr (P::BULK) {
+          if (!tc::mbar_wait(kfull + stg(it), par(it))) *failed = 1;
+        }
         float kn[2][2], vn[2][2];
+        if (nrm_async) {
+          const __half* nk = nst + stg(it) * 2 * TT + warp * WT + gq;
 #pragma unroll
-        for (int m = 0; m < 2; ++m)
+          for (int m = 0; m < 2; ++m)
 #pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const uint32_t x = __shfl_sync(0xffffffffu, nrm, 16 * m + gq + 8 * i);
-            kn[m][i] = __half2float(__ushort_as_half(static_cast<unsigned short>(x & 0xffffu)));
-            vn[m][i] = __half2float(__ushort_as_half(static_cast<unsigned short>(x >> 16)));
-          }
+            for (int i = 0; i < 2; ++i) {
+              kn[m][i] = __half2float(nk[16 * m + 8 * i]);
+              vn[m][i] = VQ ? __half2float(nk[TT + 16 * m + 8 * i]) : 1.f;
+            }
+        } else {
+          const uint32_t nrm = nrm_next;
+          nrm_next = load_norms(it + 1);
+#pragma unroll
+          for (int m = 0; m < 2; ++m)
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const uint32_t x = __shfl_sync(0xffffffffu, nrm, 16 * m + gq + 8 * i);
+              kn[m][i] = __half2float(__ushort_as_half(static_cast<unsigned short>(x & 0xffffu)));
+              vn[m][i] = __half2float(__ushort_as_half(static_cast<unsigned short>(x >> 16)));
+            }
+        }
         float z[2][NT][2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) mma_scores16<D, BITS, G>(st, warp * WT + 16 * m, tab, rep16, B, lane, z[m]);
+        for (int m = 0; m < 2; ++m) mma_scores16<D, BITS, G, false>(st, warp * WT + 16 * m, tab, rep16, B, lane, z[m]);
         // online softmax over this warp's 32 tokens; lane (gq, tq) holds head 4 nt + tq
         bool grew = false;
 #pragma unroll
@@ -200,8 +251,9 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
             for (int i = 0; i < 2; ++i) {
               const float p = (z[m][nt][i] == -INFINITY) ? 0.f : exp2f(z[m][nt][i] - m_new);
               psum += p;
-              // weight of the value product: p n^V (quantized values also carry the centroid scale 1/sqrt(d))
-              const float pv = p * (VQ ? vn[m][i] * rd : 1.f);
+              // weight of the value product: p n^V (quantized values also carry the centroid scale 1/sqrt(d));
+              // tokens past the end get 0 whatever their staged norm holds
+              const float pv = p > 0.f ? p * (VQ ? vn[m][i] * rd : 1.f) : 0.f;
               if (h < G) {
                 const int tok = warp * WT + 16 * m + gq + 8 * i;
                 if constexpr (VQ) pbuf16[((it & 1) * 8 + h) * P::PST + tok] = __float2half_rn(pv);
@@ -256,9 +308,16 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
         if (tile < ntiles) {
           const int t0 = start + tile * TT;
           const int bytes = min(TT, end - t0) * R;
-          uint8_t* dst = smem + P::OFF_V + (tile % P::NSTG) * P::STAGE_V;
+          uint8_t* dst = smem + P::OFF_V + stg(tile) * P::STAGE_V;
           const uint8_t* src = vsrc + (kv_row0 + t0) * R;
-          for (int o = rtid * P::KCH; o < bytes; o += 128 * P::KCH) cp_async<P::KCH>(dst + stage_swizzle<R>(o), src + o);
+          if constexpr (P::BULK) {
+            if (rtid == 0) {
+              mbar_arrive_expect_tx(vfull + stg(tile), bytes);
+              bulk_copy_g2s(dst, src, bytes, vfull + stg(tile));
+            }
+          } else {
+            for (int o = rtid * P::KCH; o < bytes; o += 128 * P::KCH) cp_async<P::KCH>(dst + o, src + o);
+          }
         }
         cp_async_commit();
       };
@@ -279,7 +338,10 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
             acc[mt][0] *= al0; acc[mt][1] *= al1; acc[mt][2] *= al0; acc[mt][3] *= al1;
           }
         }
-        const uint8_t* vst = smem + P::OFF_V + (j % P::NSTG) * P::STAGE_V;
+        const uint8_t* vst = smem + P::OFF_V + stg(j) * P::STAGE_V;
+        if constexpr (P::BULK) {
+          if (!tc::mbar_wait(vfull + stg(j), par(j))) *failed = 1;
+        }
         const __half* pw = pbuf16 + pb * 8 * P::PST;
 #pragma unroll
         for (int kt = 0; kt < WT / 16; ++kt) {
@@ -292,10 +354,10 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
             b1 = *reinterpret_cast<const uint32_t*>(pw + g * P::PST + k0 + 8);
           }
           uint32_t w[4][NWV];
-          load_run<R, NBV>(vst, (k0 + tf) * R + g * NBV, w[0]);
-          load_run<R, NBV>(vst, (k0 + 1 - tf) * R + g * NBV, w[1]);
-          load_run<R, NBV>(vst, (k0 + 8 + tf) * R + g * NBV, w[2]);
-          load_run<R, NBV>(vst, (k0 + 9 - tf) * R + g * NBV, w[3]);
+          load_run<R, NBV, false>(vst, (k0 + tf) * R + g * NBV, w[0]);
+          load_run<R, NBV, false>(vst, (k0 + 1 - tf) * R + g * NBV, w[1]);
+          load_run<R, NBV, false>(vst, (k0 + 8 + tf) * R + g * NBV, w[2]);
+          load_run<R, NBV, false>(vst, (k0 + 9 - tf) * R + g * NBV, w[3]);
 #pragma unroll
           for (int r = 0; r < 4; ++r)
 #pragma unroll
@@ -343,8 +405,17 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
       auto issue_v = [&](int tile) {
         if (tile < ntiles) {
           const int t0 = start + tile * TT;
-          role_copy_async<P::VCH>(smem + P::OFF_V + (tile % P::NSTG) * P::STAGE_V, vsrc + (kv_row0 + t0) * P::VROW,
-                                  min(TT, end - t0) * P::VROW, rtid);
+          uint8_t* dst = smem + P::OFF_V + stg(tile) * P::STAGE_V;
+          const uint8_t* src = vsrc + (kv_row0 + t0) * P::VROW;
+          const int bytes = min(TT, end - t0) * P::VROW;
+          if constexpr (P::BULK) {
+            if (rtid == 0) {
+              mbar_arrive_expect_tx(vfull + stg(tile), bytes);
+              bulk_copy_g2s(dst, src, bytes, vfull + stg(tile));
+            }
+          } else {
+            role_copy_async<P::VCH>(dst, src, bytes, rtid);
+          }
         }
         cp_async_commit();
       };
@@ -365,7 +436,10 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
             for (int c = 0; c < 4; ++c) { acc[g][c].x *= al; acc[g][c].y *= al; }
           }
         }
-        const uint8_t* vst = smem + P::OFF_V + (j % P::NSTG) * P::STAGE_V;
+        const uint8_t* vst = smem + P::OFF_V + stg(j) * P::STAGE_V;
+        if constexpr (P::BULK) {
+          if (!tc::mbar_wait(vfull + stg(j), par(j))) *failed = 1;
+        }
         const float2* prow = pbuf + static_cast<size_t>(pb) * TT * G;
 #pragma unroll 2
         for (int i = 0; i < WT / RPW; ++i) {
@@ -418,8 +492,10 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
 #pragma unroll
       for (int w2 = 0; w2 < KW; ++w2) s += red_l[w2 * G + tid];
       a.ws_l[part0 + static_cast<size_t>(tid) * a.splits] = s;
-      a.ws_m[part0 + static_cast<size_t>(tid) * a.splits] = M;
+      // a stage that never arrived (a copy that did not complete in about a second) poisons the output
+      a.ws_m[part0 + static_cast<size_t>(tid) * a.splits] = *failed ? __int_as_float(0x7fc00000) : M;
     }
+    done += ntiles;
   }
 }
 

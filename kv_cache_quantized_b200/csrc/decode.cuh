@@ -67,7 +67,36 @@ __device__ __forceinline__ void cp_async(void* dst, const void* src) {
   else
     asm volatile("cp.async.ca.shared.global [%0], [%1], %2;\n" ::"r"(smem_u32(dst)), "l"(src), "n"(BYTES));
 }
+// 16-byte copy that reads only the first src_bytes (1..16) of src and zero-fills the rest of dst.
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes));
+}
+
+// Stage the fp16 norms of tokens [0, n) of a tile (n <= 128, src 16-byte aligned) as 16-byte chunks of 8 tokens,
+// the last one zero-filled past n: the chunk of thread c (c < 16) of the copying group.
+__device__ __forceinline__ void stage_norms(__half* dst, const __half* src, int n, int c) {
+  const int tok0 = 8 * c;
+  if (c < 16 && tok0 < n) cp_async16_zfill(dst + tok0, src + tok0, min(16, 2 * (n - tok0)));
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+
+// Bulk (TMA engine) copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global to this CTA's
+// shared memory, completing on `mbar` as transaction bytes; the caller has armed the barrier with expect_tx.
+__device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* mbar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(mbar))
+               : "memory");
+}
+
+// Arrive once on `mbar` and add `bytes` to the transaction count of its current phase.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(bytes)
+               : "memory");
+}
+
+// Order this thread's generic-proxy accesses to shared memory before later async-proxy (bulk copy) accesses.
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;\n" ::"n"(N)); }
 

@@ -54,11 +54,11 @@ __device__ __forceinline__ uint32_t hilo_off16(const uint32_t* w, int i, uint32_
     return (bits_at<2 * BITS>(w, 2 * BITS * i) << 7) | (rep16 >> 1);
 }
 
-// The NB bytes at byte offset `off` of a staged tile (rows swizzled with stage_swizzle<R>; NB divides R and the run
-// stays inside one 16-byte chunk) into w[0 .. ceil(NB / 4)).
-template <int R, int NB>
+// The NB bytes at byte offset `off` of a staged tile (rows swizzled with stage_swizzle<R> if SWZ; the run stays
+// inside one 16-byte chunk) into w[0 .. ceil(NB / 4)).
+template <int R, int NB, bool SWZ = true>
 __device__ __forceinline__ void load_run(const uint8_t* stage, int off, uint32_t* w) {
-  const uint8_t* p = stage + stage_swizzle<R>(off);
+  const uint8_t* p = stage + (SWZ ? stage_swizzle<R>(off) : off);
   if constexpr (NB == 16) {
     const uint4 u = *reinterpret_cast<const uint4*>(p);
     w[0] = u.x; w[1] = u.y; w[2] = u.z; w[3] = u.w;
@@ -138,8 +138,8 @@ __device__ __forceinline__ void mma_b_build(const float* __restrict__ qs, const 
 }
 
 // Scaled scores (times s_h) of tokens r0 = row0 + g and r1 = r0 + 8 of a staged tile of packed rows (swizzled with
-// stage_swizzle<R>), for head 4 nt + t: out[nt][0] for r0, out[nt][1] for r1.
-template <int D, int BITS, int G>
+// stage_swizzle<R> if SWZ), for head 4 nt + t: out[nt][0] for r0, out[nt][1] for r1.
+template <int D, int BITS, int G, bool SWZ = true>
 __device__ __forceinline__ void mma_scores16(const uint8_t* st, int row0, const uint8_t* tab, uint32_t rep16,
                                              const MmaB<D, G>& B, int lane, float (&out)[MmaB<D, G>::NT][2]) {
   constexpr int R = D * BITS / 8, KT = MmaB<D, G>::KT, NT = MmaB<D, G>::NT;
@@ -147,8 +147,8 @@ __device__ __forceinline__ void mma_scores16(const uint8_t* st, int row0, const 
   constexpr int NW = (NB + 3) / 4 + 1;    // its words, plus a zero word
   const int gq = lane >> 2, tq = lane & 3;
   uint32_t w0[NW], w1[NW];
-  load_run<R, NB>(st, (row0 + gq) * R + tq * NB, w0);
-  load_run<R, NB>(st, (row0 + gq + 8) * R + tq * NB, w1);
+  load_run<R, NB, SWZ>(st, (row0 + gq) * R + tq * NB, w0);
+  load_run<R, NB, SWZ>(st, (row0 + gq + 8) * R + tq * NB, w1);
 #pragma unroll
   for (int i = (NB + 3) / 4; i < NW; ++i) w0[i] = w1[i] = 0u;
   float c[2][NT][4];

@@ -30,7 +30,8 @@ struct ScoreMmaPlan {
   static constexpr int STAGE = TT * R;
   static constexpr int NST = 5;                   // code stages: four tiles in flight per block
   static constexpr size_t OFF_STAGE = 0;
-  static constexpr size_t OFF_TAB = ((size_t)NST * STAGE + 255) / 256 * 256;
+  static constexpr size_t OFF_NRM = (size_t)NST * STAGE;                    // [NST][TT] fp16 key norms
+  static constexpr size_t OFF_TAB = (OFF_NRM + (size_t)NST * TT * 2 + 255) / 256 * 256;
   static constexpr size_t OFF_QS = OFF_TAB + tc::PairTable16<BITS>::BYTES;
   static constexpr size_t OFF_CENT = OFF_QS + (size_t)G * D * 4;
   static constexpr size_t bytes = OFF_CENT + 16 * 4;
@@ -93,13 +94,19 @@ __global__ void __launch_bounds__(256, 2) score_mma_kernel(const __grid_constant
     const int ntiles = vend > start ? (vend - start + TT - 1) / TT : 0;
 
     __syncthreads();  // the previous item is finished with the stages and the row factors
+    // key norms ride with the codes when the item's norm row starts 16-byte aligned, else each lane loads its two
+    const __half* kn_src = a.knorms + kv_row0;
+    const bool nrm_async = (reinterpret_cast<uintptr_t>(kn_src + start) & 15) == 0;
+    __half* nst = reinterpret_cast<__half*>(smem + P::OFF_NRM);
     auto issue_tile = [&](int tile) {
       if (tile < ntiles) {
         uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(tile % NST) * P::STAGE;
         const int t0 = start + tile * TT;
-        const int bytes = min(TT, vend - t0) * R;
+        const int n = min(TT, vend - t0);
+        const int bytes = n * R;
         const uint8_t* src = a.kcodes + (kv_row0 + t0) * R;
         for (int o = tid * P::KCH; o < bytes; o += P::THREADS * P::KCH) cp_async<P::KCH>(st + stage_swizzle<R>(o), src + o);
+        if (nrm_async && tid < 16) stage_norms(nst + (tile % NST) * TT, kn_src + t0, n, tid);
       }
       cp_async_commit();
     };
@@ -166,8 +173,14 @@ __global__ void __launch_bounds__(256, 2) score_mma_kernel(const __grid_constant
         }
       }
       w0[R / 4] = w1[R / 4] = 0u;
-      const float kn0 = r0 < nt_tok ? __half2float(a.knorms[kv_row0 + t0 + r0]) : 0.f;
-      const float kn1 = r1 < nt_tok ? __half2float(a.knorms[kv_row0 + t0 + r1]) : 0.f;
+      float kn0, kn1;
+      if (nrm_async) {
+        kn0 = __half2float(nst[(tile % NST) * TT + r0]);
+        kn1 = __half2float(nst[(tile % NST) * TT + r1]);
+      } else {
+        kn0 = r0 < nt_tok ? __half2float(kn_src[t0 + r0]) : 0.f;
+        kn1 = r1 < nt_tok ? __half2float(kn_src[t0 + r1]) : 0.f;
+      }
       float c[2][NT][4];  // two accumulator chains (even / odd K-tiles)
 #pragma unroll
       for (int x = 0; x < 2; ++x)

@@ -126,6 +126,33 @@ def test_attend_edge_cases(vq, gather_mode):
     assert np.all(out0 == 0.0)
 
 
+@pytest.mark.parametrize("vq", [False, True])
+def test_unaligned_norm_rows(vq):
+    """An odd cache capacity leaves most norm rows off 16-byte alignment: the kernels then load norms per lane
+    instead of staging them with the codes; scores and outputs stay the same."""
+    d, bits, Hkv, G = 128, 4, 3, 4
+    Hq = Hkv * G
+    B, T, Tcap = 2, 1000, 1003
+    k, v, s, kc, kn, vc, vn = oracle_cache(B, Hkv, T, d, bits, 750, vq)
+    q = W.normal((B, Hq, d), 751, np.float32)
+    lens = np.array([1000, 613], np.int32)
+    vargs = dict(vcodes=cuda(padded(vc, Tcap)), vnorms=cuda(padded(vn, Tcap))) if vq else dict(v=cuda(padded(v, Tcap)))
+    out = ops.attend_decode(cuda(q), cuda(padded(kc, Tcap)), cuda(padded(kn, Tcap)), cuda(s), bits, seq_lens=cuda(lens),
+                            T=T, **vargs).cpu().numpy()
+    okw = dict(vcodes=vc, vn16=vn) if vq else dict(v=v)
+    parity.check_outputs(out, oracle.decode_attention(q, kc, kn, s, bits, 1 / math.sqrt(d), seq_lens=lens, **okw))
+    if not vq:
+        sc = ops.score(cuda(q), cuda(padded(kc, Tcap)), cuda(padded(kn, Tcap)), cuda(s), bits, scale=0.5,
+                       seq_lens=cuda(lens), T=T).cpu().numpy()
+        for b in range(B):
+            for h in range(Hq):
+                Tb = lens[b]
+                want = oracle.score_lut(q[b, h], kc[b, h // G, :Tb], kn[b, h // G, :Tb], s, bits, 0.5)
+                A = parity.abs_score_scale(q[b, h].astype(np.float64), kc[b, h // G, :Tb], kn[b, h // G, :Tb], s,
+                                           bits, 0.5)
+                parity.check_scores(sc[b, h, :Tb], want, A)
+
+
 def test_dense_matches_oracle_attention():
     B, Hkv, G, T, Tcap, d = 3, 2, 4, 2100, 2200, 128
     k = W.lognormal_rows((B, Hkv, T, d), 800, dtype=np.float16)
