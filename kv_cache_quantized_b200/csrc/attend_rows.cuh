@@ -36,40 +36,48 @@ struct RowsPlan {
   static constexpr int KCH = (R % 16 == 0) ? 16 : 8;
   static constexpr int STAGE_K = TT * R;
   static constexpr int STAGE_V = TT * VROW;
-  static constexpr int STAGE_N = 2 * TT * 2;              // key norms, then value norms (fp16)
-  static constexpr int STAGE_ALL = STAGE_K + STAGE_V + STAGE_N;
+  static constexpr int STAGE_N = 2 * TT * 2;              // key norms, then value norms (fp16), with the key tile
   static constexpr int NT = MmaB<D, G>::NT;
   static constexpr int TPR = D / 8;                       // fp16 values: value lanes per token row (8 coordinates)
   static constexpr int RPW = kWarp / TPR;                 // fp16 values: value rows per warp step
   static constexpr int NVG = VQ ? KW : KW * RPW;          // value partial sums, summed at the end
   static constexpr int PST = TT + 8;                      // quantized values: weight row stride (halves), padded
   static constexpr size_t PBUF = VQ ? 2 * 8 * (size_t)PST * 2 : 2 * (size_t)TT * G * 8;
+  static constexpr size_t TAB = (size_t)PairTableKV<BITS>::BYTES;
   // everything but the stages
-  static constexpr size_t FIXED = (size_t)HiLoTable16<BITS>::BYTES + (size_t)G * D * 4 + PBUF + 2 * 8 * 8 + 8 +
-                                  2 * (size_t)KW * G * 4 + 2 * (size_t)KW * 4 + 2 * (size_t)KW * G * 4 + 16 * 4 + 128;
-  static constexpr size_t kTwoBlocks = 112 * 1024;       // per-block budget for two resident blocks per SM
-  // pipeline depth: NSTG - 1 tiles in flight per role; four stages where two blocks per SM still fit, else three,
-  // and up to six for a single block per SM (fp16 values)
-  static constexpr int NSTG = FIXED + 4 * (size_t)STAGE_ALL <= kTwoBlocks   ? 4
-                              : FIXED + 3 * (size_t)STAGE_ALL <= kTwoBlocks ? 3
-                              : FIXED + 6 * (size_t)STAGE_ALL <= 220 * 1024 ? 6
-                              : FIXED + 5 * (size_t)STAGE_ALL <= 220 * 1024 ? 5
-                                                                            : 4;
-  static constexpr size_t OFF_K = 0;                                         // [NSTG][STAGE_K], rows swizzled
-  static constexpr size_t OFF_V = OFF_K + NSTG * (size_t)STAGE_K;            // [NSTG][STAGE_V]
-  static constexpr size_t OFF_N = OFF_V + NSTG * (size_t)STAGE_V;            // [NSTG][2][TT] fp16 norms
-  static constexpr size_t STAGES_END = OFF_N + NSTG * (size_t)STAGE_N;
+  static constexpr size_t FIXED = TAB + PBUF + 2 * 8 * 8 + 8 + 2 * (size_t)KW * G * 4 +
+                                  2 * (size_t)KW * 4 + 2 * (size_t)KW * G * 4 + 16 * 4 + 128;
+  static constexpr size_t kTwoBlocks = 113 * 1024;       // per-block budget for two resident blocks per SM
+  static constexpr size_t need(int nk, int nv) {
+    return FIXED + (size_t)nk * (STAGE_K + STAGE_N) + (size_t)nv * STAGE_V;
+  }
+  // stage depths (key tiles with their norms, value tiles): NSK - 1 key tiles in flight ahead of the scoring warps
+  // and NSV - 1 value tiles ahead of the value warps; the deepest pair that keeps two blocks per SM, else a single
+  // block per SM (fp16 values) with deeper stages
+  static constexpr int PICK = need(4, 3) <= kTwoBlocks   ? 43
+                              : need(3, 3) <= kTwoBlocks ? 33
+                              : need(3, 2) <= kTwoBlocks ? 32
+                              : need(5, 4) <= 220 * 1024 ? 54
+                              : need(4, 3) <= 220 * 1024 ? 43
+                                                         : 32;
+  static constexpr int NSK = PICK / 10, NSV = PICK % 10;
+  static constexpr size_t OFF_K = 0;                                         // [NSK][STAGE_K]
+  static constexpr size_t OFF_V = OFF_K + NSK * (size_t)STAGE_K;             // [NSV][STAGE_V]
+  static constexpr size_t OFF_N = OFF_V + NSV * (size_t)STAGE_V;             // [NSK][2][TT] fp16 norms
+  static constexpr size_t STAGES_END = OFF_N + NSK * (size_t)STAGE_N;
   static constexpr size_t REDUCE_BYTES = (size_t)NVG * G * D * 4;            // final sum, reuses the stages
   static constexpr size_t OFF_TAB = ((STAGES_END > REDUCE_BYTES ? STAGES_END : REDUCE_BYTES) + 127) / 128 * 128;
-  static constexpr size_t OFF_QS = OFF_TAB + (size_t)HiLoTable16<BITS>::BYTES;  // [G][D] row factors
-  static constexpr size_t OFF_P = OFF_QS + (size_t)G * D * 4;               // [2][8][PST] fp16 or [2][TT][G] float2
+  // [G][D] row factors: read only while an item starts, before the first value tile is issued into the stages
+  static constexpr size_t OFF_QS = OFF_V;
+  static_assert((size_t)NSV * STAGE_V >= (size_t)G * D * 4, "row factors fit the value stages");
+  static constexpr size_t OFF_P = OFF_TAB + TAB;                             // [2][8][PST] fp16 or [2][TT][G] float2
   static constexpr size_t OFF_AL = OFF_P + PBUF;                             // [2][KW][G] rescale factors
   static constexpr size_t OFF_GR = OFF_AL + 2 * (size_t)KW * G * 4;         // [2][KW] rescale flags
   static constexpr size_t OFF_RM = OFF_GR + 2 * (size_t)KW * 4;             // [KW][G] running max
   static constexpr size_t OFF_RL = OFF_RM + (size_t)KW * G * 4;             // [KW][G] running sum
   static constexpr size_t OFF_CENT = OFF_RL + (size_t)KW * G * 4;
-  static constexpr size_t OFF_MB = (OFF_CENT + 16 * 4 + 7) / 8 * 8;          // [2][NSTG] stage barriers, flag
-  static constexpr size_t bytes = OFF_MB + 2 * NSTG * 8 + 8;
+  static constexpr size_t OFF_MB = (OFF_CENT + 16 * 4 + 7) / 8 * 8;          // [NSK + NSV] stage barriers, flag
+  static constexpr size_t bytes = OFF_MB + (NSK + NSV) * 8 + 8;
   // code and value tiles travel as one bulk copy each when rows are a multiple of 16 bytes (then nothing is
   // swizzled), else as 8-byte cp.async chunks
   static constexpr bool BULK = R % 16 == 0 && VROW % 16 == 0;
@@ -97,24 +105,27 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const bool scorer = warp < KW;
   const int rtid = scorer ? tid : tid - 128;  // thread index within the role
-  const uint32_t rep16 = static_cast<uint32_t>(lane & 15) << 4;
+  const uint32_t repk = static_cast<uint32_t>(lane & 15) << 3;  // the lane's hi/lo copy in the pair table
+  const uint32_t repv = 128u + (static_cast<uint32_t>(lane) << 2);  // its hi-only copy
   const float rd = rsqrtf(static_cast<float>(D));
 
-  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + P::OFF_MB);  // stage s holds its key tile
-  uint64_t* vfull = kfull + P::NSTG;                                  // stage s holds its value tile
-  volatile int* failed = reinterpret_cast<volatile int*>(kfull + 2 * P::NSTG);
+  uint64_t* kfull = reinterpret_cast<uint64_t*>(smem + P::OFF_MB);  // key stage s holds its tile
+  uint64_t* vfull = kfull + P::NSK;                                   // value stage s holds its tile
+  volatile int* failed = reinterpret_cast<volatile int*>(vfull + P::NSV);
   if (tid < 16) cent[tid] = a.cb.gamma[tid];
   if (tid == 0) {
-    for (int s = 0; s < 2 * P::NSTG; ++s) tc::mbar_init(kfull + s, 1);
+    for (int s = 0; s < P::NSK + P::NSV; ++s) tc::mbar_init(kfull + s, 1);
     *failed = 0;
   }
   __syncthreads();
-  build_hilo_table16<BITS>(cent, smem + P::OFF_TAB);
-  // tiles of earlier items of this block: tile t of an item uses stage (done + t) % NSTG, and its barrier phase of
-  // parity ((done + t) / NSTG) & 1
+  build_pair_table_kv<BITS>(cent, smem + P::OFF_TAB);
+  // tiles of earlier items of this block: tile t of an item uses key stage (done + t) % NSK and value stage
+  // (done + t) % NSV, and barrier phases of parity ((done + t) / NS) & 1
   int done = 0;
-  auto stg = [&](int tile) { return (done + tile) % P::NSTG; };
-  auto par = [&](int tile) { return static_cast<uint32_t>(((done + tile) / P::NSTG) & 1); };
+  auto kstg = [&](int tile) { return (done + tile) % P::NSK; };
+  auto kpar = [&](int tile) { return static_cast<uint32_t>(((done + tile) / P::NSK) & 1); };
+  auto vstg = [&](int tile) { return (done + tile) % P::NSV; };
+  auto vpar = [&](int tile) { return static_cast<uint32_t>(((done + tile) / P::NSV) & 1); };
 
   const int items = a.B * a.Hkv * a.splits;
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
@@ -131,6 +142,7 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
     fence_proxy_async();  // the merge region's generic writes come before the bulk copies that reuse it
     __syncthreads();      // the previous item is finished with the row factors, the stages and the merge region
     transform_queries<D, G>(qg, a.signs, a.mult, qs);
+    fence_proxy_async();  // the row factors share memory with the value stages, refilled by bulk copies
     __syncthreads();
 
     if (scorer) {
@@ -171,39 +183,39 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
           const int t0 = start + tile * TT;
           const int n = min(TT, end - t0);
           const int bytes = n * R;
-          uint8_t* dst = smem + P::OFF_K + stg(tile) * P::STAGE_K;
+          uint8_t* dst = smem + P::OFF_K + kstg(tile) * P::STAGE_K;
           const uint8_t* src = a.kcodes + (kv_row0 + t0) * R;
           if constexpr (P::BULK) {
             if (rtid == 0) {
-              mbar_arrive_expect_tx(kfull + stg(tile), bytes);
-              bulk_copy_g2s(dst, src, bytes, kfull + stg(tile));
+              mbar_arrive_expect_tx(kfull + kstg(tile), bytes);
+              bulk_copy_g2s(dst, src, bytes, kfull + kstg(tile));
             }
           } else {
             for (int o = rtid * P::KCH; o < bytes; o += 128 * P::KCH) cp_async<P::KCH>(dst + o, src + o);
           }
           if (nrm_async) {
-            __half* nd = nst + stg(tile) * 2 * TT;
+            __half* nd = nst + kstg(tile) * 2 * TT;
             if (rtid < 16) stage_norms(nd, kn_src + t0, n, rtid);
             else if (VQ && rtid < 32) stage_norms(nd + TT, vn_src + t0, n, rtid - 16);
           }
         }
         cp_async_commit();
       };
-      for (int s = 0; s < P::NSTG - 1; ++s) issue_k(s);
+      for (int s = 0; s < P::NSK - 1; ++s) issue_k(s);
       for (int it = 0; it <= ntiles; ++it) {
-        cp_async_wait<P::NSTG - 2>();  // tile it has landed; the next NSTG - 2 may still be in flight
+        cp_async_wait<P::NSK - 2>();  // tile it's norms have landed; the next NSK - 2 may still be in flight
         roles_sync();
-        issue_k(it + P::NSTG - 1);     // into the stage tile it - 1 used
+        issue_k(it + P::NSK - 1);     // into the stage tile it - 1 used
         if (it == ntiles) continue;
         const int t0 = start + it * TT;
         const int nt_tok = min(TT, end - t0);
-        const uint8_t* st = smem + P::OFF_K + stg(it) * P::STAGE_K;
+        const uint8_t* st = smem + P::OFF_K + kstg(it) * P::STAGE_K;
         if constexpr (P::BULK) {
-          if (!tc::mbar_wait(kfull + stg(it), par(it))) *failed = 1;
+          if (!tc::mbar_wait(kfull + kstg(it), kpar(it))) *failed = 1;
         }
         float kn[2][2], vn[2][2];
         if (nrm_async) {
-          const __half* nk = nst + stg(it) * 2 * TT + warp * WT + gq;
+          const __half* nk = nst + kstg(it) * 2 * TT + warp * WT + gq;
 #pragma unroll
           for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -225,7 +237,7 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
         }
         float z[2][NT][2];
 #pragma unroll
-        for (int m = 0; m < 2; ++m) mma_scores16<D, BITS, G, false>(st, warp * WT + 16 * m, tab, rep16, B, lane, z[m]);
+        for (int m = 0; m < 2; ++m) mma_scores16<D, BITS, G, false, true>(st, warp * WT + 16 * m, tab, repk, B, lane, z[m]);
         // online softmax over this warp's 32 tokens; lane (gq, tq) holds head 4 nt + tq
         bool grew = false;
 #pragma unroll
@@ -308,12 +320,12 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
         if (tile < ntiles) {
           const int t0 = start + tile * TT;
           const int bytes = min(TT, end - t0) * R;
-          uint8_t* dst = smem + P::OFF_V + stg(tile) * P::STAGE_V;
+          uint8_t* dst = smem + P::OFF_V + vstg(tile) * P::STAGE_V;
           const uint8_t* src = vsrc + (kv_row0 + t0) * R;
           if constexpr (P::BULK) {
             if (rtid == 0) {
-              mbar_arrive_expect_tx(vfull + stg(tile), bytes);
-              bulk_copy_g2s(dst, src, bytes, vfull + stg(tile));
+              mbar_arrive_expect_tx(vfull + vstg(tile), bytes);
+              bulk_copy_g2s(dst, src, bytes, vfull + vstg(tile));
             }
           } else {
             for (int o = rtid * P::KCH; o < bytes; o += 128 * P::KCH) cp_async<P::KCH>(dst + o, src + o);
@@ -321,11 +333,16 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
         }
         cp_async_commit();
       };
-      for (int s = 0; s < P::NSTG - 2; ++s) issue_v(s);
       for (int it = 0; it <= ntiles; ++it) {
-        cp_async_wait<P::NSTG - 2>();  // tile it - 1 has landed; the next NSTG - 2 may still be in flight
+        cp_async_wait<P::NSV - 2>();  // tile it - 1 has landed; the next NSV - 2 may still be in flight
         roles_sync();
-        issue_v(it + P::NSTG - 2);     // into the stage tile it - 2 used
+        // into the stage tile it - 2 used; the first tiles only now, once the scoring warps have read the row
+        // factors that share memory with the value stages
+        if (it == 0) {
+          for (int s = 0; s <= P::NSV - 2; ++s) issue_v(s);
+        } else {
+          issue_v(it + P::NSV - 2);
+        }
         if (it == 0) continue;
         const int j = it - 1;  // the tile scored in the previous step
         const int nt_tok = min(TT, end - (start + j * TT));
@@ -338,9 +355,9 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
             acc[mt][0] *= al0; acc[mt][1] *= al1; acc[mt][2] *= al0; acc[mt][3] *= al1;
           }
         }
-        const uint8_t* vst = smem + P::OFF_V + stg(j) * P::STAGE_V;
+        const uint8_t* vst = smem + P::OFF_V + vstg(j) * P::STAGE_V;
         if constexpr (P::BULK) {
-          if (!tc::mbar_wait(vfull + stg(j), par(j))) *failed = 1;
+          if (!tc::mbar_wait(vfull + vstg(j), vpar(j))) *failed = 1;
         }
         const __half* pw = pbuf16 + pb * 8 * P::PST;
 #pragma unroll
@@ -366,7 +383,7 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
           for (int mt = 0; mt < MT; ++mt) {
             uint32_t x[4];  // hi fp16 pairs (v_2p, v_2p+1) of the four tokens, p = MT g + mt
 #pragma unroll
-            for (int r = 0; r < 4; ++r) x[r] = *reinterpret_cast<const uint32_t*>(tab + hilo_off16<BITS>(w[r], mt, rep16));
+            for (int r = 0; r < 4; ++r) x[r] = *reinterpret_cast<const uint32_t*>(tab + kv_off<BITS>(w[r], mt, repv));
             mma_m16n8k16(acc[mt], __byte_perm(x[0], x[1], sel_lo), __byte_perm(x[0], x[1], sel_hi),
                          __byte_perm(x[2], x[3], sel_lo), __byte_perm(x[2], x[3], sel_hi), b0, b1);
           }
@@ -405,13 +422,13 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
       auto issue_v = [&](int tile) {
         if (tile < ntiles) {
           const int t0 = start + tile * TT;
-          uint8_t* dst = smem + P::OFF_V + stg(tile) * P::STAGE_V;
+          uint8_t* dst = smem + P::OFF_V + vstg(tile) * P::STAGE_V;
           const uint8_t* src = vsrc + (kv_row0 + t0) * P::VROW;
           const int bytes = min(TT, end - t0) * P::VROW;
           if constexpr (P::BULK) {
             if (rtid == 0) {
-              mbar_arrive_expect_tx(vfull + stg(tile), bytes);
-              bulk_copy_g2s(dst, src, bytes, vfull + stg(tile));
+              mbar_arrive_expect_tx(vfull + vstg(tile), bytes);
+              bulk_copy_g2s(dst, src, bytes, vfull + vstg(tile));
             }
           } else {
             role_copy_async<P::VCH>(dst, src, bytes, rtid);
@@ -419,11 +436,16 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
         }
         cp_async_commit();
       };
-      for (int s = 0; s < P::NSTG - 2; ++s) issue_v(s);
       for (int it = 0; it <= ntiles; ++it) {
-        cp_async_wait<P::NSTG - 2>();  // tile it - 1 has landed; the next NSTG - 2 may still be in flight
+        cp_async_wait<P::NSV - 2>();  // tile it - 1 has landed; the next NSV - 2 may still be in flight
         roles_sync();
-        issue_v(it + P::NSTG - 2);     // into the stage tile it - 2 used
+        // into the stage tile it - 2 used; the first tiles only now, once the scoring warps have read the row
+        // factors that share memory with the value stages
+        if (it == 0) {
+          for (int s = 0; s <= P::NSV - 2; ++s) issue_v(s);
+        } else {
+          issue_v(it + P::NSV - 2);
+        }
         if (it == 0) continue;
         const int j = it - 1;  // the tile scored in the previous step
         const int nt_tok = min(TT, end - (start + j * TT));
@@ -436,9 +458,9 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
             for (int c = 0; c < 4; ++c) { acc[g][c].x *= al; acc[g][c].y *= al; }
           }
         }
-        const uint8_t* vst = smem + P::OFF_V + stg(j) * P::STAGE_V;
+        const uint8_t* vst = smem + P::OFF_V + vstg(j) * P::STAGE_V;
         if constexpr (P::BULK) {
-          if (!tc::mbar_wait(vfull + stg(j), par(j))) *failed = 1;
+          if (!tc::mbar_wait(vfull + vstg(j), vpar(j))) *failed = 1;
         }
         const float2* prow = pbuf + static_cast<size_t>(pb) * TT * G;
 #pragma unroll 2

@@ -117,7 +117,12 @@ extern "C" axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, c
   if (vkind == AXR_V_QUANT_TILED) return attend_tiled_launch(bits, G, mode == kGatherTensor, a, as_stream(stream));
   // row-layout values: keys scored through warp-level MMAs in AXR_GATHER_MMA mode, else on CUDA cores
   const bool vq = vkind == AXR_V_QUANT;
-  if (mode == kGatherMma) return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));
+  if (mode == kGatherMma) {
+    // fp16 values: one warp per token range through scores, softmax and the value product (no block barrier);
+    // quantized values: scoring and value warps one tile apart
+    if (!vq && attend_fused_supported(d, bits)) return attend_fused_launch(d, bits, G, vq, a, as_stream(stream));
+    return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));
+  }
   return attend_partial_launch(d, bits, G, vq, false, a, as_stream(stream), w);
 }
 

@@ -83,12 +83,71 @@ __device__ __forceinline__ void load_run(const uint8_t* stage, int off, uint32_t
   }
 }
 
+// Key/value pair table, 256 bytes per entry e (the 2b-bit code of a coordinate pair): bytes [0, 128) hold 16 copies
+// of the hi/lo fp16 pair {hi(c_lo), hi(c_hi)}, {lo(c_lo), lo(c_hi)} (copy c at 8 c), bytes [128, 256) hold 32 copies
+// of the hi pair alone (copy c at 128 + 4 c).  The offset of a lookup is one byte permute of the code word (entry
+// into byte 1, the lane's copy offset into byte 0): a warp's 64-bit key lookups take two wavefronts and its 32-bit
+// value lookups one, whatever the entries.
+template <int BITS>
+struct PairTableKV {
+  static constexpr int L = 1 << BITS;
+  static constexpr int E = L * L;
+  static constexpr int BYTES = E * 256;
+};
+
+template <int BITS>
+__device__ __forceinline__ void build_pair_table_kv(const float* __restrict__ gamma, uint8_t* __restrict__ tab) {
+  using T = PairTableKV<BITS>;
+  for (int i = threadIdx.x; i < T::E * 48; i += blockDim.x) {
+    const int e = i / 48, slot = i % 48;
+    const float c0 = gamma[e & (T::L - 1)], c1 = gamma[e >> BITS];
+    const __half h0 = __float2half_rn(c0), h1 = __float2half_rn(c1);
+    const __half2 hi = __halves2half2(h0, h1);
+    if (slot < 16) {
+      const __half2 lo = __halves2half2(__float2half_rn(c0 - __half2float(h0)), __float2half_rn(c1 - __half2float(h1)));
+      *reinterpret_cast<uint2*>(tab + e * 256 + slot * 8) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&hi), *reinterpret_cast<const uint32_t*>(&lo));
+    } else {
+      *reinterpret_cast<uint32_t*>(tab + e * 256 + 128 + (slot - 16) * 4) = *reinterpret_cast<const uint32_t*>(&hi);
+    }
+  }
+}
+
+// Byte offset in a PairTableKV of code pair i of a run of packed codes (w: its words, one zero word past the end);
+// rep = (lane % 16) * 8 for the hi/lo copies, 128 + 4 lane for the hi-only copies.
+template <int BITS>
+__device__ __forceinline__ uint32_t kv_off(const uint32_t* w, int i, uint32_t rep) {
+  if constexpr (BITS == 4)
+    return __byte_perm(w[i >> 2], rep, 0x5504u | (static_cast<uint32_t>(i & 3) << 4));
+  else
+    return (bits_at<2 * BITS>(w, 2 * BITS * i) << 8) | rep;
+}
+
 __device__ __forceinline__ void mma_m16n8k16(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                              uint32_t b0, uint32_t b1) {
   asm volatile(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Power-of-two range scale of one head's B operand from its transformed row q~ (shared memory, one warp):
+// 2^(14 - e) with ||q~|| in [2^(e-1), 2^e), so that the fp16 planes stay far from overflow and underflow.  Any
+// consistent power of two is exact; the epilogue divides it back out.
+template <int D>
+__device__ __forceinline__ float head_scale_rows(const float* __restrict__ row) {
+  const int lane = threadIdx.x & 31;
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < D / 32; ++i) {
+    const float x = row[lane + 32 * i];
+    ss = fmaf(x, x, ss);
+  }
+  const float m = sqrtf(warp_sum(ss));
+  if (!(m > 0.f) || !isfinite(m)) return 1.f;
+  int e = 0;
+  frexpf(m, &e);
+  return ldexpf(1.f, 14 - e);
 }
 
 template <int D, int G>
@@ -137,9 +196,56 @@ __device__ __forceinline__ void mma_b_build(const float* __restrict__ qs, const 
   }
 }
 
+// Block-wide build of the B fragments into shared memory, one 32-bit entry per thread: bs[e][lane] with
+// e = (nt KT + kk) 2 + r holds the hi-column register of MmaB::bh[nt][kk][r] for that lane (mma_b_build's values);
+// the lo-column registers and the inverse scales are derived on load (mma_b_load).
+template <int D, int G>
+__device__ __forceinline__ void mma_b_stage(const float* __restrict__ qs, const float* __restrict__ scl,
+                                            uint32_t* __restrict__ bs) {
+  constexpr int KT = MmaB<D, G>::KT, NT = MmaB<D, G>::NT, NE = NT * KT * 2;
+  for (int idx = threadIdx.x; idx < NE * 32; idx += blockDim.x) {
+    const int ln = idx & 31, e = idx >> 5;
+    const int r = e & 1, kk = (e >> 1) % KT, nt = (e >> 1) / KT;
+    const int gq = ln >> 2, tq = ln & 3;
+    const int h = 4 * nt + (gq >> 1);
+    const bool hi_col = (gq & 1) == 0;
+    float v[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int j = 2 * (2 * KT * tq + 2 * kk + r) + i;
+      const float q = h < G ? qs[h * D + j] * scl[h] : 0.f;
+      const float qh = __half2float(__float2half_rn(q));
+      v[i] = hi_col ? qh : q - qh;
+    }
+    const __half2 p = __floats2half2_rn(v[0], v[1]);
+    bs[e * 32 + ln] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+}
+
+template <int D, int G>
+__device__ __forceinline__ void mma_b_load(const uint32_t* __restrict__ bs, const float* __restrict__ scl, int lane,
+                                           MmaB<D, G>& B) {
+  constexpr int KT = MmaB<D, G>::KT, NT = MmaB<D, G>::NT;
+  const bool hi_col = ((lane >> 2) & 1) == 0;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int kk = 0; kk < KT; ++kk)
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const uint32_t x = bs[((nt * KT + kk) * 2 + r) * 32 + lane];
+        B.bh[nt][kk][r] = x;
+        B.bl[nt][kk][r] = hi_col ? x : 0u;
+      }
+    const int h = 4 * nt + (lane & 3);
+    B.inv[nt] = h < G ? 1.f / scl[h] : 1.f;
+  }
+}
+
 // Scaled scores (times s_h) of tokens r0 = row0 + g and r1 = r0 + 8 of a staged tile of packed rows (swizzled with
-// stage_swizzle<R> if SWZ), for head 4 nt + t: out[nt][0] for r0, out[nt][1] for r1.
-template <int D, int BITS, int G, bool SWZ = true>
+// stage_swizzle<R> if SWZ), for head 4 nt + t: out[nt][0] for r0, out[nt][1] for r1.  The table is a HiLoTable16
+// (rep = (lane % 16) * 16), or a PairTableKV if KV (rep = (lane % 16) * 8).
+template <int D, int BITS, int G, bool SWZ = true, bool KV = false>
 __device__ __forceinline__ void mma_scores16(const uint8_t* st, int row0, const uint8_t* tab, uint32_t rep16,
                                              const MmaB<D, G>& B, int lane, float (&out)[MmaB<D, G>::NT][2]) {
   constexpr int R = D * BITS / 8, KT = MmaB<D, G>::KT, NT = MmaB<D, G>::NT;
@@ -158,12 +264,16 @@ __device__ __forceinline__ void mma_scores16(const uint8_t* st, int row0, const 
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int i = 0; i < 4; ++i) c[x][nt][i] = 0.f;
+  auto off = [&](const uint32_t* w, int i) {
+    if constexpr (KV) return kv_off<BITS>(w, i, rep16);
+    else return hilo_off16<BITS>(w, i, rep16);
+  };
 #pragma unroll
   for (int kk = 0; kk < KT; ++kk) {
-    const uint2 e00 = *reinterpret_cast<const uint2*>(tab + hilo_off16<BITS>(w0, 2 * kk, rep16));
-    const uint2 e10 = *reinterpret_cast<const uint2*>(tab + hilo_off16<BITS>(w1, 2 * kk, rep16));
-    const uint2 e01 = *reinterpret_cast<const uint2*>(tab + hilo_off16<BITS>(w0, 2 * kk + 1, rep16));
-    const uint2 e11 = *reinterpret_cast<const uint2*>(tab + hilo_off16<BITS>(w1, 2 * kk + 1, rep16));
+    const uint2 e00 = *reinterpret_cast<const uint2*>(tab + off(w0, 2 * kk));
+    const uint2 e10 = *reinterpret_cast<const uint2*>(tab + off(w1, 2 * kk));
+    const uint2 e01 = *reinterpret_cast<const uint2*>(tab + off(w0, 2 * kk + 1));
+    const uint2 e11 = *reinterpret_cast<const uint2*>(tab + off(w1, 2 * kk + 1));
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       mma_m16n8k16(c[kk & 1][nt], e00.x, e10.x, e01.x, e11.x, B.bh[nt][kk][0], B.bh[nt][kk][1]);
