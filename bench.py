@@ -34,6 +34,14 @@ METRIC = "quantized-KV decode attention: keys·heads/s and HBM GB/s vs B200 peak
 UNIT = "keys·heads/s"
 L2_BYTES = 126 * 1024 * 1024
 
+# DRAM traffic (read + write bytes) per launch of the timed attend kernel, from the ncu captures summarised under
+# profiles/ (attend_rows_long_context.md: a B=4 capture, scaled by the units processed; attend_fused_llama8b.md: full
+# size). Valid for the kernel versions those captures were taken on.
+TRAFFIC = {
+    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.537472e6 + 3.547392e6),
+    "llama8b_decode_b8_t8192_hq32_hkv8_d128_b4_v16": 169.015296e6 + 5.675264e6,
+}
+
 WORKLOADS = {
     "long_context": W.LONG_CONTEXT,
     "llama8b": W.LLAMA8B_DECODE,
@@ -345,8 +353,10 @@ def run_axr(args, w):
                    "values": "quantized b=%d" % bits if w.v_quant else "fp16", "parallelism": f"replicas x{ws}",
                    "l2": "flushed between steps (256 MiB write outside the per-step events)"},
         "hbm_gbs": alg_bytes * ws * args.steps / (step_ms / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": "attend_decode (partial + merge)", "achieved": achieved,
-                     "peak": peak, "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+        "roofline": {"bound": "hbm", "kernel": ("attend_rows_kernel" if w.v_quant else "attend_fused_kernel") +
+                     " + attend_reduce_kernel (one axr_attend_decode call)", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": TRAFFIC.get(w.name) if args.batch is None else None,
                      "algorithmic_bytes": alg_bytes, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_src == "measured" else "fallback 6.65 TB/s"},
         "e2e": {"value": key_heads / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
