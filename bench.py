@@ -175,6 +175,46 @@ def cpu_baseline(w, seconds=10.0):
                       f"{w.T} tokens each, plus the new token's write; fp64 numpy, 1 thread, {t_total:.1f} s"}
 
 
+def _gen_rows(gen, shape, seed, dev):
+    """A synthetic fp16 tensor [B, ...] drawn one batch row at a time (bounded temporary memory)."""
+    import torch
+    out = torch.empty(shape, dtype=torch.float16, device=dev)
+    for b in range(shape[0]):
+        out[b] = gen(tuple(shape[1:]), seed + 7919 * b, dev)
+    return out
+
+
+def _sweep(args, dev, time_calls):
+    """Decode sweep: B in {1, 8, 64} x T in {4096, 32768, 131072} x b in 1..4 x d in {64, 128}, Hq=32, Hkv=8,
+    fp16 V; the LUT attend and the dense fp16 kernel on caches of the same shape, L2 flushed before every call."""
+    import torch
+    from kv_cache_quantized_b200 import ops
+    rows = []
+    peak = _peaks()[0]
+    for w in W.SWEEP:
+        B, Hq, Hkv, T, d, bits = w.B, w.Hq, w.Hkv, w.T, w.d, w.bits
+        signs = torch.as_tensor(W.sign_vector(d, w.seed + 4), device=dev)
+        k = _gen_rows(W.lognormal_rows_device, (B, Hkv, T, d), w.seed, dev)
+        kc, kn = ops.write_keys(k, signs, bits)
+        v = _gen_rows(W.lognormal_rows_device, (B, Hkv, T, d), w.seed + 2, dev)
+        q = W.normal_device((B, Hq, d), w.seed + 3, dev, dtype=torch.float32)
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(ops.attend_workspace_bytes(B, Hq, Hkv, T, d), 16), dtype=torch.uint8, device=dev)
+        ms_lut = time_calls(lambda: ops.attend_decode(q, kc, kn, signs, bits, v=v, out=out, workspace=ws))
+        ms_dense = time_calls(lambda: ops.dense_decode(q, k, v, out=out, workspace=ws))
+        lut_b = (d * bits // 8 + 2 + 2 * d) * B * Hkv * T
+        dense_b = 4 * d * B * Hkv * T
+        rows.append({"B": B, "T": T, "bits": bits, "d": d,
+                     "lut_ms": ms_lut, "lut_gbs": lut_b / (ms_lut / 1e3) / 1e9,
+                     "lut_frac": lut_b / (ms_lut / 1e3) / 1e9 / peak,
+                     "dense_ms": ms_dense, "dense_gbs": dense_b / (ms_dense / 1e3) / 1e9,
+                     "dense_frac": dense_b / (ms_dense / 1e3) / 1e9 / peak,
+                     "lut_speedup_over_dense": ms_dense / ms_lut})
+        del k, kc, kn, v, q, out, ws
+        torch.cuda.empty_cache()
+    return rows
+
+
 def run_axr(args, w):
     import torch
     import torch.distributed as dist
@@ -332,6 +372,21 @@ def run_axr(args, w):
         ops.set_gather("mma")
         del sc_out
 
+    # the build's own dense fp16 decode kernel on the same shape (fp16 K and V), the bandwidth reference
+    dense = None
+    if not args.no_dense:
+        kd = _gen_rows(W.lognormal_rows_device, (B, Hkv, T, d), seed + 7, dev)
+        vd = _gen_rows(W.normal_device, (B, Hkv, T, d), seed + 8, dev)
+        ms = time_calls(lambda: ops.dense_decode(q, kd, vd, out=out, workspace=wsp))
+        dbytes = 4 * d * B * Hkv * T
+        dense = {"kernel": "attend_partial_kernel<DENSE> + attend_reduce_kernel (axr_dense_decode)", "ms": ms,
+                 "value": B * T * Hq / (ms / 1e3), "unit": UNIT, "achieved_gbs": dbytes / (ms / 1e3) / 1e9,
+                 "frac": dbytes / (ms / 1e3) / 1e9 / _peaks()[0], "algorithmic_bytes": dbytes}
+        del kd, vd
+
+    # the decode sweep (--sweep): the LUT attend with fp16 values next to the dense fp16 kernel, per shape
+    sweep = _sweep(args, dev, time_calls) if args.sweep else None
+
     # max over ranks
     from kv_cache_quantized_b200 import dist as D
     step_ms, e2e_ms, attend_avg_ms = D.max_over_ranks([step_ms, e2e_ms, float(np.mean(attend_ms))], device=dev)
@@ -363,9 +418,12 @@ def run_axr(args, w):
                 "d2h_bytes_per_step": d2h},
         "scorer": {m: dict(v_, frac=v_["achieved_gbs"] / _peaks()[0]) for m, v_ in scorer.items()},
         "attend_variants": {m: dict(v_, frac=v_["achieved_gbs"] / _peaks()[0]) for m, v_ in variants.items()},
+        "dense_reference": dense,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if sweep is not None:
+        line["sweep"] = sweep
     return line
 
 
@@ -404,6 +462,9 @@ def main(argv=None):
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch size (small ncu cases)")
     ap.add_argument("--no-scorer", action="store_true", help="skip the separate axr_score measurement")
     ap.add_argument("--no-variants", action="store_true", help="skip the tiled-value attend variants")
+    ap.add_argument("--no-dense", action="store_true", help="skip the dense fp16 bandwidth reference")
+    ap.add_argument("--sweep", action="store_true",
+                    help="also run the decode sweep (B x T x bits x d, fp16 V) against the dense fp16 kernel")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
