@@ -34,13 +34,10 @@ METRIC = "quantized-KV decode attention: keys·heads/s and HBM GB/s vs B200 peak
 UNIT = "keys·heads/s"
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM traffic (read + write bytes) per launch of the timed attend kernel, from the ncu captures summarised under
-# profiles/ (attend_rows_long_context.md: a B=4 capture, scaled by the units processed; attend_fused_llama8b.md: full
-# size). Valid for the kernel versions those captures were taken on.
-TRAFFIC = {
-    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.537472e6 + 3.547392e6),
-    "llama8b_decode_b8_t8192_hq32_hkv8_d128_b4_v16": 169.015296e6 + 5.675264e6,
-}
+# DRAM traffic (read + write bytes) per launch of the timed decode kernel, from the ncu capture summarised in
+# profiles/attend_rows_long_context.md (a B=4 capture, scaled by the units processed).  Valid for the kernel version
+# that capture was taken on; a workload without an entry reports null.
+TRAFFIC = {}
 
 WORKLOADS = {
     "long_context": W.LONG_CONTEXT,
@@ -249,34 +246,22 @@ def run_axr(args, w):
     q = W.normal_device((B, Hq, d), seed + 3, dev, dtype=torch.float32)
     knew = W.normal_device((B, Hkv, d), seed + 5, dev)
     vnew = W.normal_device((B, Hkv, d), seed + 6, dev)
-    dst = ((torch.arange(B, device=dev)[:, None] * Hkv + torch.arange(Hkv, device=dev)[None, :]) * T + (T - 1))
-    dst = dst.reshape(-1).to(torch.int64)
     out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
     wsb = ops.attend_workspace_bytes(B, Hq, Hkv, T, d)
     wsp = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
 
-    def append(kn_in, vn_in):
-        ops.write_keys(kn_in, signs, bits, codes=kc.view(-1, R), norms=kn.view(-1), dst_rows=dst)
+    def step(q_in, k_in, v_in):  # one axr_decode_step: write the new K, V at T - 1 and attend over [0, T)
         if w.v_quant:
-            ops.write_keys(vn_in, signs, bits, codes=vc.view(-1, R), norms=vn.view(-1), dst_rows=dst)
+            ops.decode_step(q_in, k_in, v_in, kc, kn, signs, bits, vcodes=vc, vnorms=vn, out=out, workspace=wsp)
         else:
-            v.view(-1, d).index_copy_(0, dst, vn_in.view(-1, d))  # fp16 values are stored as they are
+            ops.decode_step(q_in, k_in, v_in, kc, kn, signs, bits, v=v, out=out, workspace=wsp)
 
-    def attend(q_in):
-        if w.v_quant:
-            ops.attend_decode(q_in, kc, kn, signs, bits, vcodes=vc, vnorms=vn, out=out, workspace=wsp)
-        else:
-            ops.attend_decode(q_in, kc, kn, signs, bits, v=v, out=out, workspace=wsp)
-
-    launches_per_step = (2 if w.v_quant else 1) + 2  # write(s) + partial + merge
-    if not w.v_quant:
-        launches_per_step += 0  # the fp16 value append is a torch copy, not one of the library's kernels
+    launches_per_step = 2  # the decode kernel (with the new token's write) + the split merge
 
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
-        append(knew, vnew)
-        attend(q)
+        step(q, knew, vnew)
     torch.cuda.synchronize()
 
     # --- timed region: K steps, L2 flushed between steps (outside the per-step events) ---
@@ -290,15 +275,13 @@ def run_axr(args, w):
             flush.zero_()
             e0, e1, e2 = ev[i]
             e0.record(stream)
-            append(knew, vnew)
-            e1.record(stream)
-            attend(q)
+            step(q, knew, vnew)
             e2.record(stream)
         torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
     step_ms = sum(e0.elapsed_time(e2) for e0, _, e2 in ev)
-    attend_ms = [e1.elapsed_time(e2) for _, e1, e2 in ev]
+    attend_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]  # the whole step is one decode call
     clocks = clk.summary()
 
     # --- end to end through the public API: pinned host inputs in, result out, every step ---
@@ -315,8 +298,7 @@ def run_axr(args, w):
         q_d.copy_(q_h, non_blocking=True)
         k_d.copy_(k_h, non_blocking=True)
         v_d.copy_(v_h, non_blocking=True)
-        append(k_d, v_d)
-        attend(q_d)
+        step(q_d, k_d, v_d)
         o_h.copy_(out, non_blocking=True)
         b_.record(stream)
     torch.cuda.synchronize()
@@ -347,7 +329,7 @@ def run_axr(args, w):
                                                       workspace=wsp))
             variants[name] = {"ms": ms, "achieved_gbs": ab / (ms / 1e3) / 1e9, "algorithmic_bytes": ab}
         ops.set_gather("mma")
-        variants["rows"] = {"ms": float(np.mean(attend_ms)),
+        variants["rows_decode_step"] = {"ms": float(np.mean(attend_ms)),
                             "achieved_gbs": ab / (float(np.mean(attend_ms)) / 1e3) / 1e9, "algorithmic_bytes": ab}
 
     # the scorer alone (axr_score) on the same cache, every table read mode, L2 flushed before each call
@@ -408,8 +390,8 @@ def run_axr(args, w):
                    "values": "quantized b=%d" % bits if w.v_quant else "fp16", "parallelism": f"replicas x{ws}",
                    "l2": "flushed between steps (256 MiB write outside the per-step events)"},
         "hbm_gbs": alg_bytes * ws * args.steps / (step_ms / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": ("attend_rows_kernel" if w.v_quant else "attend_fused_kernel") +
-                     " + attend_reduce_kernel (one axr_attend_decode call)", "achieved": achieved,
+        "roofline": {"bound": "hbm", "kernel": "attend_rows_kernel (with the new token's write) + "
+                     "attend_reduce_kernel (one axr_decode_step call)", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": TRAFFIC.get(w.name) if args.batch is None else None,
                      "algorithmic_bytes": alg_bytes, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"

@@ -175,6 +175,25 @@ AXR_API axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, cons
                              void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * axr_decode_step -- one decode step in one call.  The new token's key and value (k_new, v_new: [B, Hkv, d] fp16)
+ * are written into the cache at position len_b - 1 of each batch row (len_b = seq_lens[b], or T): keys through the
+ * write path of axr_write_keys (codes and fp16 norm), values the same way (AXR_V_QUANT) or as they are (AXR_V_F16).
+ * Then axr_attend_decode runs over positions [0, len_b), the new token included.  The write happens inside the
+ * decode launch, by the block that attends over that position, before that block copies the position's tile in, so
+ * the step needs no separate append launch.  Digest, Key Points 2 ("transform on write") for the write, and
+ * axr_attend_decode for the read.  Row value layouts only (AXR_V_F16, AXR_V_QUANT).  Batch rows with len_b = 0 get
+ * out = 0 and nothing is written.
+ *   kcodes, knorms, v, vnorms [dev]: the cache as for axr_attend_decode; one position per (b, KV head) is written;
+ *   k_new, v_new [dev] [B, Hkv, d] fp16, 16-byte aligned.
+ * Errors: as axr_attend_decode; AXR_EINVAL for the tiled value layout or a null or misaligned k_new / v_new.
+ */
+AXR_API axr_status axr_decode_step(const float* q, const uint16_t* k_new, const uint16_t* v_new, uint8_t* kcodes,
+                                   uint16_t* knorms, axr_vkind vkind, void* v, uint16_t* vnorms,
+                                   const int32_t* seq_lens, int B, int Hq, int Hkv, int T, int Tcap, int d, int bits,
+                                   const int8_t* signs, float scale, float* out, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/*
  * axr_attend_decode_static -- axr_attend_decode without a workspace argument, for callers that cannot allocate
  * device memory (code running inside a memory pool it does not own, plugins handed only input and output pointers,
  * decode steps that must not touch an allocator).  The paper has no counterpart: this is a deployment convenience.

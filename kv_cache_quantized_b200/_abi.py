@@ -32,6 +32,7 @@ SIGNATURES = {
     "axr_score": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p]),
     "axr_attend_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "axr_attend_decode": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p, _sz, _p]),
+    "axr_decode_step": (_i, [_p, _p, _p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p, _sz, _p]),
     "axr_dense_decode": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
     "axr_select_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "axr_select_signs": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _p, _p, _p, _sz, _p]),

@@ -77,13 +77,14 @@ axr_status carve_workspace(axr::DecodeArgs& a, int d, void* ws, size_t ws_bytes,
 }
 }  // namespace
 
-extern "C" axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, const uint16_t* knorms,
-                                        axr_vkind vkind, const void* v, const uint16_t* vnorms,
-                                        const int32_t* seq_lens, int B, int Hq, int Hkv, int T, int Tcap, int d,
-                                        int bits, const int8_t* signs, float scale, float* out, void* workspace,
-                                        size_t ws_bytes, void* stream) {
+namespace {
+// axr_attend_decode, and axr_decode_step when knew / vnew are given (the new token written by the decode launch)
+axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, const uint16_t* knorms,
+                       axr_vkind vkind, const void* v, const uint16_t* vnorms, const int32_t* seq_lens, int B, int Hq,
+                       int Hkv, int T, int Tcap, int d, int bits, const int8_t* signs, float scale, float* out,
+                       void* workspace, size_t ws_bytes, void* stream, const uint16_t* knew, const uint16_t* vnew) {
   using namespace axr;
-  const char* w = "axr_attend_decode";
+  const bool step = knew != nullptr || vnew != nullptr;
   axr_status st = check_decode_sizes(w, B, Hq, Hkv, T, Tcap, d);
   if (st != AXR_OK) return st;
   if (bits < 1 || bits > 4) return set_error(AXR_EUNSUPPORTED, "%s: bits=%d outside 1..4", w, bits);
@@ -93,7 +94,10 @@ extern "C" axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, c
     return set_error(AXR_EUNSUPPORTED, "%s: tiled values need d = 128 (d=%d)", w, d);
   if (vkind == AXR_V_QUANT_TILED && Tcap % 128)
     return set_error(AXR_EINVAL, "%s: tiled values need Tcap a multiple of 128 (Tcap=%d)", w, Tcap);
+  if (step && vkind == AXR_V_QUANT_TILED) return set_error(AXR_EINVAL, "%s: the row value layouts only", w);
   if (B == 0) return set_error(AXR_OK, "");
+  if (step && (!knew || !vnew)) return set_error(AXR_EINVAL, "%s: null pointer", w);
+  if (step && (!aligned(knew, 16) || !aligned(vnew, 16))) return set_error(AXR_EINVAL, "%s: misaligned pointer", w);
   if (!q || !kcodes || !knorms || !signs || !v || !out || (vkind != AXR_V_F16 && !vnorms))
     return set_error(AXR_EINVAL, "%s: null pointer", w);
   if (!aligned(q, 16) || !aligned(kcodes, 16) || !aligned(knorms, 4) || !aligned(out, 16) || !aligned(v, 16) ||
@@ -111,12 +115,15 @@ extern "C" axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, c
   if (st != AXR_OK) return st;
   a.kcodes = kcodes; a.knorms = reinterpret_cast<const __half*>(knorms); a.signs = signs; a.out = out;
   a.v = v; a.vnorms = reinterpret_cast<const __half*>(vnorms); a.cb = *cb;
+  a.knew = reinterpret_cast<const __half*>(knew); a.vnew = reinterpret_cast<const __half*>(vnew);
   const int G = Hq / Hkv;
   const int mode = g_gather.load();
+  const bool vq = vkind == AXR_V_QUANT;
+  // decode step: the kernel whose prologue writes the new token (scores through warp-level MMAs)
+  if (step) return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));
   // tiled values: the tcgen05 kernel in AXR_GATHER_TENSOR mode, else warp-level MMAs for keys and values
   if (vkind == AXR_V_QUANT_TILED) return attend_tiled_launch(bits, G, mode == kGatherTensor, a, as_stream(stream));
   // row-layout values: keys scored through warp-level MMAs in AXR_GATHER_MMA mode, else on CUDA cores
-  const bool vq = vkind == AXR_V_QUANT;
   if (mode == kGatherMma) {
     // fp16 values: one warp per token range through scores, softmax and the value product (no block barrier);
     // quantized values: scoring and value warps one tile apart
@@ -124,6 +131,26 @@ extern "C" axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, c
     return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));
   }
   return attend_partial_launch(d, bits, G, vq, false, a, as_stream(stream), w);
+}
+}  // namespace
+
+extern "C" axr_status axr_attend_decode(const float* q, const uint8_t* kcodes, const uint16_t* knorms,
+                                        axr_vkind vkind, const void* v, const uint16_t* vnorms,
+                                        const int32_t* seq_lens, int B, int Hq, int Hkv, int T, int Tcap, int d,
+                                        int bits, const int8_t* signs, float scale, float* out, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  return attend_impl("axr_attend_decode", q, kcodes, knorms, vkind, v, vnorms, seq_lens, B, Hq, Hkv, T, Tcap, d,
+                     bits, signs, scale, out, workspace, ws_bytes, stream, nullptr, nullptr);
+}
+
+extern "C" axr_status axr_decode_step(const float* q, const uint16_t* k_new, const uint16_t* v_new, uint8_t* kcodes,
+                                      uint16_t* knorms, axr_vkind vkind, void* v, uint16_t* vnorms,
+                                      const int32_t* seq_lens, int B, int Hq, int Hkv, int T, int Tcap, int d,
+                                      int bits, const int8_t* signs, float scale, float* out, void* workspace,
+                                      size_t ws_bytes, void* stream) {
+  if (!k_new || !v_new) return axr::set_error(AXR_EINVAL, "axr_decode_step: null pointer");
+  return attend_impl("axr_decode_step", q, kcodes, knorms, vkind, v, vnorms, seq_lens, B, Hq, Hkv, T, Tcap, d, bits,
+                     signs, scale, out, workspace, ws_bytes, stream, k_new, v_new);
 }
 
 extern "C" axr_status axr_dense_decode(const float* q, const uint16_t* k, const uint16_t* v,

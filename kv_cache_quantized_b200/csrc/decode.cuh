@@ -37,6 +37,8 @@ struct DecodeArgs {
   const __half* vnorms;      // [B, Hkv, Tcap] (quantized V)
   const int32_t* seq_lens;   // [B] or null
   const int8_t* signs;       // [D]
+  const __half* knew;        // [B, Hkv, D] fp16: decode step, the new token's key, written at position len - 1
+  const __half* vnew;        // [B, Hkv, D] fp16: its value (both null outside a decode step)
   float* scores;             // [B, Hq, T] (scorer)
   float* ws_o;               // [B, Hq, S, D]
   float* ws_m;               // [B, Hq, S]  running max, log2 units

@@ -246,6 +246,46 @@ def attend_decode(q, kcodes, knorms, signs, bits, v=None, vcodes=None, vnorms=No
     return out
 
 
+def decode_step(q, k_new, v_new, kcodes, knorms, signs, bits, v=None, vcodes=None, vnorms=None, scale=None,
+                seq_lens=None, T=None, out=None, workspace=None):
+    """One decode step in one launch: k_new, v_new (float16 [B, Hkv, d]) are written into the cache at position
+    seq_lens[b] - 1 of each batch row (T - 1 without seq_lens) -- keys as codes and norms, values the same way
+    (vcodes/vnorms) or as they are (v) -- and attention then runs over positions [0, seq_lens[b]).  Row value
+    layouts only.  Returns out [B, Hq, d] float32; the cache tensors are updated in place."""
+    d = q.shape[-1]
+    B, Hq, Hkv, Tcap, T = _cache_dims(q, kcodes, knorms, d, bits, T)
+    _need_cuda("signs", signs, torch.int8)
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        _need_cuda(name, t, torch.float16)
+        if tuple(t.shape) != (B, Hkv, d) or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [B, Hkv, d] float16 tensor")
+    seq_lens = _lens(seq_lens, B)
+    if (v is None) == (vcodes is None):
+        raise ValueError("pass exactly one of v or vcodes")
+    if v is not None:
+        _need_cuda("v", v, torch.float16)
+        if tuple(v.shape) != (B, Hkv, Tcap, d):
+            raise ValueError("v must be [B, Hkv, Tcap, d]")
+        vkind, vptr, vnptr = _abi.V_F16, _ptr(v), None
+    else:
+        _need_cuda("vcodes", vcodes, torch.uint8)
+        _need_cuda("vnorms", vnorms, torch.float16)
+        if vcodes.shape != kcodes.shape or vnorms.shape != knorms.shape:
+            raise ValueError("vcodes / vnorms must have the key cache's shapes (row layout)")
+        vkind, vptr, vnptr = _abi.V_QUANT, _ptr(vcodes), _ptr(vnorms)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    _need_cuda("out", out, torch.float32)
+    nbytes = attend_workspace_bytes(B, Hq, Hkv, T, d)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = _abi.lib().axr_decode_step(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(kcodes), _ptr(knorms), vkind, vptr, vnptr,
+                                    _ptr(seq_lens), B, Hq, Hkv, T, Tcap, d, bits, _ptr(signs), scale, _ptr(out),
+                                    _ptr(ws), ws.numel(), _stream())
+    _abi.check(st, "axr_decode_step")
+    return out
+
+
 def dense_decode(q, k, v, scale=None, seq_lens=None, T=None, out=None, workspace=None):
     """Decode attention over an unquantized float16 K/V cache [B, Hkv, Tcap, d] (the bandwidth reference)."""
     _need_cuda("q", q, torch.float32)

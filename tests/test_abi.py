@@ -101,6 +101,19 @@ def test_attend_tiled_argument_errors(L):
                                FAKE, 1 << 20, None) == 1  # unknown vkind
 
 
+def test_decode_step_argument_errors(L):
+    call = lambda kn=FAKE, vn_new=FAKE, vkind=1, d=128: L.axr_decode_step(
+        FAKE, kn, vn_new, FAKE, FAKE, vkind, FAKE, FAKE, None, 2, 8, 2, 200, 256, d, 4, FAKE, 0.1, FAKE, FAKE,
+        1 << 20, None)
+    assert call(kn=None) == 1            # the new key is required
+    assert call(vn_new=None) == 1        # and the new value
+    assert call(kn=FAKE + 8) == 1        # 16-byte aligned
+    assert call(vkind=2) == 1            # row value layouts only
+    assert call(d=32) == 2
+    assert L.axr_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, 1, FAKE, FAKE, None, 0, 8, 2, 200, 256, 128, 4, FAKE,
+                             0.1, FAKE, FAKE, 1 << 20, None) == 0  # B = 0: nothing to do
+
+
 def test_score_argument_errors(L):
     args = lambda **kw: dict(dict(q=FAKE, kc=FAKE, kn=FAKE, sl=None, B=2, Hq=8, Hkv=2, T=10, Tcap=16, d=128,
                                   bits=4, s=FAKE, scale=1.0, out=FAKE), **kw)

@@ -153,6 +153,68 @@ def test_unaligned_norm_rows(vq):
                 parity.check_scores(sc[b, h, :Tb], want, A)
 
 
+@pytest.mark.parametrize("vq", [False, True])
+@pytest.mark.parametrize("d,bits,G", [(128, 4, 4), (64, 2, 8), (128, 3, 1)])
+def test_decode_step(vq, d, bits, G):
+    """axr_decode_step writes the new token exactly as axr_write_keys does and attends over it: the same bits in the
+    cache, the same output as a separate append + attend, and parity with the oracle over the full cache."""
+    B, Hkv, T, Tcap = 3, 2, 900, 912
+    Hq = Hkv * G
+    k, v, s, kc, kn, vc, vn = oracle_cache(B, Hkv, T, d, bits, 950 + d + bits + G, vq)
+    q = W.normal((B, Hq, d), 951, np.float32)
+    lens = np.array([900, 1, 517], np.int32)  # the new token: the last position, the first, a middle one
+    pos = lens - 1
+    knew = np.stack([k[b, :, pos[b]] for b in range(B)])  # [B, Hkv, d]
+    vnew = np.stack([v[b, :, pos[b]] for b in range(B)])
+    # cache copies with garbage at each new token's position
+    def stale(a, fill):
+        a = padded(a, Tcap).copy()
+        for b in range(B):
+            a[b, :, pos[b]] = fill
+        return a
+    kc_g, kn_g = cuda(stale(kc, 0x5a)), cuda(stale(kn, np.float16(3.0)))
+    if vq:
+        vargs = dict(vcodes=cuda(stale(vc, 0xa5)), vnorms=cuda(stale(vn, np.float16(2.0))))
+    else:
+        vargs = dict(v=cuda(stale(v, np.float16(7.0))))
+    out = ops.decode_step(cuda(q), cuda(knew), cuda(vnew), kc_g, kn_g, cuda(s), bits, seq_lens=cuda(lens), T=T,
+                          **vargs).cpu().numpy()
+    # the written token matches axr_write_keys on the same vectors
+    st = cuda(s)
+    wk_c, wk_n = ops.write_keys(cuda(knew.reshape(-1, d)), st, bits)
+    for b in range(B):
+        for h in range(Hkv):
+            i = b * Hkv + h
+            assert np.array_equal(kc_g[b, h, pos[b]].cpu().numpy(), wk_c[i].cpu().numpy())
+            assert kn_g[b, h, pos[b]].item() == wk_n[i].item()
+    if vq:
+        wv_c, wv_n = ops.write_keys(cuda(vnew.reshape(-1, d)), st, bits)
+        for b in range(B):
+            for h in range(Hkv):
+                i = b * Hkv + h
+                assert np.array_equal(vargs["vcodes"][b, h, pos[b]].cpu().numpy(), wv_c[i].cpu().numpy())
+                assert vargs["vnorms"][b, h, pos[b]].item() == wv_n[i].item()
+    else:
+        for b in range(B):
+            assert np.array_equal(vargs["v"][b, :, pos[b]].cpu().numpy(), vnew[b])
+    # the same output as attend over the now complete cache
+    again = ops.attend_decode(cuda(q), kc_g, kn_g, cuda(s), bits, seq_lens=cuda(lens), T=T, **vargs).cpu().numpy()
+    # the same kernel for quantized values (identical bits); fp16 values may take the other kernel, whose warps split
+    # the tokens differently: fp16 weights rounded against other running maxima (2^-11 relative each)
+    num = np.linalg.norm((out - again).reshape(B * Hq, d), axis=1)
+    den = np.linalg.norm(again.reshape(B * Hq, d), axis=1)
+    assert np.all(num <= 2.0 ** -11 * np.maximum(den, 1e-30)), (num / np.maximum(den, 1e-30)).max()
+    # parity with the oracle over the whole cache (codes of the new token: the write path's own)
+    kc_w = kc_g.cpu().numpy()[:, :, :T]
+    kn_w = kn_g.cpu().numpy()[:, :, :T]
+    if vq:
+        okw = dict(vcodes=vargs["vcodes"].cpu().numpy()[:, :, :T], vn16=vargs["vnorms"].cpu().numpy()[:, :, :T])
+    else:
+        okw = dict(v=v)
+    want = oracle.decode_attention(q, kc_w, kn_w, s, bits, 1 / math.sqrt(d), seq_lens=lens, **okw)
+    parity.check_outputs(out, want)
+
+
 def test_dense_matches_oracle_attention():
     B, Hkv, G, T, Tcap, d = 3, 2, 4, 2100, 2200, 128
     k = W.lognormal_rows((B, Hkv, T, d), 800, dtype=np.float16)
