@@ -37,7 +37,9 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM traffic (read + write bytes) per launch of the timed decode kernel, from the ncu capture summarised in
 # profiles/attend_rows_long_context.md (a B=4 capture, scaled by the units processed).  Valid for the kernel version
 # that capture was taken on; a workload without an entry reports null.
-TRAFFIC = {}
+TRAFFIC = {
+    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.562048e6 + 3.795712e6),
+}
 
 WORKLOADS = {
     "long_context": W.LONG_CONTEXT,
