@@ -21,39 +21,10 @@
 // fp32 FMA product (value lanes own 8 coordinates of a row).
 #pragma once
 
+#include "append.cuh"
 #include "mma_score.cuh"
-#include "write_vec.cuh"
 
 namespace axr {
-
-// Decode step: warp 0 (key) or warp 1 (value) of the block attending over the new token writes it into the cache at
-// `row` ([B, Hkv, Tcap] numbering) through the write path -- codes and fp16 norm, or the fp16 value as it is -- and
-// makes the write visible to the bulk copies and cp.async reads that follow a block barrier.
-template <int D, int BITS, bool VQ>
-__device__ __forceinline__ void append_token(const DecodeArgs& a, int b, int hk, size_t row, int which, int lane,
-                                             uint8_t* idx_scratch) {
-  constexpr int VPL = WarpVec<D>::VPL, LANES = WarpVec<D>::LANES, L = 1 << BITS, R = D * BITS / 8;
-  const __half* src = (which == 0 ? a.knew : a.vnew) + (static_cast<size_t>(b) * a.Hkv + hk) * D;
-  if (which == 1 && !VQ) {  // fp16 values are stored as they are
-    __half* dst = static_cast<__half*>(const_cast<void*>(a.v)) + row * D;
-    for (int j = lane; j < D; j += kWarp) dst[j] = src[j];
-  } else {
-    float sg[VPL];
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) sg[i] = lane < LANES ? sign_of(a.signs[lane * VPL + i]) : 0.0f;
-    float tau[L - 1];
-#pragma unroll
-    for (int k = 0; k < L - 1; ++k) tau[k] = a.cb.tau[k];
-    const float n = quantize_vector<D, BITS, __half>(src, sg, tau, lane, idx_scratch);
-    __syncwarp();
-    uint8_t* codes = const_cast<uint8_t*>(which == 0 ? a.kcodes : static_cast<const uint8_t*>(a.v));
-    __half* norms = const_cast<__half*>(which == 0 ? a.knorms : a.vnorms);
-    pack_row<D, BITS>(idx_scratch, codes + row * R, lane);
-    if (lane == 0) norms[row] = __float2half_rn(n);
-  }
-  __threadfence();  // the stores reach the device-wide view ...
-  asm volatile("fence.proxy.async.global;\n" ::: "memory");  // ... and the async proxy of the bulk copies
-}
 
 template <int D, int BITS, int G, bool VQ>
 struct RowsPlan {
@@ -174,8 +145,12 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
     if (a.knew != nullptr && len > 0 && start <= len - 1 && len - 1 < end) {
       // decode step: this item holds the new token (position len - 1): warp 0 writes its key and warp 1 its value
       // through the write path, before any of the item's tiles is copied
-      if (warp < 2) append_token<D, BITS, VQ>(a, b, hk, kv_row0 + (len - 1), warp, lane,
-                                                reinterpret_cast<uint8_t*>(smem + P::OFF_P) + warp * D);
+      if (warp < 2) {
+        append_row<D, BITS, VQ>(a, b, hk, kv_row0 + (len - 1), warp, lane,
+                                reinterpret_cast<uint8_t*>(smem + P::OFF_P) + warp * D);
+        __threadfence();  // the stores reach the device-wide view ...
+        asm volatile("fence.proxy.async.global;\n" ::: "memory");  // ... and the async proxy of the bulk copies
+      }
     }
     transform_queries<D, G>(qg, a.signs, a.mult, qs);
     fence_proxy_async();  // the row factors share memory with the value stages, refilled by bulk copies
@@ -207,8 +182,9 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
         const int t = start + tile * TT + warp * WT + lane;
         uint32_t r = 0x3c00u << 16;  // value norm 1 for fp16 values
         if (!nrm_async && tile < ntiles && t < end) {
-          r = __half_as_ushort(__ldg(kn_src + t));
-          if constexpr (VQ) r |= static_cast<uint32_t>(__half_as_ushort(__ldg(vn_src + t))) << 16;
+          // loads cached in L2 only: a decode step writes the new token's norms in this launch
+          r = __half_as_ushort(__ldcg(kn_src + t));
+          if constexpr (VQ) r |= static_cast<uint32_t>(__half_as_ushort(__ldcg(vn_src + t))) << 16;
           else r |= 0x3c00u << 16;
         }
         return r;

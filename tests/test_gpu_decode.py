@@ -154,11 +154,13 @@ def test_unaligned_norm_rows(vq):
 
 
 @pytest.mark.parametrize("vq", [False, True])
-@pytest.mark.parametrize("d,bits,G", [(128, 4, 4), (64, 2, 8), (128, 3, 1)])
-def test_decode_step(vq, d, bits, G):
+@pytest.mark.parametrize("d,bits,G,Tcap", [(128, 4, 4, 912), (64, 2, 8, 912), (128, 3, 1, 912), (128, 4, 4, 1003),
+                                           (64, 2, 8, 1003)])
+def test_decode_step(vq, d, bits, G, Tcap):
     """axr_decode_step writes the new token exactly as axr_write_keys does and attends over it: the same bits in the
-    cache, the same output as a separate append + attend, and parity with the oracle over the full cache."""
-    B, Hkv, T, Tcap = 3, 2, 900, 912
+    cache, the same output as a separate append + attend, and parity with the oracle over the full cache.  Tcap 1003
+    leaves the norm rows unaligned (norms read from global memory rather than staged with the tiles)."""
+    B, Hkv, T = 3, 2, 900
     Hq = Hkv * G
     k, v, s, kc, kn, vc, vn = oracle_cache(B, Hkv, T, d, bits, 950 + d + bits + G, vq)
     q = W.normal((B, Hq, d), 951, np.float32)
@@ -213,6 +215,52 @@ def test_decode_step(vq, d, bits, G):
         okw = dict(v=v)
     want = oracle.decode_attention(q, kc_w, kn_w, s, bits, 1 / math.sqrt(d), seq_lens=lens, **okw)
     parity.check_outputs(out, want)
+
+
+@pytest.mark.parametrize("vq", [False, True])
+def test_decode_step_many_items(vq):
+    """More (batch row, KV head, split) items than resident blocks, ragged rows (one full, one of a single token):
+    blocks carry several items, some of them holding a new token.  The step writes each token exactly as
+    axr_write_keys does and gives the output of attend over the completed cache."""
+    B, Hkv, G, T, d, bits = 8, 8, 4, 4096, 128, 4
+    Tcap = T + 8
+    Hq = Hkv * G
+    rng = np.random.default_rng(977)
+    lens = rng.integers(1, T + 1, size=B).astype(np.int32)
+    lens[0], lens[1] = T, 1
+    st = cuda(W.sign_vector(d, 978))
+    k = cuda(W.lognormal_rows((B, Hkv, Tcap, d), 979, dtype=np.float16))
+    v = cuda(W.lognormal_rows((B, Hkv, Tcap, d), 980, dtype=np.float16))
+    q = cuda(W.normal((B, Hq, d), 981, np.float32))
+    kc, kn = ops.write_keys(k, st, bits)
+    pos = torch.from_numpy(lens.astype(np.int64) - 1)
+    bi = torch.arange(B)
+    knew = k[bi, :, pos].contiguous()  # [B, Hkv, d]
+    vnew = v[bi, :, pos].contiguous()
+    kc[bi, :, pos] = 0x5a
+    kn[bi, :, pos] = 3.0
+    if vq:
+        vc, vn = ops.write_keys(v, st, bits)
+        vc[bi, :, pos] = 0xa5
+        vn[bi, :, pos] = 2.0
+        vargs = dict(vcodes=vc, vnorms=vn)
+    else:
+        vv = v.clone()
+        vv[bi, :, pos] = 7.0
+        vargs = dict(v=vv)
+    sl = cuda(lens)
+    out = ops.decode_step(q, knew, vnew, kc, kn, st, bits, seq_lens=sl, T=T, **vargs)
+    wk_c, wk_n = ops.write_keys(knew, st, bits)
+    assert torch.equal(kc[bi, :, pos], wk_c) and torch.equal(kn[bi, :, pos], wk_n)
+    if vq:
+        wv_c, wv_n = ops.write_keys(vnew, st, bits)
+        assert torch.equal(vc[bi, :, pos], wv_c) and torch.equal(vn[bi, :, pos], wv_n)
+    else:
+        assert torch.equal(vv[bi, :, pos], vnew)
+    again = ops.attend_decode(q, kc, kn, st, bits, seq_lens=sl, T=T, **vargs)
+    num = torch.linalg.vector_norm(out - again, dim=-1)
+    den = torch.linalg.vector_norm(again, dim=-1)
+    assert bool(torch.all(num <= 2.0 ** -11 * den)), float((num / den).max())
 
 
 def test_dense_matches_oracle_attention():
