@@ -34,11 +34,11 @@ METRIC = "quantized-KV decode attention: keys·heads/s and HBM GB/s vs B200 peak
 UNIT = "keys·heads/s"
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM traffic (read + write bytes) per launch of the timed decode kernel, from the ncu capture summarised in
-# profiles/attend_rows_long_context.md (a B=4 capture, scaled by the units processed).  Valid for the kernel version
-# that capture was taken on; a workload without an entry reports null.
+# DRAM traffic (read + write bytes) per launch of the timed decode kernel, from an ncu capture of dram__bytes_read.sum
+# and dram__bytes_write.sum on the same workload at B=4 (half the units), scaled by the units processed.  Valid for
+# the kernel version that capture was taken on; a workload without an entry reports null.
 TRAFFIC = {
-    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.562048e6 + 3.795712e6),
+    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.582016e6 + 3.122944e6),
 }
 
 WORKLOADS = {

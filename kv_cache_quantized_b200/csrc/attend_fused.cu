@@ -13,7 +13,7 @@ axr_status launch(const DecodeArgs& a, cudaStream_t st) {
   if (rs != AXR_OK) return rs;
   const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent: one block per SM
   k1<<<static_cast<unsigned>(items < kSmCount ? items : kSmCount), S::THREADS, S::bytes, st>>>(a);
-  attend_reduce_kernel<D, VQ><<<a.B * a.Hq, D, 0, st>>>(a);
+  launch_reduce<D, VQ>(a, st);
   return check_launch("axr_attend_decode");
 }
 

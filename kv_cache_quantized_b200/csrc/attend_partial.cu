@@ -15,7 +15,7 @@ axr_status launch(const DecodeArgs& a, cudaStream_t st, const char* what) {
   const long resident = static_cast<long>(S::MIN_BLOCKS) * kSmCount;
   const unsigned grid = static_cast<unsigned>(items < resident ? items : resident);
   k1<<<grid, kDecThreads, S::bytes, st>>>(a);
-  attend_reduce_kernel<D, VQ><<<a.B * a.Hq, D, 0, st>>>(a);
+  launch_reduce<D, VQ>(a, st);
   return check_launch(what);
 }
 

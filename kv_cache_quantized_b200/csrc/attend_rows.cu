@@ -14,7 +14,7 @@ axr_status launch(const DecodeArgs& a, cudaStream_t st) {
   const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent blocks loop over the items
   const long resident = static_cast<long>(S::MIN_BLOCKS) * kSmCount;
   k1<<<static_cast<unsigned>(items < resident ? items : resident), kDecThreads, S::bytes, st>>>(a);
-  attend_reduce_kernel<D, VQ><<<a.B * a.Hq, D, 0, st>>>(a);
+  launch_reduce<D, VQ>(a, st);
   return check_launch("axr_attend_decode");
 }
 

@@ -120,6 +120,9 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
   }
   __syncthreads();
   build_pair_table_kv<BITS>(cent, smem + P::OFF_TAB);
+  // the split merge, launched as this grid's programmatic dependent, may be scheduled from now on (its blocks wait
+  // for this grid's completion before reading anything)
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
   // tiles of earlier items of this block: tile t of an item uses key stage (done + t) % NSK and value stage
   // (done + t) % NSV, and barrier phases of parity ((done + t) / NS) & 1
   int done = 0;

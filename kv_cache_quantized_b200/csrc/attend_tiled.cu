@@ -16,7 +16,7 @@ axr_status launch_tcv(const DecodeArgs& a, cudaStream_t st) {
   const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent: one CTA per SM
   const unsigned grid = static_cast<unsigned>(items < kSmCount ? items : kSmCount);
   k1<<<grid, S::THREADS, S::bytes, st>>>(a);
-  attend_reduce_kernel<128, true><<<a.B * a.Hq, 128, 0, st>>>(a);
+  launch_reduce<128, true>(a, st);
   return check_launch("axr_attend_decode");
 }
 
@@ -29,7 +29,7 @@ axr_status launch_mma(const DecodeArgs& a, cudaStream_t st) {
   const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent blocks loop over the items
   const long resident = static_cast<long>(S::MIN_BLOCKS) * kSmCount;
   k1<<<static_cast<unsigned>(items < resident ? items : resident), kDecThreads, S::bytes, st>>>(a);
-  attend_reduce_kernel<128, true><<<a.B * a.Hq, 128, 0, st>>>(a);
+  launch_reduce<128, true>(a, st);
   return check_launch("axr_attend_decode");
 }
 

@@ -594,6 +594,8 @@ template <int D, bool VQ>
 __global__ void __launch_bounds__(D) attend_reduce_kernel(const __grid_constant__ DecodeArgs a) {
   __shared__ float vec[D];
   const int bh = blockIdx.x, j = threadIdx.x;
+  // launched as a programmatic dependent of the decode kernel: its partials are complete and visible after this
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");
   const float* m = a.ws_m + static_cast<size_t>(bh) * a.splits;
   const float* l = a.ws_l + static_cast<size_t>(bh) * a.splits;
   const float* o = a.ws_o + static_cast<size_t>(bh) * a.splits * D;

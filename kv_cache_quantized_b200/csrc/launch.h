@@ -17,6 +17,25 @@ axr_status ensure_smem(K kernel, size_t bytes, const char* what) {
   return AXR_OK;
 }
 
+// The split merge after a decode kernel, launched as its programmatic dependent: its blocks are scheduled as the
+// decode kernel's blocks retire and wait (griddepcontrol.wait) for that grid's completion and memory flush before
+// reading the partials, so the launch latency overlaps the decode kernel's tail.  Without programmatic launches in
+// the stream (e.g. an older driver) the wait returns at once and ordinary stream order holds.
+template <int D, bool VQ>
+void launch_reduce(const DecodeArgs& a, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.Hq));
+  cfg.blockDim = dim3(D);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, attend_reduce_kernel<D, VQ>, a);
+}
+
 // Row-layout cache, one warp per token range through scores, softmax and the value product, all as warp-level MMAs
 // (attend_fused.cu); only for rows of whole 16-byte chunks (attend_fused_supported).  Used for fp16 values.
 bool attend_fused_supported(int d, int bits);
