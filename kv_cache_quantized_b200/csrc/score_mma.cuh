@@ -143,7 +143,10 @@ __global__ void __launch_bounds__(256, 2) score_mma_kernel(const __grid_constant
     const Geo x0 = geo(blockIdx.x);
     const int n0 = next_with_tiles(blockIdx.x);
     const Geo x1 = n0 >= 0 ? geo(n0) : x0;
-    for (int u = 0; u < NST - 1; ++u) issue_slot(x0, x1, n0 >= 0, 0, u);
+    // bulk copies: warp 0 alone issues (thread 0 the codes, its lanes the norms); the other warps skip the slot
+    // arithmetic, and their cp.async waits find no groups
+    if (!P::BULK || warp == 0)
+      for (int u = 0; u < NST - 1; ++u) issue_slot(x0, x1, n0 >= 0, 0, u);
   }
 
   int done = 0;  // tiles of this block's earlier items
@@ -181,19 +184,21 @@ __global__ void __launch_bounds__(256, 2) score_mma_kernel(const __grid_constant
       const int nt_tok = min(TT, x.vend - t0);
       cp_async_wait<NST - 2>();
       __syncthreads();  // the tile's norms (and cp.async codes) are complete everywhere; the previous stage is free
-      issue_slot(x, xn, nn >= 0, done, tile + NST - 1);
+      if (!P::BULK || warp == 0) issue_slot(x, xn, nn >= 0, done, tile + NST - 1);
       const uint8_t* st = smem + P::OFF_STAGE + static_cast<size_t>(s) * P::STAGE;
       if constexpr (P::BULK) {
         if (!tc::mbar_wait(full + s, static_cast<uint32_t>(((done + tile) / NST) & 1))) *failed = 1;
       }
       // a code tile that never arrived (a copy that did not complete in about a second) poisons the scores
       const float poison = *failed ? __int_as_float(0x7fc00000) : rd;
+      // both M tiles unconditionally (rows past the tile's end hold stale codes -- any byte is a valid table
+      // index -- whose scores are dropped), so that their lookup and MMA chains interleave
+      float sc[2][NT][2];
+#pragma unroll
+      for (int m = 0; m < 2; ++m) mma_scores16<D, BITS, G, false>(st, warp * WT + 16 * m, tab, rep16, B, lane, sc[m]);
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
         const int row0 = warp * WT + 16 * m;
-        if (row0 >= nt_tok) break;
-        float sc[NT][2];
-        mma_scores16<D, BITS, G, false>(st, row0, tab, rep16, B, lane, sc);
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int r = row0 + gq + 8 * i;
@@ -202,7 +207,7 @@ __global__ void __launch_bounds__(256, 2) score_mma_kernel(const __grid_constant
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
               const int h = 4 * nt + tq;
-              if (h < G) out[static_cast<size_t>(h) * a.T + t0 + r] = sc[nt][i] * B.inv[nt] * f;
+              if (h < G) out[static_cast<size_t>(h) * a.T + t0 + r] = sc[m][nt][i] * B.inv[nt] * f;
             }
           }
         }
