@@ -3,17 +3,18 @@
 //
 // AXELRAM Key Points (1st, 2nd items): a token's score is the gather-sum of q~_j c_k at its stored indices, times
 // its stored norm.  The table is read in factored form with both factors split into hi and lo fp16 planes (about 22
-// bits): A = the token's centroids (hi plane, then lo plane, along K), B = the query's planes (column 2h: hi(s_h q~_h)
-// against both A planes, column 2h+1: lo(s_h q~_h) against the hi plane), so that C[t][2h] + C[t][2h+1] = s_h times
-// the score up to the product of the two lo parts.
+// bits each).  One MMA covers 8 tokens: A row g is token g's hi plane and row g + 8 its lo plane (coordinates along
+// K); B column 2h is hi(s_h q~_h) and column 2h + 1 lo(s_h q~_h).  The four products of the two splits then sum to
+// s_h times the score: C[g][2h] + C[g][2h + 1] + C[g + 8][2h] + C[g + 8][2h + 1].
 //
 // K order: the d/2 coordinate pairs are dealt to the four lanes t of a row group in contiguous slices, lane t owning
 // pairs [t d/8, (t + 1) d/8) of every token, so that one load fetches a lane's codes of a row.  K-tile kk, k index
 // 2t + i + 8 r (i, r in {0, 1}) is coordinate 2 p + i of pair p = t d/8 + 2 kk + r.  Fragments of lane (g, t):
-//   A: pairs 2 kk and 2 kk + 1 of the lane's slice, tokens g and g + 8 -- one lookup in the hi/lo pair table gives
-//      the hi register (K-tile kk) and the lo register (the same K-tile of the lo plane) of a pair;
+//   A: one lookup in the hi/lo pair table per pair (2 kk + r) of the lane's slice of token g gives two registers,
+//      the pair's hi plane (row g) and lo plane (row g + 8): with r = 0 they are A registers 0 and 1, with r = 1
+//      registers 2 and 3, so the loads land in the operand as they are;
 //   B: registers built once per (batch, KV head) and kept for the item;
-//   C: head 4 nt + t's sum for tokens g and g + 8 (n-tile nt covers heads 4 nt .. 4 nt + 3).
+//   C: head 4 nt + t's four partial sums for token g (n-tile nt covers heads 4 nt .. 4 nt + 3).
 #pragma once
 
 #include "decode.cuh"
@@ -152,10 +153,9 @@ __device__ __forceinline__ float head_scale_rows(const float* __restrict__ row) 
 
 template <int D, int G>
 struct MmaB {
-  static constexpr int KT = D / 16;              // K-tiles per plane
+  static constexpr int KT = D / 16;              // K-tiles
   static constexpr int NT = G <= 4 ? 1 : 2;      // n-tiles of 8 columns
-  uint32_t bh[NT][KT][2];                        // against the hi plane of A
-  uint32_t bl[NT][KT][2];                        // against the lo plane of A (lo columns zero)
+  uint32_t bh[NT][KT][2];                        // columns 2h, 2h + 1: hi and lo plane of s_h q~_h
   float inv[NT];                                 // 1 / scale of head 4 nt + t
 };
 
@@ -186,7 +186,6 @@ __device__ __forceinline__ void mma_b_build(const float* __restrict__ qs, const 
         }
         const __half2 p = __floats2half2_rn(v[0], v[1]);
         B.bh[nt][kk][r] = *reinterpret_cast<const uint32_t*>(&p);
-        B.bl[nt][kk][r] = hi_col ? B.bh[nt][kk][r] : 0u;
       }
     }
     float sc2 = 1.f;
@@ -197,8 +196,8 @@ __device__ __forceinline__ void mma_b_build(const float* __restrict__ qs, const 
 }
 
 // Block-wide build of the B fragments into shared memory, one 32-bit entry per thread: bs[e][lane] with
-// e = (nt KT + kk) 2 + r holds the hi-column register of MmaB::bh[nt][kk][r] for that lane (mma_b_build's values);
-// the lo-column registers and the inverse scales are derived on load (mma_b_load).
+// e = (nt KT + kk) 2 + r holds MmaB::bh[nt][kk][r] for that lane (mma_b_build's values); the inverse scales are
+// derived on load (mma_b_load).
 template <int D, int G>
 __device__ __forceinline__ void mma_b_stage(const float* __restrict__ qs, const float* __restrict__ scl,
                                             uint32_t* __restrict__ bs) {
@@ -226,17 +225,12 @@ template <int D, int G>
 __device__ __forceinline__ void mma_b_load(const uint32_t* __restrict__ bs, const float* __restrict__ scl, int lane,
                                            MmaB<D, G>& B) {
   constexpr int KT = MmaB<D, G>::KT, NT = MmaB<D, G>::NT;
-  const bool hi_col = ((lane >> 2) & 1) == 0;
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
     for (int kk = 0; kk < KT; ++kk)
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const uint32_t x = bs[((nt * KT + kk) * 2 + r) * 32 + lane];
-        B.bh[nt][kk][r] = x;
-        B.bl[nt][kk][r] = hi_col ? x : 0u;
-      }
+      for (int r = 0; r < 2; ++r) B.bh[nt][kk][r] = bs[((nt * KT + kk) * 2 + r) * 32 + lane];
     const int h = 4 * nt + (lane & 3);
     B.inv[nt] = h < G ? 1.f / scl[h] : 1.f;
   }
@@ -257,7 +251,7 @@ __device__ __forceinline__ void mma_scores16(const uint8_t* st, int row0, const 
   load_run<R, NB, SWZ>(st, (row0 + gq + 8) * R + tq * NB, w1);
 #pragma unroll
   for (int i = (NB + 3) / 4; i < NW; ++i) w0[i] = w1[i] = 0u;
-  float c[2][NT][4];
+  float c[2][NT][4];  // [token g, token g + 8][n-tile]
 #pragma unroll
   for (int x = 0; x < 2; ++x)
 #pragma unroll
@@ -270,20 +264,21 @@ __device__ __forceinline__ void mma_scores16(const uint8_t* st, int row0, const 
   };
 #pragma unroll
   for (int kk = 0; kk < KT; ++kk) {
+    // {hi, lo} of pairs 2 kk (A registers 0, 1) and 2 kk + 1 (registers 2, 3) of token g, then of token g + 8
     const uint2 e00 = *reinterpret_cast<const uint2*>(tab + off(w0, 2 * kk));
-    const uint2 e10 = *reinterpret_cast<const uint2*>(tab + off(w1, 2 * kk));
     const uint2 e01 = *reinterpret_cast<const uint2*>(tab + off(w0, 2 * kk + 1));
+    const uint2 e10 = *reinterpret_cast<const uint2*>(tab + off(w1, 2 * kk));
     const uint2 e11 = *reinterpret_cast<const uint2*>(tab + off(w1, 2 * kk + 1));
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      mma_m16n8k16(c[kk & 1][nt], e00.x, e10.x, e01.x, e11.x, B.bh[nt][kk][0], B.bh[nt][kk][1]);
-      mma_m16n8k16(c[kk & 1][nt], e00.y, e10.y, e01.y, e11.y, B.bl[nt][kk][0], B.bl[nt][kk][1]);
+      mma_m16n8k16(c[0][nt], e00.x, e00.y, e01.x, e01.y, B.bh[nt][kk][0], B.bh[nt][kk][1]);
+      mma_m16n8k16(c[1][nt], e10.x, e10.y, e11.x, e11.y, B.bh[nt][kk][0], B.bh[nt][kk][1]);
     }
   }
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    out[nt][0] = (c[0][nt][0] + c[1][nt][0]) + (c[0][nt][1] + c[1][nt][1]);
-    out[nt][1] = (c[0][nt][2] + c[1][nt][2]) + (c[0][nt][3] + c[1][nt][3]);
+    out[nt][0] = (c[0][nt][0] + c[0][nt][1]) + (c[0][nt][2] + c[0][nt][3]);
+    out[nt][1] = (c[1][nt][0] + c[1][nt][1]) + (c[1][nt][2] + c[1][nt][3]);
   }
 }
 
