@@ -38,7 +38,7 @@ L2_BYTES = 126 * 1024 * 1024
 # and dram__bytes_write.sum on the same workload at B=4 (half the units), scaled by the units processed.  Valid for
 # the kernel version that capture was taken on; a workload without an entry reports null.
 TRAFFIC = {
-    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.582016e6 + 3.122944e6),
+    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.560768e6 + 3.692800e6),
 }
 
 WORKLOADS = {
