@@ -5,17 +5,21 @@
 namespace axr {
 namespace {
 
+// The C entry point a launch serves, for error messages: decode steps carry the new token.
+const char* entry_name(const DecodeArgs& a) { return a.knew != nullptr ? "axr_decode_step" : "axr_attend_decode"; }
+
 template <int D, int BITS, int G, bool VQ>
 axr_status launch(const DecodeArgs& a, cudaStream_t st) {
   using S = RowsPlan<D, BITS, G, VQ>;
   auto k1 = attend_rows_kernel<D, BITS, G, VQ>;
-  axr_status rs = ensure_smem(k1, S::bytes, "axr_attend_decode");
+  const char* what = entry_name(a);
+  axr_status rs = ensure_smem(k1, S::bytes, what);
   if (rs != AXR_OK) return rs;
   const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent blocks loop over the items
   const long resident = static_cast<long>(S::MIN_BLOCKS) * kSmCount;
   k1<<<static_cast<unsigned>(items < resident ? items : resident), kDecThreads, S::bytes, st>>>(a);
   launch_reduce<D, VQ>(a, st);
-  return check_launch("axr_attend_decode");
+  return check_launch(what);
 }
 
 template <int D, int BITS>
@@ -26,7 +30,7 @@ axr_status by_g(int G, bool vq, const DecodeArgs& a, cudaStream_t st) {
     case 4: return vq ? launch<D, BITS, 4, true>(a, st) : launch<D, BITS, 4, false>(a, st);
     case 8: return vq ? launch<D, BITS, 8, true>(a, st) : launch<D, BITS, 8, false>(a, st);
   }
-  return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: G=%d", G);
+  return set_error(AXR_EUNSUPPORTED, "%s: G=%d", entry_name(a), G);
 }
 
 template <int D>
@@ -37,7 +41,7 @@ axr_status by_bits(int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t s
     case 3: return by_g<D, 3>(G, vq, a, st);
     case 4: return by_g<D, 4>(G, vq, a, st);
   }
-  return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: bits=%d", bits);
+  return set_error(AXR_EUNSUPPORTED, "%s: bits=%d", entry_name(a), bits);
 }
 
 }  // namespace
@@ -45,7 +49,7 @@ axr_status by_bits(int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t s
 axr_status attend_rows_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st) {
   if (d == 64) return by_bits<64>(bits, G, vq, a, st);
   if (d == 128) return by_bits<128>(bits, G, vq, a, st);
-  return set_error(AXR_EUNSUPPORTED, "axr_attend_decode: d=%d", d);
+  return set_error(AXR_EUNSUPPORTED, "%s: d=%d", entry_name(a), d);
 }
 
 }  // namespace axr
