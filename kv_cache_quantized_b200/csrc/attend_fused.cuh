@@ -8,8 +8,8 @@
 //
 // Block structure: one block of NW warps per SM, persistent over (batch, KV head, split) items.  Tiles of 128 tokens
 // (codes, values and norms: one bulk copy each, completing on the stage's mbarrier) stream through NS stages; warp w
-// takes the two M = 16 tiles [32 (w % 4), 32 (w % 4) + 32) of every (NW / 4)-th tile.  Per visit the warp scores its
-// 32 tokens (lane (g, t) holds head t's scores of tokens g and g + 8 of each M tile), updates its own running max and
+// takes the two 16-token groups [32 (w % 4), 32 (w % 4) + 32) of every (NW / 4)-th tile.  Per visit the warp scores its
+// 32 tokens (lane (g, t) holds head t's scores of tokens g and g + 8 of each group), updates its own running max and
 // sum, moves the weights p n^V / sqrt(d) into the B-operand layout of the value MMA with warp shuffles (heads as
 // columns, token pairs along K) and accumulates O^T (d x heads) += V^T P^T, the A operand (V^T) coming from the same
 // pair table (hi fp16 copies) with two byte permutes per register.  The last of the four warps to leave a stage
@@ -24,7 +24,7 @@ namespace axr {
 template <int D, int BITS, int G, bool VQ>
 struct FusedPlan {
   static constexpr int TT = 128;                         // tokens per tile
-  static constexpr int MPW = 2;                          // M = 16 tiles per warp per visit
+  static constexpr int MPW = 2;                          // 16-token groups per warp per visit
   static constexpr int WPT = TT / (16 * MPW);            // warps sharing one tile
   static constexpr int NW = G <= 4 ? 16 : 8;             // warps per block (G = 8 needs more registers)
   static constexpr int THREADS = 32 * NW;
@@ -223,7 +223,7 @@ attend_fused_kernel(const __grid_constant__ DecodeArgs a) {
       const int nt_tok = min(TT, end - t0);
       const int row_w = (warp % WPT) * 16 * MPW;  // first of this warp's tokens in the tile
 
-      // ---- key scores of the warp's MPW x 16 tokens; lane (g, t) holds tokens g, g + 8 of each M tile, head 4 nt + t
+      // ---- key scores of the warp's MPW x 16 tokens; lane (g, t) holds tokens g, g + 8 of each group, head 4 nt + t
       float z[MPW][NT][2];
 #pragma unroll
       for (int m = 0; m < MPW; ++m) mma_scores16<D, BITS, G, false, true>(st, row_w + 16 * m, tab, repk, B, lane, z[m]);

@@ -7,7 +7,7 @@
 // values the product stays in the rotated domain (one inverse transform per output, in the merge kernel).
 //
 // Block structure (256 threads, persistent over (batch, KV head, split) items): scoring warps 0..3 own tokens
-// [32 w, 32 w + 32) of every 128-token tile, score them as two M = 16 tiles (lane (g, t) gets head t's scores of
+// [32 w, 32 w + 32) of every 128-token tile, score them as two 16-token groups (lane (g, t) gets head t's scores of
 // tokens g, g + 8, 16 + g, 24 + g) and keep the running max and sum of their tokens (online softmax); value warp
 // 4 + w consumes the same tokens one tile later against the same running max.  One block barrier per tile; the
 // streams of the four warps are merged at the end of an item.

@@ -2,14 +2,15 @@
 //
 // AXELRAM Key Points (1st, 2nd items): every cached token's score is the gather-sum of the query's table entries at
 // the token's stored indices, times its stored norm.  The table is read in factored form (mma_score.cuh): each
-// token's centroids, split into hi and lo fp16 planes (about 22 bits), form a row of A; the query's hi/lo planes
-// form B, built once per (batch, KV head) and kept in registers; lane (g, t) ends with head t's score of tokens g
-// and g + 8 of an M = 16 tile.  There is no shuffle reduction and no cross-warp hand-off inside a tile: warp w owns
-// tokens [32 w, 32 w + 32) of each 256-token tile (two M = 16 tiles).  Code tiles arrive as one bulk copy each
-// (completing on a per-stage mbarrier), norms as 16-byte cp.async chunks, four stages deep, with one block barrier
-// per tile.  Blocks are persistent (two per SM) over (batch, KV head, split) items and build the pair table once;
-// the tile pipeline runs on from one item into the next (slots past an item's end carry the next item's first
-// tiles), the next item's queries are fetched one item ahead, and the B fragments are built once per block.
+// token's centroids, split into hi and lo fp16 planes (about 22 bits), form two rows of A (one MMA covers 8
+// tokens); the query's hi/lo planes form B, built once per (batch, KV head) and kept in registers; lane (g, t) ends
+// with head t's score of tokens g and g + 8 of a 16-token group.  There is no shuffle reduction and no cross-warp
+// hand-off inside a tile: warp w owns tokens [32 w, 32 w + 32) of each 256-token tile (two 16-token groups).  Code
+// tiles arrive as one bulk copy each (completing on a per-stage mbarrier), norms as 16-byte cp.async chunks, four
+// stages deep, issued by warp 0 alone, with one block barrier per tile.  Blocks are persistent (two per SM) over
+// (batch, KV head, split) items and build the pair table once; the tile pipeline runs on from one item into the
+// next (slots past an item's end carry the next item's first tiles), the next item's queries are fetched one item
+// ahead, and the B fragments are built once per block.
 #pragma once
 
 #include "mma_score.cuh"
