@@ -103,8 +103,4 @@ __device__ __forceinline__ uint32_t bits_at(const uint32_t* w, int pos) {
   return __funnelshift_r(w[wi], w[wi + 1], sh) & ((1u << B) - 1u);
 }
 
-__device__ __forceinline__ float half_bits_to_float(uint16_t h) {
-  return __half2float(__ushort_as_half(h));
-}
-
 }  // namespace axr

@@ -73,26 +73,6 @@ __device__ inline void cursor_next(const DecodeArgs& a, TileCursor& c) {
   c.ntr = c.b < a.B ? row_tiles(a, c.b) : 0;
 }
 
-// qs[g][j] = mult * (H (s .* q_g))_j for the G heads, by the nwarps warps of one role (rwarp = warp within it).
-template <int D, int G>
-__device__ __forceinline__ void transform_queries_role(const float* __restrict__ q, const int8_t* __restrict__ signs,
-                                                       float mult, float* __restrict__ qs, int rwarp, int nwarps) {
-  constexpr int VPL = WarpVec<D>::VPL;
-  const int lane = threadIdx.x & 31;
-  const float norm = mult * rsqrtf(static_cast<float>(D));
-  for (int g = rwarp; g < G; g += nwarps) {
-    float v[VPL];
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int j = lane * VPL + i;
-      v[i] = q[g * D + j] * sign_of(signs[j]);
-    }
-    fwht_warp<D>(v, lane);
-#pragma unroll
-    for (int i = 0; i < VPL; ++i) qs[g * D + lane * VPL + i] = v[i] * norm;
-  }
-}
-
 // A wait whose outcome is the same in every lane of the warp (the tcgen05 loads and stores that follow are
 // warp-collective).
 __device__ __forceinline__ bool warp_wait(uint64_t* mbar, uint32_t parity) {

@@ -182,10 +182,6 @@ __device__ __forceinline__ uint32_t pair_off(const uint32_t* w, int i, uint32_t 
   }
 }
 
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
 // Power-of-two range scale of one head's query operand: 2^(14 - e) with |mult| * ||q|| in [2^(e-1), 2^e).  Every
 // |q~_j| is at most |mult| * ||q|| (the transform is orthonormal), so the scaled factors stay below 2^14 in fp16
 // while keeping fp16's relative precision; the epilogue divides it out.  Computed by a whole warp from the query in
