@@ -297,9 +297,11 @@ def test_split_count_invariance():
     assert np.max(np.abs(a - b)) <= 1e-5 * np.max(np.abs(a))
 
 
-def _full_size(w, samples, seed_q=None):
+def _full_size(w, samples, seed_q=None, step=False):
     """Full-size workload in the benchmark's launch configuration: the cache is written on the GPU, attention runs
-    on the GPU; sampled (batch, head) outputs are recomputed by the oracle from the same host inputs."""
+    on the GPU; sampled (batch, head) outputs are recomputed by the oracle from the same host inputs.  With step,
+    also the call the benchmark times: axr_decode_step writing token T - 1 itself over a cache whose position T - 1
+    is stale must leave the cache as the writer does, and its sampled outputs must match the oracle too."""
     inp = W.decode_inputs(w)
     k, v, q, s = inp["k"], inp["v"], inp["q"], inp["signs"]
     st = cuda(s)
@@ -310,6 +312,27 @@ def _full_size(w, samples, seed_q=None):
     else:
         out = ops.attend_decode(cuda(q), kc, kn, st, w.bits, v=cuda(v))
     out = out.cpu().numpy()
+    got = None
+    if step:
+        kc_s, kn_s = kc.clone(), kn.clone()
+        kc_s[:, :, -1] = 0x5a
+        kn_s[:, :, -1] = 3.0
+        knew, vnew = cuda(k[:, :, -1]), cuda(v[:, :, -1])  # [B, Hkv, d]
+        if w.v_quant:
+            vc_s, vn_s = vc.clone(), vn.clone()
+            vc_s[:, :, -1] = 0xa5
+            vn_s[:, :, -1] = 2.0
+            vargs = dict(vcodes=vc_s, vnorms=vn_s)
+        else:
+            v_s = cuda(v)
+            v_s[:, :, -1] = 7.0
+            vargs = dict(v=v_s)
+        got = ops.decode_step(cuda(q), knew, vnew, kc_s, kn_s, st, w.bits, **vargs).cpu().numpy()
+        assert torch.equal(kc_s, kc) and torch.equal(kn_s, kn)
+        if w.v_quant:
+            assert torch.equal(vc_s, vc) and torch.equal(vn_s, vn)
+        else:
+            assert torch.equal(v_s, cuda(v))
     kc_h, kn_h = kc.cpu().numpy(), kn.cpu().numpy()
     vc_h = vn_h = None
     if w.v_quant:
@@ -329,6 +352,8 @@ def _full_size(w, samples, seed_q=None):
             want = oracle.decode_attention(q[b:b + 1, h:h + 1], okc[None, None], okn[None, None], s, w.bits, scale,
                                            v=v[b:b + 1, hk:hk + 1])
         parity.check_outputs(out[b:b + 1, h:h + 1], want)
+        if got is not None:
+            parity.check_outputs(got[b:b + 1, h:h + 1], want)
         # and the scores of this head against the oracle on the oracle's codes
         sc = ops.score(cuda(q[b:b + 1, hk * w.G:(hk + 1) * w.G]), cuda(okc[None, None]), cuda(okn[None, None]), st,
                        w.bits, scale=scale).cpu().numpy()[0, h - hk * w.G]
@@ -338,11 +363,11 @@ def _full_size(w, samples, seed_q=None):
 
 
 def test_llama8b_shaped_decode_full_size():
-    _full_size(W.LLAMA8B_DECODE, [(0, 0), (3, 13), (7, 31)])
+    _full_size(W.LLAMA8B_DECODE, [(0, 0), (3, 13), (7, 31)], step=True)
 
 
 def test_long_context_kv_quantized_full_size():
-    _full_size(W.LONG_CONTEXT, [(0, 1), (5, 22), (7, 31)])
+    _full_size(W.LONG_CONTEXT, [(0, 1), (5, 22), (7, 31)], step=True)
 
 
 @pytest.mark.parametrize("B,T,bits,d", [(1, 131072, 1, 64), (1, 131072, 3, 128), (64, 4096, 2, 128),
