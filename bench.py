@@ -177,6 +177,8 @@ def cpu_baseline(w, seconds=10.0):
 def _packed_inputs(tensors, device=None, pinned=False):
     """One byte buffer holding `tensors` back to back, each at a 16-byte aligned offset, and a view of each (its
     dtype and shape) into it; filled with the tensors' values.  On the host, pinned if asked."""
+    import torch
+
     offs, n = [], 0
     for t in tensors:
         n = (n + 15) // 16 * 16

@@ -1,0 +1,45 @@
+"""Host-side helpers of the benchmark, on the CPU: the packed input buffer of the end-to-end arm and the
+algorithmic byte counts behind the roofline fraction."""
+
+import numpy as np
+import torch
+
+import bench
+from kv_cache_quantized_b200 import workloads as W
+
+
+def test_packed_inputs_views_hold_the_tensors():
+    q = torch.randn(8, 32, 128)
+    k = torch.randn(8, 8, 128).half()
+    v = torch.randn(8, 8, 128).half()
+    buf, (qv, kv, vv) = bench._packed_inputs([q, k, v])
+    assert buf.dtype == torch.uint8
+    assert buf.numel() == q.numel() * 4 + k.numel() * 2 + v.numel() * 2  # offsets already 16-byte multiples
+    for view, t in ((qv, q), (kv, k), (vv, v)):
+        assert view.dtype == t.dtype and view.shape == t.shape and view.is_contiguous()
+        assert view.data_ptr() % 16 == 0
+        assert torch.equal(view, t)
+    # one copy into the buffer refreshes every view
+    buf2, views2 = bench._packed_inputs([torch.zeros_like(q), torch.zeros_like(k), torch.zeros_like(v)])
+    buf2.copy_(buf)
+    assert all(torch.equal(a, b) for a, b in zip(views2, (q, k, v)))
+
+
+def test_packed_inputs_pads_odd_sizes_to_16_bytes():
+    a = torch.arange(3, dtype=torch.float16)   # 6 bytes
+    b = torch.arange(5, dtype=torch.float32)   # 20 bytes, starts at 16
+    buf, (av, bv) = bench._packed_inputs([a, b])
+    assert buf.numel() == 16 + 20
+    assert bv.data_ptr() - buf.data_ptr() == 16
+    assert torch.equal(av, a) and torch.equal(bv, b)
+
+
+def test_algorithmic_bytes_per_key_head():
+    # long context: 64 B key codes + 2 B norm, and the same for quantized values
+    assert bench._bytes_per_key_head(W.LONG_CONTEXT) == 132
+    # Llama-shaped: 66 B of key codes and norm + 256 B of fp16 values
+    assert bench._bytes_per_key_head(W.LLAMA8B_DECODE) == 322
+    w = W.LONG_CONTEXT
+    units = w.B * w.Hkv * w.T
+    assert units * bench._bytes_per_key_head(w) == 276_824_064
+    assert np.isclose(bench.TRAFFIC[w.name] / (units * bench._bytes_per_key_head(w)), 1.028, atol=0.01)
