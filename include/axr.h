@@ -14,6 +14,9 @@
  *    a caller-provided workspace whose size comes from the matching *_workspace_bytes() function.
  *  - Device work is asynchronous on `stream`.  Argument errors are detected on the host and returned before any
  *    launch (no device work is queued).  Launch errors come from cudaGetLastError and return AXR_ECUDA.
+ *  - The decode entry points launch their split merge as a programmatic dependent of the decode kernel on the same
+ *    stream (its blocks wait on the device for the decode kernel's completion); work the caller enqueues before or
+ *    after keeps plain stream order.
  *  - On any status other than AXR_OK, axr_last_error() returns a thread-local human-readable message.
  *  - Fixed notation: d head dim (power of two), b bits per index, L = 2^b levels, s the +-1 sign vector, H the
  *    Sylvester Walsh-Hadamard matrix scaled by 1/sqrt(d) (symmetric, H*H = I), G = Hq/Hkv (query head h reads KV
