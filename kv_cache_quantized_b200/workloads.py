@@ -77,6 +77,33 @@ def layer_scaled_keys(shape, seed: int, dtype=np.float16) -> np.ndarray:
     return (x * f.reshape((-1,) + (1,) * (len(shape) - 1))).astype(dtype)
 
 
+def outlier_direction_keys(shape, seed: int, pattern_seed: int, n_out: int = 8, m: float = 4.0,
+                           layer_scale: bool = True, dtype=np.float16) -> np.ndarray:
+    """Keys [Lyr, S, Hkv, N, d] with structure the sign pattern can see: N(0,1) noise plus a per-token multiple of a
+    fixed outlier direction, x_t = z_t + a_t mu, a_t ~ N(0,1), where mu (one per layer and KV head) is +-m on n_out
+    channels with fixed signs and 0 elsewhere (outlier channels with fixed sign relations), the whole layer times
+    10^U(-1,1) if layer_scale (layer-wise norm heterogeneity).  The outlier patterns and layer factors come from
+    pattern_seed alone, so calibration and held-out sets drawn with different `seed` share them.  Under the
+    transform mu becomes H(s * mu), and the sign pattern decides whether that varying direction lands on a few
+    coordinates (clipped by the codebook) or spreads over many."""
+    g = rng(seed)
+    gp = rng(pattern_seed)
+    Lyr, S, Hkv, N, d = shape
+    x = g.standard_normal(shape)
+    a = g.standard_normal((Lyr, S, Hkv, N))
+    nb = min(n_out, d)
+    for layer in range(Lyr):
+        for h in range(Hkv):
+            ch = gp.choice(d, size=nb, replace=False)
+            mu = np.zeros(d)
+            mu[ch] = m * np.where(gp.random(nb) < 0.5, -1.0, 1.0)
+            x[layer, :, h] += a[layer, :, h, :, None] * mu
+    if layer_scale:
+        f = 10.0 ** gp.uniform(-1.0, 1.0, size=Lyr)
+        x *= f.reshape((-1,) + (1,) * (len(shape) - 1))
+    return x.astype(dtype)
+
+
 # ---------------------------------------------------------------------------------------------------------------
 # Named workloads.
 # ---------------------------------------------------------------------------------------------------------------
@@ -160,14 +187,18 @@ def decode_inputs(w: Decode, T: int | None = None, B: int | None = None):
 
 
 def calibration_inputs(c: Calibration, layers: int | None = None, seqs: int | None = None,
-                       tokens: int | None = None, n_cand: int | None = None):
-    """Host tensors of a calibration set (optionally reduced).  q f32, k/v f16, candidates int8."""
+                       tokens: int | None = None, n_cand: int | None = None, keys: str = "layer_scaled"):
+    """Host tensors of a calibration set (optionally reduced).  q f32, k/v f16, candidates int8.  keys:
+    "layer_scaled" (i.i.d. N(0,1) times the per-layer factor) or "outlier_direction" (outlier_direction_keys)."""
     Lyr = c.layers if layers is None else layers
     S = c.seqs if seqs is None else seqs
     N = c.tokens if tokens is None else tokens
     C = c.n_cand if n_cand is None else n_cand
     q = normal((Lyr, S, c.Hq, N, c.d), c.seed, dtype=np.float32)
-    k = layer_scaled_keys((Lyr, S, c.Hkv, N, c.d), c.seed + 1)
+    if keys == "outlier_direction":
+        k = outlier_direction_keys((Lyr, S, c.Hkv, N, c.d), c.seed + 1, c.seed + 5)
+    else:
+        k = layer_scaled_keys((Lyr, S, c.Hkv, N, c.d), c.seed + 1)
     v = normal((Lyr, S, c.Hkv, N, c.d), c.seed + 2, dtype=np.float16)
     return {"q": q, "k": k, "v": v, "candidates": candidate_signs(C, c.d, c.seed + 3)}
 
@@ -207,3 +238,13 @@ def outlier_keys_device(shape, seed: int, device, n_outliers: int = 4, factor: f
     ch = torch.as_tensor(outlier_channels(shape[-1], n_outliers, seed + 7919), device=device)
     x[..., ch] *= factor
     return x.to(dtype)
+
+
+def layer_scaled_keys_device(shape, seed: int, device, dtype=None):
+    """layer_scaled_keys' distribution drawn on the device: N(0,1) times a per-layer factor 10^U(-1,1)."""
+    import torch
+    dtype = torch.float16 if dtype is None else dtype
+    g = _torch_gen(seed, device)
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    f = 10.0 ** (2.0 * torch.rand(shape[0], generator=g, device=device, dtype=torch.float32) - 1.0)
+    return (x * f.view((-1,) + (1,) * (len(shape) - 1))).to(dtype)

@@ -25,7 +25,9 @@ ai-navigate-news digest -- Key Points and Abstract -- and by the mlsanity index 
   reconstructed explicitly).
 * Sign-pattern selection (Key Points, 4th item; Abstract): a one-time, gradient-free choice among candidate sign
   vectors on a few calibration samples.  Objective taken here: attention-output MSE of quantized-K attention
-  against unquantized fp64 attention; the first index of the minimum wins.
+  against unquantized fp64 attention; the first index of the minimum wins.  Over the whole model (one sign
+  vector), or layer by layer (one sign vector per layer: the pages trace the sensitivity to layer-wise norm
+  heterogeneity).
 
 Every function below is pinned by a ``-m "not gpu"`` test against closed forms, library routines or invariants
 (tests/test_oracle_*.py).  Nothing here is "parity unpinned".
@@ -55,6 +57,7 @@ __all__ = [
     "decode_attention",
     "attention",
     "select_signs",
+    "select_signs_per_layer",
     "multiplication_counts",
 ]
 
@@ -349,6 +352,31 @@ def select_signs(q, k, v, candidates, bits, causal=True):
         out = attention(q, khat, v, causal)
         mse[ci] = np.mean((out - ref) ** 2)
     return mse, int(np.argmin(mse))
+
+
+def select_signs_per_layer(q, k, v, candidates, bits, causal=True):
+    """One sign vector per layer (the sensitivity is traced to layer-wise norm heterogeneity: AXELRAM Abstract;
+    Key Points, 3rd and 4th items).  For every layer l and candidate c, the MSE of quantized-K attention against
+    fp64 unquantized attention over every (sequence, query head, position, dim) of layer l only; each layer picks
+    the first index of its own minimum.
+
+    q [Lyr, S, Hq, N, d]; k, v [Lyr, S, Hkv, N, d]; candidates [C, d] of +-1.
+    Returns (mse float64 [Lyr, C], best int64 [Lyr]).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    d = q.shape[-1]
+    Lyr = q.shape[0]
+    mse = np.zeros((Lyr, len(candidates)), dtype=np.float64)
+    for layer in range(Lyr):
+        ref = attention(q[layer], k[layer], v[layer], causal)
+        for ci, s in enumerate(candidates):
+            codes, n16 = write(k[layer], s, bits)
+            khat = dequantize(codes, n16, s, bits, d)
+            out = attention(q[layer], khat, v[layer], causal)
+            mse[layer, ci] = np.mean((out - ref) ** 2)
+    return mse, np.argmin(mse, axis=1)
 
 
 # ---------------------------------------------------------------------------------------------------------------
