@@ -105,3 +105,62 @@ def test_sign_applied_after_transform_is_caught(monkeypatch):
     _patch(monkeypatch, "rotate", bad_rotate)
     with pytest.raises(AssertionError):
         TW.test_rotate_inverse(8)
+
+
+# ---- LOOKAT oracle -------------------------------------------------------------------------------------------------
+
+import oracle.lookat as LK  # noqa: E402
+import tests.test_oracle_lookat as TL  # noqa: E402
+
+
+def _patch_lk(monkeypatch, name, fn):
+    monkeypatch.setattr(LK, name, fn)
+    monkeypatch.setattr(oracle, name, fn)
+
+
+def test_farthest_centroid_is_caught(monkeypatch):
+    monkeypatch.setattr(LK, "_nearest", lambda dist: np.argmax(dist, axis=1))
+    with pytest.raises(AssertionError):
+        TL.test_fp32_decision_matches_fp64_nearest_except_near_ties()
+
+
+def test_interleaved_subspaces_are_caught(monkeypatch):
+    def bad_split(x, m):  # subspace i takes coordinates i, i + m, i + 2m, ... instead of a contiguous run
+        x = np.asarray(x)
+        d = x.shape[-1]
+        return np.swapaxes(x.reshape(x.shape[:-1] + (d // m, m)), -1, -2)
+    _patch_lk(monkeypatch, "pq_split", bad_split)
+    with pytest.raises(AssertionError):
+        TL.test_per_subspace_encoding_is_the_product_codebook_search()
+
+
+def test_transposed_adc_table_is_caught(monkeypatch):
+    real = LK.pq_table
+
+    def bad_score(q, codes, codebooks, scale=1.0):  # the table read with the code as the row index
+        tab = real(q, codebooks)
+        codes = np.asarray(codes)
+        m, K = tab.shape
+        full = np.zeros((max(m, K), max(m, K)))
+        full[:m, :K] = tab
+        return scale * full.T[np.arange(m)[None, :], codes].sum(axis=-1)
+    _patch_lk(monkeypatch, "pq_score", bad_score)
+    with pytest.raises(AssertionError):
+        TL.test_adc_score_is_the_reconstructed_dot_product(4, 16)
+
+
+def test_kmeans_mean_without_division_is_caught(monkeypatch):
+    def bad_kmeans(xs, init, iters):
+        c = np.asarray(init, dtype=np.float32).copy()
+        x64 = np.asarray(xs).astype(np.float64)
+        assign = np.zeros(len(x64), dtype=np.int64)
+        for _ in range(iters):
+            assign = LK._nearest(LK.pq_distances_f32(xs, c))
+            for k in range(c.shape[0]):
+                members = x64[assign == k]
+                if len(members):
+                    c[k] = members.sum(axis=0).astype(np.float32)
+        return c, assign
+    _patch_lk(monkeypatch, "pq_kmeans", bad_kmeans)
+    with pytest.raises(AssertionError):
+        TL.test_kmeans_matches_scikit_learn_lloyd()
