@@ -31,6 +31,11 @@ sys.path.insert(0, ROOT)
 from kv_cache_quantized_b200 import workloads as W  # noqa: E402
 
 METRIC = "quantized-KV decode attention: keys·heads/s and HBM GB/s vs B200 peak"
+# What the timed kernel computes: u8 packed codes; key scores as fp16 x fp16 -> fp32 MMAs on hi/lo planes of the
+# centroids and the query (about 22 bits each); the value product as fp16 x fp16 -> fp32 MMAs of the weights and the
+# hi plane of the value centroids; softmax and the merge in fp32.
+DTYPE = "u8 codes; fp16 hi/lo x fp16 hi/lo -> fp32 MMA (keys), fp16 x fp16 -> fp32 MMA (values), fp32 softmax"
+NOMINAL_HBM_GBS = 8000.0  # the HBM bandwidth the target is stated against (about 8 TB/s), beside the measured copy
 UNIT = "keys·heads/s"
 L2_BYTES = 126 * 1024 * 1024
 
@@ -130,48 +135,125 @@ def _dist():
     return ws, rank, local
 
 
-def cpu_baseline(w, seconds=10.0):
-    """The fp64 oracle, as it stands, on one core: decode steps of single (batch row, KV head) units of the same
-    workload (G query heads over T cached tokens, plus the new token's write), repeated for about `seconds`."""
+def _oracle_unit(w, kc, kn, vc, vn, k, v, q, s, hk):
+    """One (batch row, KV head) unit of the decode step through the oracle: the new token's write, then G query
+    heads over the T cached tokens."""
     import oracle
-    try:
-        from threadpoolctl import threadpool_limits
-    except ImportError:  # pragma: no cover
-        threadpool_limits = None
+    scale = 1.0 / math.sqrt(w.d)
+    nk = oracle.write(k[-1:], s, w.bits)
+    if w.v_quant:
+        oracle.write(v[-1:], s, w.bits)
+    kc[-1:], kn[-1:] = nk
+    qq = q[hk * w.G:(hk + 1) * w.G][None]
+    if w.v_quant:
+        oracle.decode_attention(qq, kc[None, None], kn[None, None], s, w.bits, scale, vcodes=vc[None, None],
+                                vn16=vn[None, None])
+    else:
+        oracle.decode_attention(qq, kc[None, None], kn[None, None], s, w.bits, scale, v=v[None, None])
+
+
+def _oracle_proc(w, seed, cmd_q, res_q, ready):
+    """Spawned oracle process: draws one (batch row, KV head) unit of the workload's shape from its own seed, then
+    for every command `seconds` runs decode steps of that unit through the oracle on one thread for that long and
+    reports (unit-steps, seconds).  None ends it."""
+    from threadpoolctl import threadpool_limits
+    import oracle
+    with threadpool_limits(1):
+        if w.keys == "outlier":
+            k = W.outlier_keys((w.T, w.d), seed)
+        else:
+            k = W.lognormal_rows((w.T, w.d), seed, dtype=np.float16)
+        v = (W.lognormal_rows((w.T, w.d), seed + 1, dtype=np.float16) if w.v_quant
+             else W.normal((w.T, w.d), seed + 1, np.float16))
+        q = W.normal((w.Hq, w.d), seed + 2, np.float32)
+        s = W.sign_vector(w.d, w.seed + 4)
+        kc, kn = oracle.write(k, s, w.bits)
+        vc, vn = oracle.write(v, s, w.bits) if w.v_quant else (None, None)
+        ready.wait()
+        while True:
+            seconds = cmd_q.get()
+            if seconds is None:
+                return
+            t0 = time.perf_counter()
+            units = 0
+            while units == 0 or time.perf_counter() - t0 < seconds:
+                _oracle_unit(w, kc, kn, vc, vn, k, v, q, s, 0)
+                units += 1
+            res_q.put((units, time.perf_counter() - t0))
+
+
+class OracleCores:
+    """One spawned oracle process per available core (os.sched_getaffinity), each on one thread with its own unit;
+    step(seconds) runs them concurrently and returns key-heads per second of all of them together."""
+
+    def __init__(self, w):
+        import multiprocessing as mp
+        self.w = w
+        self.n = len(os.sched_getaffinity(0))
+        ctx = mp.get_context("spawn")
+        self.res_q = ctx.Queue()
+        self.cmd_q = [ctx.Queue() for _ in range(self.n)]
+        ready = ctx.Barrier(self.n + 1)
+        self.procs = [ctx.Process(target=_oracle_proc, args=(w, 900_000 + 10 * i, self.cmd_q[i], self.res_q, ready),
+                                  daemon=True) for i in range(self.n)]
+        for p_ in self.procs:
+            p_.start()
+        ready.wait(timeout=600)
+        self.units = 0
+        self.seconds = 0.0
+
+    def step(self, seconds):
+        for q_ in self.cmd_q:
+            q_.put(seconds)
+        res = [self.res_q.get(timeout=600 + 10 * seconds) for _ in range(self.n)]
+        units = sum(u for u, _ in res)
+        t = max(t_ for _, t_ in res)
+        self.units += units
+        self.seconds += t
+        return units * self.w.T * self.w.G / t
+
+    def close(self):
+        for q_ in self.cmd_q:
+            q_.put(None)
+        for p_ in self.procs:
+            p_.join(timeout=30)
+
+
+def cpu_baseline(w, seconds=10.0, all_cores=True):
+    """The fp64 oracle, as it stands, on the host cores: decode steps of single (batch row, KV head) units of the
+    workload (G query heads over T cached tokens, plus the new token's write) for about `seconds`.  First on one
+    thread; then, with all_cores, on every available core at once (OracleCores, one process and one unit per
+    core, the same time): the reported value is the all-core one, the one-thread figure rides along."""
+    import oracle
+    from threadpoolctl import threadpool_limits
     inp = W.decode_inputs(w, B=1)
     k, v, q, s = inp["k"][0], inp["v"][0], inp["q"][0], inp["signs"]
-    scale = 1.0 / math.sqrt(w.d)
-    ctx = threadpool_limits(1) if threadpool_limits else None
-    if ctx:
-        ctx.__enter__()
-    try:
-        units = 0
-        t_total = 0.0
-        hk = 0
+    with threadpool_limits(1):
+        units, t_total, hk = 0, 0.0, 0
         while t_total < seconds and hk < w.Hkv:
             kc, kn = oracle.write(k[hk], s, w.bits)  # cache state (setup, not timed)
             vc, vn = oracle.write(v[hk], s, w.bits) if w.v_quant else (None, None)
             t0 = time.perf_counter()
-            nk = oracle.write(k[hk, -1:], s, w.bits)  # the step's append of the new token
-            if w.v_quant:
-                oracle.write(v[hk, -1:], s, w.bits)
-            qq = q[hk * w.G:(hk + 1) * w.G][None]
-            kc[-1:], kn[-1:] = nk
-            if w.v_quant:
-                oracle.decode_attention(qq, kc[None, None], kn[None, None], s, w.bits, scale, vcodes=vc[None, None],
-                                        vn16=vn[None, None])
-            else:
-                oracle.decode_attention(qq, kc[None, None], kn[None, None], s, w.bits, scale, v=v[None, hk:hk + 1])
+            _oracle_unit(w, kc, kn, vc, vn, k[hk], v[hk], q, s, hk)
             t_total += time.perf_counter() - t0
             units += 1
             hk += 1
+    one = units * w.T * w.G / t_total
+    one_sample = (f"{units} of {w.B * w.Hkv} (batch row, KV head) units of {w.name}: {w.G} query heads x {w.T} "
+                  f"tokens each, plus the new token's write; fp64 numpy, 1 thread, {t_total:.1f} s")
+    out = {"value": one, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": one_sample}
+    if not all_cores:
+        return out
+    pool = OracleCores(w)
+    try:
+        many = pool.step(seconds)
     finally:
-        if ctx:
-            ctx.__exit__(None, None, None)
-    key_heads = units * w.T * w.G
-    return {"value": key_heads / t_total, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{units} of {w.B * w.Hkv} (batch row, KV head) units of {w.name}: {w.G} query heads x "
-                      f"{w.T} tokens each, plus the new token's write; fp64 numpy, 1 thread, {t_total:.1f} s"}
+        pool.close()
+    out.update({"value": many, "cores": pool.n, "single_core_value": one,
+                "sample": f"{pool.n} processes, one thread and one (batch row, KV head) unit of {w.name}'s shape "
+                          f"each ({w.G} query heads x {w.T} tokens, plus the new token's write), fp64 numpy: "
+                          f"{pool.units} unit-steps in {pool.seconds:.1f} s; single_core_value: {one_sample}"})
+    return out
 
 
 def _packed_inputs(tensors, device=None, pinned=False):
@@ -261,7 +343,7 @@ def run_axr(args, w):
     vt = vtn = None
     if w.v_quant:
         vc, vn = ops.write_keys(v, signs, bits)
-        if not args.no_variants and d == 128:  # the tiled value layout, for the variants below
+        if args.variants and d == 128:  # the tiled value layout, for the variants below
             vt, vtn = ops.write_values_tiled(v, signs, bits)
         del v
         v = None
@@ -370,8 +452,11 @@ def run_axr(args, w):
                 b2.record(stream)
             torch.cuda.synchronize()
             ms = float(np.mean([a_.elapsed_time(b2) for a_, b2 in evs]))
-            sbytes = (R + 2 + 4 * w.G) * B * Hkv * T
-            scorer[mode] = {"ms": ms, "achieved_gbs": sbytes / (ms / 1e3) / 1e9, "algorithmic_bytes": sbytes}
+            sbytes = (R + 2 + 4 * w.G) * B * Hkv * T   # codes + norms read, fp32 scores written
+            cbytes = (R + 2) * B * Hkv * T             # codes + norms only
+            scorer[mode] = {"ms": ms, "achieved_gbs": sbytes / (ms / 1e3) / 1e9, "algorithmic_bytes": sbytes,
+                            "achieved_gbs_codes_norms": cbytes / (ms / 1e3) / 1e9,
+                            "algorithmic_bytes_codes_norms": cbytes}
         ops.set_gather("mma")
         del sc_out
 
@@ -406,7 +491,7 @@ def run_axr(args, w):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "u8 codes / f32 math", "data": "synthetic",
+        "dtype": DTYPE, "data": "synthetic",
         "config": {"workload": w.name, "B": B, "T": T, "Hq": Hq, "Hkv": Hkv, "d": d, "bits": bits,
                    "values": "quantized b=%d" % bits if w.v_quant else "fp16", "parallelism": f"replicas x{ws}",
                    "l2": "flushed between steps (256 MiB write outside the per-step events)"},
@@ -414,12 +499,16 @@ def run_axr(args, w):
         "roofline": {"bound": "hbm", "kernel": "attend_rows_kernel (with the new token's write) + "
                      "attend_reduce_kernel (one axr_decode_step call)", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
                      "traffic": TRAFFIC.get(w.name) if args.batch is None else None,
                      "algorithmic_bytes": alg_bytes, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_src == "measured" else "fallback 6.65 TB/s"},
         "e2e": {"value": key_heads / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "scorer": {m: dict(v_, frac=v_["achieved_gbs"] / _peaks()[0]) for m, v_ in scorer.items()},
+        "scorer": {m: dict(v_, frac=v_["achieved_gbs"] / peak, frac_codes_norms=v_["achieved_gbs_codes_norms"] / peak,
+                           frac_of_nominal_8tbs=v_["achieved_gbs"] / NOMINAL_HBM_GBS,
+                           frac_codes_norms_of_nominal_8tbs=v_["achieved_gbs_codes_norms"] / NOMINAL_HBM_GBS)
+                   for m, v_ in scorer.items()},
         "attend_variants": {m: dict(v_, frac=v_["achieved_gbs"] / _peaks()[0]) for m, v_ in variants.items()},
         "dense_reference": dense,
         "gpu_launches": launches_per_step * args.steps,
@@ -430,21 +519,110 @@ def run_axr(args, w):
     return line
 
 
+def _fp32_alu_peak():
+    """FP32 FMA-pipe peak of one B200, from unit counts and the maximum SM clock: 148 SMs x 128 FP32 lanes x 2 flop
+    per FMA x clocks.max.sm (MEASURED_PEAKS.json sm_max_mhz, else 1965 MHz)."""
+    mhz = 1965.0
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            mhz = float(json.load(f).get("sm_max_mhz", mhz))
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def select_flops(c, n_cand):
+    """Algorithmic flops of one selection: per candidate, layer, sequence and query head, causal attention over N
+    positions is N(N+1)/2 (query, key) pairs, each a d-long dot product for the score and a d-long update of the
+    output: 2 x 2d flops per pair."""
+    return n_cand * c.layers * c.seqs * c.Hq * (c.tokens * (c.tokens + 1) // 2) * 4 * c.d
+
+
+def run_select(args):
+    """Sign selection at the calibration set's full size (36 layers x 8 sequences x 512 tokens, Hq=16, Hkv=2, d=128,
+    200 candidates): one step = one axr_select_signs call per bit width b in {2, 3, 4} (the whole-model pick),
+    timed with CUDA events on the stream; inputs resident on the device."""
+    import torch
+    from kv_cache_quantized_b200 import ops
+    c = W.QWEN3B_SELECT
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    shape_q = (c.layers, c.seqs, c.Hq, c.tokens, c.d)
+    shape_k = (c.layers, c.seqs, c.Hkv, c.tokens, c.d)
+    q = W.normal_device(shape_q, c.seed, dev, dtype=torch.float32)
+    k = W.layer_scaled_keys_device(shape_k, c.seed + 1, dev)
+    v = W.normal_device(shape_k, c.seed + 2, dev)
+    cands = torch.as_tensor(W.candidate_signs(c.n_cand, c.d, c.seed + 3), device=dev)
+    ws = torch.empty(ops.select_workspace_bytes(c.layers, c.seqs, c.tokens, c.Hq, c.Hkv, c.d, c.n_cand),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+    per_bits = {}
+    for bits in c.bits:
+        for _ in range(args.warmup):
+            ops.select_signs(q, k, v, cands, bits, workspace=ws)
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        with ClockSampler(0) as clk:
+            for a_, b_ in evs:
+                a_.record(stream)
+                mse, best = ops.select_signs(q, k, v, cands, bits, workspace=ws)
+                b_.record(stream)
+            torch.cuda.synchronize()
+        ms = [a_.elapsed_time(b_) for a_, b_ in evs]
+        per_bits[bits] = {"ms": float(np.mean(ms)), "best": int(best.item()), "clocks": clk.summary()}
+    flops = select_flops(c, c.n_cand)
+    step_ms = sum(v_["ms"] for v_ in per_bits.values())
+    peak = _fp32_alu_peak()
+    achieved = flops * len(c.bits) / (step_ms / 1e3) / 1e12
+    qpos = c.n_cand * c.layers * c.seqs * c.Hq * c.tokens * len(c.bits)
+    # the oracle on a bounded sample: 1 layer x 1 sequence x 4 candidates at the full head count and length
+    import oracle
+    from threadpoolctl import threadpool_limits
+    inp = W.calibration_inputs(c, layers=1, seqs=1, n_cand=4)
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        oracle.select_signs(inp["q"], inp["k"], inp["v"], inp["candidates"], 4)
+        t_cpu = time.perf_counter() - t0
+    cpu_qpos = 4 * c.Hq * c.tokens
+    return {
+        "metric": "sign selection at full calibration size: candidate-query evaluations/s (and FP32 TFLOP/s)",
+        "value": qpos / (step_ms / 1e3), "unit": "candidate·query/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 SIMT attention, f64 reference and accumulation", "data": "synthetic",
+        "config": {"workload": c.name, "layers": c.layers, "seqs": c.seqs, "tokens": c.tokens, "Hq": c.Hq,
+                   "Hkv": c.Hkv, "d": c.d, "bits": list(c.bits), "n_cand": c.n_cand, "causal": True,
+                   "l2": "inputs (1.4 GB) and workspace (1.8 GB) larger than L2"},
+        "per_bits": {str(b): v_ for b, v_ in per_bits.items()},
+        "roofline": {"bound": "alu", "kernel": "select_attention_kernel<128, float> (candidate attention)",
+                     "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": None, "algorithmic_flops_per_selection": flops,
+                     "peak_source": "148 SMs x 128 FP32 lanes x 2 x sm_max_mhz"},
+        "gpu_launches": len(c.bits) * args.steps * (3 + 2 * -(-c.n_cand // 8)),
+        "cpu_baseline": {"value": cpu_qpos / t_cpu, "unit": "candidate·query/s", "cores": 1, "kind": "oracle",
+                         "sample": f"1 layer x 1 sequence x 4 candidates of {c.name} at b=4 "
+                                   f"({c.Hq} heads x {c.tokens} positions), fp64 numpy, 1 thread, {t_cpu:.1f} s"},
+    }
+
+
 def run_reference(args, w):
     """The oracle as it stands on this host's cores, in place of the reference implementation (the pages ship no
-    code); one bounded sample per step."""
+    code): one OracleCores step (all cores at once, a bounded sample of the workload) per benchmark step."""
     ws, rank, _ = _dist()
     if rank != 0:
         return None
-    for _ in range(args.warmup):
-        pass
-    vals = []
-    cb = None
-    for _ in range(args.steps):
-        cb = cpu_baseline(w, seconds=args.cpu_seconds / max(args.steps, 1))
-        vals.append(cb["value"])
+    per_step = max(args.cpu_seconds / max(args.steps, 1), 0.5)
+    pool = OracleCores(w)
+    try:
+        for _ in range(args.warmup):
+            pool.step(0.2)
+        pool.units, pool.seconds = 0, 0.0
+        vals = [pool.step(per_step) for _ in range(args.steps)]
+    finally:
+        pool.close()
     value = float(np.mean(vals))
-    cb["value"] = value
+    cb = {"value": value, "unit": UNIT, "cores": pool.n, "kind": "oracle",
+          "sample": f"{pool.n} processes, one thread and one (batch row, KV head) unit of {w.name}'s shape each "
+                    f"({w.G} query heads x {w.T} tokens, plus the new token's write), fp64 numpy; {args.steps} "
+                    f"steps of {per_step:.1f} s: {pool.units} unit-steps"}
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -459,18 +637,27 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["axr", "reference"], default="axr")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="long_context")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["select"], default="long_context")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU time budget of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch size (small ncu cases)")
     ap.add_argument("--no-scorer", action="store_true", help="skip the separate axr_score measurement")
-    ap.add_argument("--no-variants", action="store_true", help="skip the tiled-value attend variants")
+    ap.add_argument("--variants", action="store_true",
+                    help="also time the attend over the tiled value layout (MMA and tcgen05 value products)")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense fp16 bandwidth reference")
     ap.add_argument("--sweep", action="store_true",
                     help="also run the decode sweep (B x T x bits x d, fp16 V) against the dense fp16 kernel")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.workload == "select":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the select workload's oracle timing rides in its "
+                              "own line's cpu_baseline"}), flush=True)
+            return
+        if _dist()[1] == 0:
+            print(json.dumps(run_select(args)), flush=True)
+        return
     w = WORKLOADS[args.workload]
     if args.batch is not None:
         import dataclasses

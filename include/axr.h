@@ -10,8 +10,9 @@
  * ---------------------------------------
  *  - Plain C types only.  fp16 tensors are passed as uint16_t* holding IEEE binary16 bit patterns.  `stream` is a
  *    cudaStream_t (NULL = the legacy default stream).  Device pointers are marked [dev], host pointers [host].
- *  - The caller owns every buffer.  The library never allocates device memory; entry points that need scratch take
- *    a caller-provided workspace whose size comes from the matching *_workspace_bytes() function.
+ *  - The caller owns every buffer.  No entry point allocates device memory per call; entry points that need scratch
+ *    take a caller-provided workspace whose size comes from the matching *_workspace_bytes() function.  The one
+ *    exception is axr_attend_decode_static, which uses a fixed 4 MiB module-scope device array instead.
  *  - Device work is asynchronous on `stream`.  Argument errors are detected on the host and returned before any
  *    launch (no device work is queued).  Launch errors come from cudaGetLastError and return AXR_ECUDA.
  *  - The decode entry points launch their split merge as a programmatic dependent of the decode kernel on the same
@@ -64,6 +65,25 @@ typedef enum axr_vkind { AXR_V_F16 = 0, AXR_V_QUANT = 1, AXR_V_QUANT_TILED = 2 }
 
 /* Thread-local message for the last non-OK status returned on this thread (empty string if none). */
 AXR_API const char* axr_last_error(void);
+
+/*
+ * Device status word.  Every spin-wait inside the library's kernels (on an mbarrier that a bulk copy completes, or on
+ * a pipeline stage being armed) gives up after a bounded number of polls, about a second, instead of hanging the
+ * GPU.  A block that gave up writes NaN into the outputs it owns and sets AXR_STATUS_WAIT_TIMEOUT in the status word
+ * of its device; the call that launched it has already returned AXR_OK.  The word is sticky (calls never clear it).
+ *
+ * axr_device_status -- synchronizes the current device (cudaDeviceSynchronize), then copies its status word to
+ * *flags [host].  clear != 0 resets the word to 0 after reading.  Returns AXR_ECUDA with a message when
+ * AXR_STATUS_WAIT_TIMEOUT is set, AXR_OK otherwise; AXR_EINVAL for a null flags pointer.  A caller that wants to
+ * tell a timed-out call from NaN inputs checks the word after the call.
+ *
+ * axr_selftest_wait_timeout -- the library's test of that give-up path: one block waits on an mbarrier that nothing
+ * arrives on (no copy pending), gives up after `polls` polls (1 .. 2^20), sets AXR_STATUS_WAIT_TIMEOUT and returns.
+ * The GPU context stays usable.  Asynchronous on `stream`.  Not part of the method.
+ */
+#define AXR_STATUS_WAIT_TIMEOUT 1u
+AXR_API axr_status axr_device_status(unsigned int* flags, int clear);
+AXR_API axr_status axr_selftest_wait_timeout(int polls, void* stream);
 
 /* ABI version: major*10000 + minor*100 + patch. */
 AXR_API int axr_version(void);
@@ -131,8 +151,12 @@ AXR_API axr_status axr_score(const float* q, const uint8_t* kcodes, const uint16
  * Table read mode of axr_score (process-wide; default AXR_GATHER_MMA, the fastest on B200).  Every mode computes the same table
  * entries LUT[j][k] = scale * q~_j * c_k (AXELRAM Key Points, 2nd item) summed at each token's indices, and they agree
  * to within the score tolerance:
- *   AXR_GATHER_TABLE     the d x 2^b table (G heads wide) is materialised in shared memory and gathered entry by
- *                        entry, one thread per token;
+ *   AXR_GATHER_TABLE     the table itself sits in shared memory, G heads wide (one 16-byte entry serves four
+ *                        heads), and each token is one thread summing one lookup per field of its code row: a
+ *                        field of W bits covers W/b coordinates, its entry the sum of their q~_j c_k -- W = 8 at
+ *                        b <= 2 (byte-indexed tables of 4 or 8 coordinates), 6 at b = 3, 8 or 4 at b = 4 (by
+ *                        G, as the tables fit); axr_attend_decode over fp16 values in this mode also reads the
+ *                        keys through it (values on the CUDA cores);
  *   AXR_GATHER_FACTORED  the table is held factored -- row factor q~_j in registers, column factor c_k gathered two
  *                        coordinates at a time from a byte-indexed pair table -- and each entry is formed by the
  *                        packed fp32 FMA that accumulates it; half the shared-memory wavefronts of TABLE;
@@ -197,6 +221,36 @@ AXR_API axr_status axr_decode_step(const float* q, const uint16_t* k_new, const 
                                    void* stream);
 
 /*
+ * Paged caches.  A serving KV cache is allocated in blocks: the pages quantize every token once on write and read it
+ * many times (AXELRAM Key Points, 2nd item), and a server hands out cache space a block at a time.  The paged entry
+ * points read (and axr_decode_step_paged writes) the same per-token rows through a block table:
+ *   block_table [dev] [B, max_blocks] int32: logical block j of batch row b (tokens [j bt, (j + 1) bt)) lives in
+ *               pool block block_table[b * max_blocks + j]; only the entries of blocks below ceil(len_b / bt) are
+ *               read, and each must be a valid block of the pools;
+ *   block_tokens bt, a power of two in [16, 2^20];
+ *   pools       codes [num_blocks, Hkv, bt, R] uint8, norms [num_blocks, Hkv, bt] fp16, values [num_blocks, Hkv, bt,
+ *               d] fp16 (AXR_V_F16) or codes + norms shaped like the keys (AXR_V_QUANT): the bt rows of one (block,
+ *               KV head) are contiguous.  Row r = (p Hkv + hk) bt + o of a pool is token o of block p for KV head
+ *               hk, so axr_write_keys with dst_rows fills a pool (prefill) the same way;
+ *   T           an upper bound of the sequence lengths, <= max_blocks * bt (it sizes the workspace and the splits);
+ *               seq_lens [B] (or NULL: every row has T tokens).
+ * Everything else (arguments, results, alignment, workspace, errors) is as in axr_attend_decode / axr_decode_step;
+ * AXR_EINVAL also for a bad block size, T above the table's reach, a null or misaligned table, or tiled values.
+ */
+AXR_API axr_status axr_attend_decode_paged(const float* q, const uint8_t* kcodes, const uint16_t* knorms,
+                                           axr_vkind vkind, const void* v, const uint16_t* vnorms,
+                                           const int32_t* block_table, int max_blocks, int block_tokens,
+                                           const int32_t* seq_lens, int B, int Hq, int Hkv, int T, int d, int bits,
+                                           const int8_t* signs, float scale, float* out, void* workspace,
+                                           size_t ws_bytes, void* stream);
+AXR_API axr_status axr_decode_step_paged(const float* q, const uint16_t* k_new, const uint16_t* v_new,
+                                         uint8_t* kcodes, uint16_t* knorms, axr_vkind vkind, void* v,
+                                         uint16_t* vnorms, const int32_t* block_table, int max_blocks,
+                                         int block_tokens, const int32_t* seq_lens, int B, int Hq, int Hkv, int T,
+                                         int d, int bits, const int8_t* signs, float scale, float* out,
+                                         void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * axr_attend_decode_static -- axr_attend_decode without a workspace argument, for callers that cannot allocate
  * device memory (code running inside a memory pool it does not own, plugins handed only input and output pointers,
  * decode steps that must not touch an allocator).  The paper has no counterpart: this is a deployment convenience.
@@ -206,7 +260,8 @@ AXR_API axr_status axr_decode_step(const float* q, const uint16_t* k_new, const 
  *   Arguments, layouts and results are those of axr_attend_decode.
  *   Sizes whose axr_attend_workspace_bytes() exceeds the fixed array return AXR_EWORKSPACE (use axr_attend_decode).
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress, with that device
- *   current); make that first call before any stream capture.
+ *   current) and keeps it; make that first call before any stream capture.  The kept address dies with the
+ *   device's context: do not call this entry point on a device after cudaDeviceReset in the same process.
  *   All calls share the one array: calls that may overlap on the GPU (different streams, or different host threads
  *   on one device) race and must be serialised by the caller.  The array keeps the last call's contents; every slot
  *   a call reads is written by that call first, so no clearing is needed.
@@ -227,6 +282,47 @@ AXR_API axr_status axr_dense_decode(const float* q, const uint16_t* k, const uin
                             int Hq, int Hkv, int T, int Tcap, int d, float scale, float* out, void* workspace,
                             size_t ws_bytes, void* stream);
 
+/*
+ * LOOKAT product quantization (the newx.sg summary and abstract of "LOOKAT: Lookup-Optimized Key-Attention for
+ * Memory-Efficient Transformers"): keys are cut into m subspaces of d/m coordinates (subspace i = coordinates
+ * [i d/m, (i+1) d/m)), each with a codebook of K <= 256 centroids learned by k-means; a key is stored as m one-byte
+ * indices; a query scores it through a per-query table T[i][k] = q^(i) . C_i[k] (asymmetric distance computation:
+ * the query is exact, no key is reconstructed).  The pages print no formulas; these are the textbook definitions.
+ * Supported: d in {64, 128}, m in {2, 4, 8, 16}, 1 <= K <= 256, G in {1, 2, 4, 8}.
+ *
+ * axr_pq_train -- Lloyd's k-means of one head's keys, per subspace, from the initial centroids in codebooks:
+ *   each of `iters` iterations assigns every subvector to its nearest centroid (the rule of axr_pq_encode) and
+ *   moves every centroid with members to their mean (fp64 sums, rounded to fp32); a centroid without members
+ *   stays.  x [dev] [n_vec, d] (AXR_F16 or AXR_F32); codebooks [dev] in/out [m, K, d/m] f32;
+ *   workspace [dev] >= axr_pq_train_workspace_bytes(d, m, K), 16-aligned.
+ * axr_pq_encode -- the nearest centroid of every subvector: squared Euclidean distance formed in fp32 as
+ *   sum_j (x_j - c_j)^2 in increasing j, each operation rounded (no fused multiply-add), lowest index on a tie.
+ *   x [dev] [n_vec, d]; codebooks [dev] [heads, m, K, d/m] f32, vector r using set (r / head_period) % heads
+ *   (a [B, Hkv, Tcap, d] cache: heads = Hkv, head_period = Tcap; new tokens [B, Hkv, d]: head_period = 1);
+ *   dst_rows [dev] [n_vec] int64 destination rows, or NULL for row r; codes [dev] out [rows, m] uint8.
+ * axr_pq_score -- scores[b, h, t] = scale * sum_i T[i][codes[b, hk, t, i]] for t < len_b, -inf for len_b <= t < T;
+ *   q [dev] [B, Hq, d] f32; codes [dev] [B, Hkv, Tcap, m]; codebooks [dev] [Hkv, m, K, d/m] f32 (one set per KV
+ *   head); the table is built in shared memory per (batch row, KV head), G heads wide.
+ * axr_pq_attend_decode -- decode attention with those scores (times `scale`) over fp16 values [dev]
+ *   [B, Hkv, Tcap, d]: online softmax per split of the token axis, the value product, the split merge;
+ *   workspace as axr_attend_decode (axr_attend_workspace_bytes).
+ * Errors: AXR_EINVAL (pointers, sizes, alignment: q/v/out 16 bytes, codes 4 (m >= 4) or 2, codebooks 4),
+ * AXR_EUNSUPPORTED (d, m, K, G, subspace width), AXR_EWORKSPACE, AXR_ECUDA.  n_vec == 0 / B == 0 are no-ops.
+ */
+AXR_API size_t axr_pq_train_workspace_bytes(int d, int m, int K);
+AXR_API axr_status axr_pq_train(const void* x, axr_dtype x_dtype, int64_t n_vec, int d, int m, int K, int iters,
+                                float* codebooks, void* workspace, size_t ws_bytes, void* stream);
+AXR_API axr_status axr_pq_encode(const void* x, axr_dtype x_dtype, int64_t n_vec, int d, int m, int K,
+                                 const float* codebooks, int heads, int head_period, const int64_t* dst_rows,
+                                 uint8_t* codes, void* stream);
+AXR_API axr_status axr_pq_score(const float* q, const uint8_t* codes, const float* codebooks, const int32_t* seq_lens,
+                                int B, int Hq, int Hkv, int T, int Tcap, int d, int m, int K, float scale,
+                                float* scores, void* stream);
+AXR_API axr_status axr_pq_attend_decode(const float* q, const uint8_t* codes, const float* codebooks,
+                                        const uint16_t* v, const int32_t* seq_lens, int B, int Hq, int Hkv, int T,
+                                        int Tcap, int d, int m, int K, float scale, float* out, void* workspace,
+                                        size_t ws_bytes, void* stream);
+
 /* Bytes of workspace for axr_select_signs with these sizes. */
 AXR_API size_t axr_select_workspace_bytes(int n_layers, int n_seq, int n_tok, int Hq, int Hkv, int d, int n_cand);
 
@@ -246,6 +342,25 @@ AXR_API size_t axr_select_workspace_bytes(int n_layers, int n_seq, int n_tok, in
 AXR_API axr_status axr_select_signs(const float* q, const uint16_t* k, const uint16_t* v, int n_layers, int n_seq, int n_tok,
                             int Hq, int Hkv, int d, int bits, const int8_t* candidates, int n_cand, int causal,
                             double* mse_out, int32_t* best_out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * axr_select_signs_per_layer -- the same one-time selection with one sign vector per layer.  The pages trace the
+ * sign sensitivity to layer-wise norm heterogeneity (AXELRAM Abstract; Key Points, 3rd and 4th items): a pattern
+ * that suits the high-norm layers need not suit the others, and the write path takes its sign vector per call,
+ * so a model may hold one per layer.  Objective of candidate c for layer l: the mean over every (sequence, query
+ * head, position, coordinate) of layer l of (o_quant - o_ref)^2, with o_quant, o_ref and the causal rule as in
+ * axr_select_signs.  The mean over layers of mse_layers_out[:, c] equals axr_select_signs' mse_out[c].
+ *   inputs and workspace as axr_select_signs (the same axr_select_workspace_bytes);
+ *   mse_layers_out [dev] out [n_layers, n_cand] f64;
+ *   best_layers_out [dev] out [n_layers] int32: per layer the first index of the minimum of its row;
+ *   mse_parts_out [dev] out [n_layers, n_seq, n_cand] f64, the MSE of each (layer, calibration sequence), or NULL.
+ * Errors: as axr_select_signs.
+ */
+AXR_API axr_status axr_select_signs_per_layer(const float* q, const uint16_t* k, const uint16_t* v, int n_layers,
+                                              int n_seq, int n_tok, int Hq, int Hkv, int d, int bits,
+                                              const int8_t* candidates, int n_cand, int causal,
+                                              double* mse_layers_out, int32_t* best_layers_out,
+                                              double* mse_parts_out, void* workspace, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

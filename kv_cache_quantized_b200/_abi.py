@@ -16,6 +16,7 @@ STATUS = {0: "AXR_OK", 1: "AXR_EINVAL", 2: "AXR_EUNSUPPORTED", 3: "AXR_ECUDA", 4
 F32, F16 = 0, 1
 V_F16, V_QUANT, V_QUANT_TILED = 0, 1, 2
 GATHER_FACTORED, GATHER_TABLE, GATHER_TENSOR, GATHER_MMA = 0, 1, 2, 3
+STATUS_WAIT_TIMEOUT = 1
 
 _p = ctypes.c_void_p
 _i = ctypes.c_int
@@ -33,12 +34,25 @@ SIGNATURES = {
     "axr_attend_workspace_bytes": (_sz, [_i, _i, _i, _i, _i]),
     "axr_attend_decode": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p, _sz, _p]),
     "axr_decode_step": (_i, [_p, _p, _p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p, _sz, _p]),
+    "axr_attend_decode_paged": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _p, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p,
+                                     _sz, _p]),
+    "axr_decode_step_paged": (_i, [_p, _p, _p, _p, _p, _i, _p, _p, _p, _i, _i, _p, _i, _i, _i, _i, _i, _i, _p, _f, _p,
+                                   _p, _sz, _p]),
     "axr_dense_decode": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
     "axr_select_workspace_bytes": (_sz, [_i, _i, _i, _i, _i, _i, _i]),
     "axr_select_signs": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _p, _p, _p, _sz, _p]),
+    "axr_select_signs_per_layer": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _i, _i, _p, _p, _p, _p, _sz,
+                                        _p]),
     "axr_attend_decode_static": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _p, _f, _p, _p]),
     "axr_attend_static_scratch_bytes": (_sz, []),
+    "axr_pq_train_workspace_bytes": (_sz, [_i, _i, _i]),
+    "axr_pq_train": (_i, [_p, _i, _i64, _i, _i, _i, _i, _p, _p, _sz, _p]),
+    "axr_pq_encode": (_i, [_p, _i, _i64, _i, _i, _i, _p, _i, _i, _p, _p, _p]),
+    "axr_pq_score": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p]),
+    "axr_pq_attend_decode": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
     "axr_set_gather": (_i, [_i]),
+    "axr_device_status": (_i, [_p, _i]),
+    "axr_selftest_wait_timeout": (_i, [_i, _p]),
     "axr_get_gather": (_i, []),
 }
 

@@ -426,6 +426,8 @@ attend_fused_kernel(const __grid_constant__ DecodeArgs a) {
     }
     done += ntiles;
   }
+  __syncthreads();
+  report_wait_failure(a, failed);
 }
 
 }  // namespace axr

@@ -140,7 +140,7 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
     const int start = split * a.chunk;
     const int end = min(start + a.chunk, len);
     const int ntiles = end > start ? (end - start + TT - 1) / TT : 0;
-    const size_t kv_row0 = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
+    const RowMap rm = row_map(a, b, hk);  // cache row of each token (contiguous or through the block table)
     const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
 
     fence_proxy_async();  // the merge region's generic writes come before the bulk copies that reuse it
@@ -149,7 +149,7 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
       // decode step: this item holds the new token (position len - 1): warp 0 writes its key and warp 1 its value
       // through the write path, before any of the item's tiles is copied
       if (warp < 2) {
-        append_row<D, BITS, VQ>(a, b, hk, kv_row0 + (len - 1), warp, lane,
+        append_row<D, BITS, VQ>(a, b, hk, rm(len - 1), warp, lane,
                                 reinterpret_cast<uint8_t*>(smem + P::OFF_P) + warp * D);
         __threadfence();  // the stores reach the device-wide view ...
         asm volatile("fence.proxy.async.global;\n" ::: "memory");  // ... and the async proxy of the bulk copies
@@ -176,18 +176,18 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
       // norms: staged with the codes when both norm rows start 16-byte aligned (cp.async), else raw fp16 values of
       // token `lane` of the warp's share of a tile (key norm | value norm << 16) loaded one tile ahead into registers
       // and converted only when used
-      const __half* kn_src = a.knorms + kv_row0;
-      const __half* vn_src = VQ ? a.vnorms + kv_row0 : nullptr;
-      const bool nrm_async = (reinterpret_cast<uintptr_t>(kn_src + start) & 15) == 0 &&
-                             (!VQ || (reinterpret_cast<uintptr_t>(vn_src + start) & 15) == 0);
+      // (a paged pool's blocks hold >= 16 tokens, so its norm chunks are aligned whenever the pool's base is)
+      const bool nrm_async = (reinterpret_cast<uintptr_t>(a.knorms + rm(start)) & 15) == 0 &&
+                             (!VQ || (reinterpret_cast<uintptr_t>(a.vnorms + rm(start)) & 15) == 0);
       __half* nst = reinterpret_cast<__half*>(smem + P::OFF_N);
       auto load_norms = [&](int tile) -> uint32_t {
         const int t = start + tile * TT + warp * WT + lane;
         uint32_t r = 0x3c00u << 16;  // value norm 1 for fp16 values
         if (!nrm_async && tile < ntiles && t < end) {
           // loads cached in L2 only: a decode step writes the new token's norms in this launch
-          r = __half_as_ushort(__ldcg(kn_src + t));
-          if constexpr (VQ) r |= static_cast<uint32_t>(__half_as_ushort(__ldcg(vn_src + t))) << 16;
+          const size_t row = rm(t);
+          r = __half_as_ushort(__ldcg(a.knorms + row));
+          if constexpr (VQ) r |= static_cast<uint32_t>(__half_as_ushort(__ldcg(a.vnorms + row))) << 16;
           else r |= 0x3c00u << 16;
         }
         return r;
@@ -199,19 +199,18 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
           const int n = min(TT, end - t0);
           const int bytes = n * R;
           uint8_t* dst = smem + P::OFF_K + kstg(tile) * P::STAGE_K;
-          const uint8_t* src = a.kcodes + (kv_row0 + t0) * R;
           if constexpr (P::BULK) {
             if (rtid == 0) {
               mbar_arrive_expect_tx(kfull + kstg(tile), bytes);
-              bulk_copy_g2s(dst, src, bytes, kfull + kstg(tile));
+              copy_rows_bulk<R>(dst, a.kcodes, rm, t0, n, kfull + kstg(tile));
             }
           } else {
-            for (int o = rtid * P::KCH; o < bytes; o += 128 * P::KCH) cp_async<P::KCH>(dst + o, src + o);
+            copy_rows_async<P::KCH, R>(dst, a.kcodes, rm, t0, n, rtid);
           }
           if (nrm_async) {
             __half* nd = nst + kstg(tile) * 2 * TT;
-            if (rtid < 16) stage_norms(nd, kn_src + t0, n, rtid);
-            else if (VQ && rtid < 32) stage_norms(nd + TT, vn_src + t0, n, rtid - 16);
+            if (rtid < 16) stage_norms_map(nd, a.knorms, rm, t0, n, rtid);
+            else if (VQ && rtid < 32) stage_norms_map(nd + TT, a.vnorms, rm, t0, n, rtid - 16);
           }
         }
         cp_async_commit();
@@ -334,16 +333,15 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
       auto issue_v = [&](int tile) {
         if (tile < ntiles) {
           const int t0 = start + tile * TT;
-          const int bytes = min(TT, end - t0) * R;
+          const int n = min(TT, end - t0);
           uint8_t* dst = smem + P::OFF_V + vstg(tile) * P::STAGE_V;
-          const uint8_t* src = vsrc + (kv_row0 + t0) * R;
           if constexpr (P::BULK) {
             if (rtid == 0) {
-              mbar_arrive_expect_tx(vfull + vstg(tile), bytes);
-              bulk_copy_g2s(dst, src, bytes, vfull + vstg(tile));
+              mbar_arrive_expect_tx(vfull + vstg(tile), n * R);
+              copy_rows_bulk<R>(dst, vsrc, rm, t0, n, vfull + vstg(tile));
             }
           } else {
-            for (int o = rtid * P::KCH; o < bytes; o += 128 * P::KCH) cp_async<P::KCH>(dst + o, src + o);
+            copy_rows_async<P::KCH, R>(dst, vsrc, rm, t0, n, rtid);
           }
         }
         cp_async_commit();
@@ -437,16 +435,15 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
       auto issue_v = [&](int tile) {
         if (tile < ntiles) {
           const int t0 = start + tile * TT;
+          const int n = min(TT, end - t0);
           uint8_t* dst = smem + P::OFF_V + vstg(tile) * P::STAGE_V;
-          const uint8_t* src = vsrc + (kv_row0 + t0) * P::VROW;
-          const int bytes = min(TT, end - t0) * P::VROW;
           if constexpr (P::BULK) {
             if (rtid == 0) {
-              mbar_arrive_expect_tx(vfull + vstg(tile), bytes);
-              bulk_copy_g2s(dst, src, bytes, vfull + vstg(tile));
+              mbar_arrive_expect_tx(vfull + vstg(tile), n * P::VROW);
+              copy_rows_bulk<P::VROW>(dst, vsrc, rm, t0, n, vfull + vstg(tile));
             }
           } else {
-            role_copy_async<P::VCH>(dst, src, bytes, rtid);
+            copy_rows_async<P::VCH, P::VROW>(dst, vsrc, rm, t0, n, rtid);
           }
         }
         cp_async_commit();
@@ -534,6 +531,8 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
     }
     done += ntiles;
   }
+  __syncthreads();
+  report_wait_failure(a, failed);
 }
 
 }  // namespace axr

@@ -20,7 +20,9 @@ std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {nullptr};
 
 // Device address of the array on the current device.  In host code `g_attend_scratch` names a host-side stand-in,
-// not device memory, so the address has to be looked up once per device with that device current.
+// not device memory, so the address has to be looked up once per device with that device current.  The cached
+// address belongs to the device's current context: after a cudaDeviceReset in the same process it is stale, and
+// this entry point must not be called on that device again.
 axr_status scratch_for_current_device(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);

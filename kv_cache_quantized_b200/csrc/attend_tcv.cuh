@@ -537,6 +537,7 @@ attend_tcv_kernel(const __grid_constant__ DecodeArgs a) {
 
   tc::fence_before();
   __syncthreads();
+  report_wait_failure(a, failed);
   if (*failed) {  // make this CTA's partials NaN so that the merged output shows the failure
     for (int item = blockIdx.x; item < items; item += gridDim.x) {
       const ItemGeo g = item_geo(a, item);

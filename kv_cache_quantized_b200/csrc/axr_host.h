@@ -21,6 +21,9 @@ inline axr_status check_launch(const char* what) {
 
 inline bool supported_g(int G) { return G == 1 || G == 2 || G == 4 || G == 8; }
 
+// Device address of the current device's status word (status.cu), or null if it could not be looked up.
+unsigned int* status_word();
+
 // Split of the token axis for the decode kernels: the number of token chunks per (batch, KV head) and the chunk
 // length.  Depends only on the sizes, so a workspace sized by axr_attend_workspace_bytes always fits.
 struct SplitPlan {

@@ -26,6 +26,7 @@ DecodeArgs base_args(int B, int Hq, int Hkv, int T, int Tcap, const int32_t* seq
   memset(&a, 0, sizeof(a));
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.T = T; a.Tcap = Tcap;
   a.seq_lens = seq_lens; a.q = q; a.mult = mult;
+  a.status = status_word();
   const SplitPlan p = plan_splits(B, Hkv, T);
   a.splits = p.splits; a.chunk = p.chunk;
   return a;
@@ -55,6 +56,7 @@ extern "C" axr_status axr_score(const float* q, const uint8_t* kcodes, const uin
   const int G = Hq / Hkv;
   const int mode = g_gather.load();
   if (mode == kGatherTensor) return score_tc_launch(d, bits, G, a, as_stream(stream));
+  if (mode == kGatherTable) return table_score_launch(d, bits, G, a, as_stream(stream));
   return score_launch(d, bits, G, mode, a, as_stream(stream));
 }
 
@@ -82,9 +84,23 @@ namespace {
 axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, const uint16_t* knorms,
                        axr_vkind vkind, const void* v, const uint16_t* vnorms, const int32_t* seq_lens, int B, int Hq,
                        int Hkv, int T, int Tcap, int d, int bits, const int8_t* signs, float scale, float* out,
-                       void* workspace, size_t ws_bytes, void* stream, const uint16_t* knew, const uint16_t* vnew) {
+                       void* workspace, size_t ws_bytes, void* stream, const uint16_t* knew, const uint16_t* vnew,
+                       const int32_t* block_table = nullptr, int max_blocks = 0, int block_tokens = 0) {
   using namespace axr;
   const bool step = knew != nullptr || vnew != nullptr;
+  const bool paged = block_table != nullptr;
+  int shift = 0;
+  if (paged) {
+    while (shift < 31 && (1 << shift) < block_tokens) ++shift;
+    if (block_tokens < 16 || block_tokens > (1 << 20) || (1 << shift) != block_tokens)
+      return set_error(AXR_EINVAL, "%s: block_tokens=%d is not a power of two in [16, 2^20]", w, block_tokens);
+    if (max_blocks <= 0 || static_cast<long>(T) > static_cast<long>(max_blocks) * block_tokens)
+      return set_error(AXR_EINVAL, "%s: T=%d exceeds max_blocks=%d x block_tokens=%d", w, T, max_blocks,
+                       block_tokens);
+    if (!aligned(block_table, 4)) return set_error(AXR_EINVAL, "%s: misaligned block table", w);
+    if (vkind == AXR_V_QUANT_TILED) return set_error(AXR_EINVAL, "%s: paged pools take the row value layouts", w);
+    Tcap = T;  // no capacity stride: rows come through the block table
+  }
   axr_status st = check_decode_sizes(w, B, Hq, Hkv, T, Tcap, d);
   if (st != AXR_OK) return st;
   if (bits < 1 || bits > 4) return set_error(AXR_EUNSUPPORTED, "%s: bits=%d outside 1..4", w, bits);
@@ -119,10 +135,16 @@ axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, con
   const int G = Hq / Hkv;
   const int mode = g_gather.load();
   const bool vq = vkind == AXR_V_QUANT;
-  // decode step: the kernel whose prologue writes the new token (scores through warp-level MMAs)
-  if (step) return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));
+  if (paged) {
+    a.block_table = block_table; a.max_blocks = max_blocks; a.block_shift = shift;
+  }
+  // decode step and paged pools: the kernel that writes the new token in its prologue and reads rows through the
+  // block table (scores through warp-level MMAs)
+  if (step || paged) return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));
   // tiled values: the tcgen05 kernel in AXR_GATHER_TENSOR mode, else warp-level MMAs for keys and values
   if (vkind == AXR_V_QUANT_TILED) return attend_tiled_launch(bits, G, mode == kGatherTensor, a, as_stream(stream));
+  // fp16 values in AXR_GATHER_TABLE mode: the literal table in shared memory, values on the CUDA cores
+  if (mode == kGatherTable && !vq) return table_attend_launch(d, bits, G, a, as_stream(stream));
   // row-layout values: keys scored through warp-level MMAs in AXR_GATHER_MMA mode, else on CUDA cores
   if (mode == kGatherMma) {
     // fp16 values: one warp per token range through scores, softmax and the value product (no block barrier);
@@ -151,6 +173,31 @@ extern "C" axr_status axr_decode_step(const float* q, const uint16_t* k_new, con
   if (!k_new || !v_new) return axr::set_error(AXR_EINVAL, "axr_decode_step: null pointer");
   return attend_impl("axr_decode_step", q, kcodes, knorms, vkind, v, vnorms, seq_lens, B, Hq, Hkv, T, Tcap, d, bits,
                      signs, scale, out, workspace, ws_bytes, stream, k_new, v_new);
+}
+
+extern "C" axr_status axr_attend_decode_paged(const float* q, const uint8_t* kcodes, const uint16_t* knorms,
+                                              axr_vkind vkind, const void* v, const uint16_t* vnorms,
+                                              const int32_t* block_table, int max_blocks, int block_tokens,
+                                              const int32_t* seq_lens, int B, int Hq, int Hkv, int T, int d,
+                                              int bits, const int8_t* signs, float scale, float* out,
+                                              void* workspace, size_t ws_bytes, void* stream) {
+  if (!block_table) return axr::set_error(AXR_EINVAL, "axr_attend_decode_paged: null block table");
+  return attend_impl("axr_attend_decode_paged", q, kcodes, knorms, vkind, v, vnorms, seq_lens, B, Hq, Hkv, T, T, d,
+                     bits, signs, scale, out, workspace, ws_bytes, stream, nullptr, nullptr, block_table, max_blocks,
+                     block_tokens);
+}
+
+extern "C" axr_status axr_decode_step_paged(const float* q, const uint16_t* k_new, const uint16_t* v_new,
+                                            uint8_t* kcodes, uint16_t* knorms, axr_vkind vkind, void* v,
+                                            uint16_t* vnorms, const int32_t* block_table, int max_blocks,
+                                            int block_tokens, const int32_t* seq_lens, int B, int Hq, int Hkv, int T,
+                                            int d, int bits, const int8_t* signs, float scale, float* out,
+                                            void* workspace, size_t ws_bytes, void* stream) {
+  if (!k_new || !v_new) return axr::set_error(AXR_EINVAL, "axr_decode_step_paged: null pointer");
+  if (!block_table) return axr::set_error(AXR_EINVAL, "axr_decode_step_paged: null block table");
+  return attend_impl("axr_decode_step_paged", q, kcodes, knorms, vkind, v, vnorms, seq_lens, B, Hq, Hkv, T, T, d,
+                     bits, signs, scale, out, workspace, ws_bytes, stream, k_new, v_new, block_table, max_blocks,
+                     block_tokens);
 }
 
 extern "C" axr_status axr_dense_decode(const float* q, const uint16_t* k, const uint16_t* v,

@@ -48,7 +48,52 @@ struct DecodeArgs {
   int splits, chunk;
   float mult;                // factor folded into the table (score: scale; attend: scale * log2(e))
   Codebook cb;
+  unsigned int* status;      // the device's status word (axr_device_status), or null
+  const int32_t* block_table;  // paged caches: [B, max_blocks] pool block of each logical block; null: contiguous
+  int max_blocks;            // paged: entries per block-table row
+  int block_shift;           // paged: log2 of the tokens per block
 };
+
+// Cache row of token t of one (batch row, KV head).  Contiguous caches [B, Hkv, Tcap] number the rows
+// (b Hkv + hk) Tcap + t; paged pools [num_blocks, Hkv, bt] number them (block_table[b][t / bt] Hkv + hk) bt + t % bt,
+// so the bt tokens of one (block, KV head) are contiguous.
+struct RowMap {
+  const int32_t* table;  // the batch row's block table, or null (contiguous)
+  size_t base;           // contiguous: (b Hkv + hk) Tcap; paged: hk bt
+  size_t stride;         // paged: Hkv bt, the rows of one block
+  int shift;             // paged: log2 bt
+  __device__ __forceinline__ size_t operator()(int t) const {
+    if (!table) return base + static_cast<size_t>(t);
+    return static_cast<size_t>(__ldg(table + (t >> shift))) * stride + base +
+           static_cast<size_t>(t & ((1 << shift) - 1));
+  }
+  // rows from t to the end of t's block (contiguous caches: unbounded)
+  __device__ __forceinline__ int run(int t) const {
+    return table ? (1 << shift) - (t & ((1 << shift) - 1)) : (1 << 30);
+  }
+};
+
+__device__ __forceinline__ RowMap row_map(const DecodeArgs& a, int b, int hk) {
+  RowMap m;
+  if (a.block_table) {
+    m.table = a.block_table + static_cast<size_t>(b) * a.max_blocks;
+    m.shift = a.block_shift;
+    m.base = static_cast<size_t>(hk) << a.block_shift;
+    m.stride = static_cast<size_t>(a.Hkv) << a.block_shift;
+  } else {
+    m.table = nullptr;
+    m.shift = 0;
+    m.base = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
+    m.stride = 0;
+  }
+  return m;
+}
+
+// A block whose bounded wait gave up (its `failed` flag set) records it in the device's status word, beside the
+// NaN it writes into its outputs.  Called by every thread at the kernel's end; thread 0 reports.
+__device__ __forceinline__ void report_wait_failure(const DecodeArgs& a, volatile int* failed) {
+  if (threadIdx.x == 0 && *failed && a.status) atomicOr(a.status, 1u);
+}
 
 __device__ __forceinline__ int row_len(const DecodeArgs& a, int b) {
   if (!a.seq_lens) return a.T;
@@ -81,6 +126,13 @@ __device__ __forceinline__ void stage_norms(__half* dst, const __half* src, int 
   if (c < 16 && tok0 < n) cp_async16_zfill(dst + tok0, src + tok0, min(16, 2 * (n - tok0)));
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
+// stage_norms for rows [t0, t0 + n) of one (batch row, KV head) through its row map (blocks hold >= 8 tokens, so an
+// 8-token chunk never straddles two)
+__device__ __forceinline__ void stage_norms_map(__half* dst, const __half* norms, const RowMap& rm, int t0, int n,
+                                                int c) {
+  const int tok0 = 8 * c;
+  if (c < 16 && tok0 < n) cp_async16_zfill(dst + tok0, norms + rm(t0 + tok0), min(16, 2 * (n - tok0)));
+}
 
 // Bulk (TMA engine) copy of `bytes` (a multiple of 16; both addresses 16-byte aligned) from global to this CTA's
 // shared memory, completing on `mbar` as transaction bytes; the caller has armed the barrier with expect_tx.
@@ -95,6 +147,32 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(mbar)), "r"(bytes)
                : "memory");
+}
+
+// Bulk copies of the rows [t0, t0 + n) of one (batch row, KV head), RB bytes each (a multiple of 16), into dst: one
+// copy per run of rows contiguous in global memory (one for a contiguous cache, one per block for a paged pool),
+// all completing on `mbar`, which the caller has armed with the total.
+template <int RB>
+__device__ __forceinline__ void copy_rows_bulk(uint8_t* dst, const uint8_t* src, const RowMap& rm, int t0, int n,
+                                               uint64_t* mbar) {
+  for (int o = 0; o < n;) {
+    const int seg = min(n - o, rm.run(t0 + o));
+    bulk_copy_g2s(dst + static_cast<size_t>(o) * RB, src + rm(t0 + o) * RB, static_cast<uint32_t>(seg * RB), mbar);
+    o += seg;
+  }
+}
+
+// The same rows as CH-byte cp.async chunks spread over a role's 128 threads (RB a multiple of CH).
+template <int CH, int RB>
+__device__ __forceinline__ void copy_rows_async(uint8_t* dst, const uint8_t* src, const RowMap& rm, int t0, int n,
+                                                int rtid) {
+  const int bytes = n * RB;
+  if (!rm.table) {
+    const uint8_t* s = src + rm(t0) * RB;
+    for (int o = rtid * CH; o < bytes; o += 128 * CH) cp_async<CH>(dst + o, s + o);
+  } else {
+    for (int o = rtid * CH; o < bytes; o += 128 * CH) cp_async<CH>(dst + o, src + rm(t0 + o / RB) * RB + o % RB);
+  }
 }
 
 // Order this thread's generic-proxy accesses to shared memory before later async-proxy (bulk copy) accesses.

@@ -55,6 +55,11 @@ axr_status attend_tiled_launch(int bits, int G, bool tensor, const DecodeArgs& a
 // Scores only (score.cu): mode is one of kGatherTable, kGatherFactored, kGatherMma.
 axr_status score_launch(int d, int bits, int G, int mode, const DecodeArgs& a, cudaStream_t st);
 
+// The literal table in shared memory (lut.cu): multi-coordinate fields, G-wide entries; scores, and attend over
+// fp16 values.
+axr_status table_score_launch(int d, int bits, int G, const DecodeArgs& a, cudaStream_t st);
+axr_status table_attend_launch(int d, int bits, int G, const DecodeArgs& a, cudaStream_t st);
+
 // Scores only on the tcgen05 tensor cores (score_tc.cu).
 axr_status score_tc_launch(int d, int bits, int G, const DecodeArgs& a, cudaStream_t st);
 

@@ -217,6 +217,8 @@ __global__ void __launch_bounds__(256, 2) score_mma_kernel(const __grid_constant
     done += x.ntiles;
   }
   cp_async_wait<0>();
+  __syncthreads();
+  report_wait_failure(a, failed);
 }
 
 }  // namespace axr

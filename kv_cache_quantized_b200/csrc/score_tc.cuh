@@ -349,6 +349,7 @@ score_tc_kernel(const __grid_constant__ DecodeArgs a) {
 
   tc::fence_before();
   __syncthreads();
+  report_wait_failure(a, failed);
   if (*failed) {  // the scores of this CTA's tiles are not valid
     TileCursor cur;
     cursor_init(a, g0, cur);

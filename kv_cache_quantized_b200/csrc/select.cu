@@ -8,8 +8,10 @@
 //      sign flip, Walsh-Hadamard, threshold count, fp16 norm) and is reconstructed in the original domain,
 //      k^ = s .* H(n16 * c[idx]) -- for a prefill-shaped calibration set this is the cheap direction (one transform
 //      per key instead of one per query), and q . k^ equals the table score exactly up to rounding;
-//   3. fp32 tiled attention with k^, squared error against o_ref accumulated per candidate in fp64;
-//   4. mse = sum / count, best = first index of the minimum.
+//   3. fp32 tiled attention with k^, squared error against o_ref accumulated in fp64 per (candidate, layer,
+//      sequence);
+//   4. mse = sum / count, best = first index of the minimum: over every layer (one sign vector for the model), or
+//      per layer (one sign vector per layer, axr_select_signs_per_layer).
 #include <cmath>
 
 #include "axr_host.h"
@@ -27,11 +29,13 @@ struct SelArgs {
   const int8_t* cand;   // [C, D]
   double* oref;         // [Ly, S, Hq, N, D]
   float* khat;          // [chunk, Ly, S, Hkv, N, D]
-  double* acc;          // [C]
-  double* mse;          // [C]
-  int32_t* best;
+  double* acc;          // [C, Ly, S] squared-error sums
+  double* mse;          // [C], or [Ly, C] per layer
+  int32_t* best;        // [1], or [Ly] per layer
+  double* parts;        // [Ly, S, C] per-(layer, sequence) MSEs, or null
   int Ly, S, Hq, Hkv, N, C;
   int c0, nc;           // candidate chunk [c0, c0 + nc)
+  int D_;               // head dim (for the finalize kernel)
   int causal;
   Codebook cb;
 };
@@ -245,21 +249,40 @@ __global__ void __launch_bounds__(kSelThreads) select_attention_kernel(const __g
     if (tid == 0) {
       double t = 0.0;
       for (int w = 0; w < kSelThreads / kWarp; ++w) t += werr[w];
-      atomicAdd(a.acc + a.c0 + ci, t);
+      atomicAdd(a.acc + static_cast<size_t>(a.c0 + ci) * a.Ly * a.S + ls, t);
     }
   }
 }
 
-__global__ void select_finalize_kernel(const __grid_constant__ SelArgs a, double count) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  int best = 0;
-  double bv = INFINITY;
-  for (int c = 0; c < a.C; ++c) {
-    const double m = a.acc[c] / count;
-    a.mse[c] = m;
-    if (m < bv) { bv = m; best = c; }
+// MSEs from the per-(candidate, layer, sequence) sums (each over Hq * N * D elements), summed in a fixed order.
+// per_layer: mse [Ly, C] and best [Ly] (one pick per layer); else mse [C] over every layer and best [1].
+__global__ void select_finalize_kernel(const __grid_constant__ SelArgs a, int per_layer) {
+  const double per_part = static_cast<double>(a.Hq) * a.N * a.D_;
+  const int groups = per_layer ? a.Ly : 1;
+  const int lpg = per_layer ? 1 : a.Ly;  // layers per group
+  for (int i = threadIdx.x; i < groups * a.C; i += blockDim.x) {
+    const int g = i / a.C, c = i % a.C;
+    const double* acc = a.acc + static_cast<size_t>(c) * a.Ly * a.S;
+    double t = 0.0;
+    for (int l = g * lpg; l < (g + 1) * lpg; ++l)
+      for (int sq = 0; sq < a.S; ++sq) t += acc[l * a.S + sq];
+    a.mse[i] = t / (per_part * lpg * a.S);
   }
-  *a.best = best;
+  if (a.parts)
+    for (int i = threadIdx.x; i < a.Ly * a.S * a.C; i += blockDim.x) {
+      const int c = i % a.C, ls = i / a.C;
+      a.parts[i] = a.acc[static_cast<size_t>(c) * a.Ly * a.S + ls] / per_part;
+    }
+  __syncthreads();
+  for (int g = threadIdx.x; g < groups; g += blockDim.x) {
+    int best = 0;
+    double bv = INFINITY;
+    for (int c = 0; c < a.C; ++c) {
+      const double m = a.mse[g * a.C + c];
+      if (m < bv) { bv = m; best = c; }
+    }
+    a.best[g] = best;
+  }
 }
 
 struct SelLayout {
@@ -275,12 +298,12 @@ SelLayout sel_layout(int Ly, int S, int N, int Hq, int Hkv, int d, int C) {
   L.oref = 0;
   L.khat = up(qn * sizeof(double));
   L.acc = L.khat + up(kn * chunk * sizeof(float));
-  L.total = L.acc + up(static_cast<size_t>(C) * sizeof(double));
+  L.total = L.acc + up(static_cast<size_t>(C) * Ly * S * sizeof(double));
   return L;
 }
 
 template <int D, int BITS>
-axr_status run_select(SelArgs a, cudaStream_t st) {
+axr_status run_select(SelArgs a, int per_layer, cudaStream_t st) {
   using RC = AttnCfg<D, double, true>;
   using FC = AttnCfg<D, float, false>;
   auto kref = select_attention_kernel<D, double, true>;
@@ -288,7 +311,7 @@ axr_status run_select(SelArgs a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kref, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RC::smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FC::smem);
   if (e != cudaSuccess) return set_error(AXR_ECUDA, "axr_select_signs: %s", cudaGetErrorString(e));
-  e = cudaMemsetAsync(a.acc, 0, sizeof(double) * a.C, st);
+  e = cudaMemsetAsync(a.acc, 0, sizeof(double) * a.C * a.Ly * a.S, st);
   if (e != cudaSuccess) return set_error(AXR_ECUDA, "axr_select_signs: %s", cudaGetErrorString(e));
   const int qtiles = (a.N + RC::BQ - 1) / RC::BQ;
   a.c0 = 0;
@@ -308,20 +331,57 @@ axr_status run_select(SelArgs a, cudaStream_t st) {
     rs = check_launch("axr_select_signs (candidates)");
     if (rs != AXR_OK) return rs;
   }
-  const double count = static_cast<double>(a.Ly) * a.S * a.Hq * a.N * D;
-  select_finalize_kernel<<<1, 32, 0, st>>>(a, count);
+  a.D_ = D;
+  select_finalize_kernel<<<1, 256, 0, st>>>(a, per_layer);
   return check_launch("axr_select_signs (finalize)");
 }
 
 template <int D>
-axr_status select_bits(int bits, const SelArgs& a, cudaStream_t st) {
+axr_status select_bits(int bits, const SelArgs& a, int per_layer, cudaStream_t st) {
   switch (bits) {
-    case 1: return run_select<D, 1>(a, st);
-    case 2: return run_select<D, 2>(a, st);
-    case 3: return run_select<D, 3>(a, st);
-    case 4: return run_select<D, 4>(a, st);
+    case 1: return run_select<D, 1>(a, per_layer, st);
+    case 2: return run_select<D, 2>(a, per_layer, st);
+    case 3: return run_select<D, 3>(a, per_layer, st);
+    case 4: return run_select<D, 4>(a, per_layer, st);
   }
   return set_error(AXR_EUNSUPPORTED, "axr_select_signs: bits=%d", bits);
+}
+
+axr_status select_impl(const char* w, const float* q, const uint16_t* k, const uint16_t* v, int n_layers, int n_seq,
+                       int n_tok, int Hq, int Hkv, int d, int bits, const int8_t* candidates, int n_cand, int causal,
+                       double* mse_out, int32_t* best_out, double* parts_out, int per_layer, void* workspace,
+                       size_t ws_bytes, void* stream) {
+  if (n_layers <= 0 || n_seq <= 0 || n_tok <= 0 || Hq <= 0 || Hkv <= 0 || n_cand <= 0)
+    return set_error(AXR_EINVAL, "%s: sizes must be positive", w);
+  if (Hq % Hkv) return set_error(AXR_EINVAL, "%s: Hq=%d not a multiple of Hkv=%d", w, Hq, Hkv);
+  if (d != 8 && d != 64 && d != 128) return set_error(AXR_EUNSUPPORTED, "%s: d=%d not in {8,64,128}", w, d);
+  if (bits < 1 || bits > 4) return set_error(AXR_EUNSUPPORTED, "%s: bits=%d outside 1..4", w, bits);
+  if (!q || !k || !v || !candidates || !mse_out || !best_out) return set_error(AXR_EINVAL, "%s: null pointer", w);
+  if (!aligned(q, 4) || !aligned(k, 2) || !aligned(v, 2) || !aligned(mse_out, 8) || !aligned(best_out, 4) ||
+      (parts_out && !aligned(parts_out, 8)))
+    return set_error(AXR_EINVAL, "%s: misaligned pointer", w);
+  const SelLayout L = sel_layout(n_layers, n_seq, n_tok, Hq, Hkv, d, n_cand);
+  if (!workspace || ws_bytes < L.total)
+    return set_error(AXR_EWORKSPACE, "%s: workspace of %zu bytes, need %zu", w, workspace ? ws_bytes : 0, L.total);
+  if (!aligned(workspace, 16)) return set_error(AXR_EINVAL, "%s: workspace not 16-byte aligned", w);
+  const Codebook* cb = codebook_for(d, bits);
+  if (!cb) return set_error(AXR_EINVAL, "%s: codebook unavailable", w);
+  SelArgs a;
+  memset(&a, 0, sizeof(a));
+  char* base = static_cast<char*>(workspace);
+  a.q = q; a.k = reinterpret_cast<const __half*>(k); a.v = reinterpret_cast<const __half*>(v);
+  a.cand = candidates; a.mse = mse_out; a.best = best_out; a.parts = parts_out;
+  a.oref = reinterpret_cast<double*>(base + L.oref);
+  a.khat = reinterpret_cast<float*>(base + L.khat);
+  a.acc = reinterpret_cast<double*>(base + L.acc);
+  a.Ly = n_layers; a.S = n_seq; a.Hq = Hq; a.Hkv = Hkv; a.N = n_tok; a.C = n_cand; a.causal = causal ? 1 : 0;
+  a.cb = *cb;
+  cudaStream_t st = as_stream(stream);
+  switch (d) {
+    case 8: return select_bits<8>(bits, a, per_layer, st);
+    case 64: return select_bits<64>(bits, a, per_layer, st);
+    default: return select_bits<128>(bits, a, per_layer, st);
+  }
 }
 
 }  // namespace
@@ -337,36 +397,17 @@ extern "C" axr_status axr_select_signs(const float* q, const uint16_t* k, const 
                                        int n_tok, int Hq, int Hkv, int d, int bits, const int8_t* candidates,
                                        int n_cand, int causal, double* mse_out, int32_t* best_out, void* workspace,
                                        size_t ws_bytes, void* stream) {
-  using namespace axr;
-  const char* w = "axr_select_signs";
-  if (n_layers <= 0 || n_seq <= 0 || n_tok <= 0 || Hq <= 0 || Hkv <= 0 || n_cand <= 0)
-    return set_error(AXR_EINVAL, "%s: sizes must be positive", w);
-  if (Hq % Hkv) return set_error(AXR_EINVAL, "%s: Hq=%d not a multiple of Hkv=%d", w, Hq, Hkv);
-  if (d != 8 && d != 64 && d != 128) return set_error(AXR_EUNSUPPORTED, "%s: d=%d not in {8,64,128}", w, d);
-  if (bits < 1 || bits > 4) return set_error(AXR_EUNSUPPORTED, "%s: bits=%d outside 1..4", w, bits);
-  if (!q || !k || !v || !candidates || !mse_out || !best_out) return set_error(AXR_EINVAL, "%s: null pointer", w);
-  if (!aligned(q, 4) || !aligned(k, 2) || !aligned(v, 2) || !aligned(mse_out, 8) || !aligned(best_out, 4))
-    return set_error(AXR_EINVAL, "%s: misaligned pointer", w);
-  const SelLayout L = sel_layout(n_layers, n_seq, n_tok, Hq, Hkv, d, n_cand);
-  if (!workspace || ws_bytes < L.total)
-    return set_error(AXR_EWORKSPACE, "%s: workspace of %zu bytes, need %zu", w, workspace ? ws_bytes : 0, L.total);
-  if (!aligned(workspace, 16)) return set_error(AXR_EINVAL, "%s: workspace not 16-byte aligned", w);
-  const Codebook* cb = codebook_for(d, bits);
-  if (!cb) return set_error(AXR_EINVAL, "%s: codebook unavailable", w);
-  SelArgs a;
-  memset(&a, 0, sizeof(a));
-  char* base = static_cast<char*>(workspace);
-  a.q = q; a.k = reinterpret_cast<const __half*>(k); a.v = reinterpret_cast<const __half*>(v);
-  a.cand = candidates; a.mse = mse_out; a.best = best_out;
-  a.oref = reinterpret_cast<double*>(base + L.oref);
-  a.khat = reinterpret_cast<float*>(base + L.khat);
-  a.acc = reinterpret_cast<double*>(base + L.acc);
-  a.Ly = n_layers; a.S = n_seq; a.Hq = Hq; a.Hkv = Hkv; a.N = n_tok; a.C = n_cand; a.causal = causal ? 1 : 0;
-  a.cb = *cb;
-  cudaStream_t st = as_stream(stream);
-  switch (d) {
-    case 8: return select_bits<8>(bits, a, st);
-    case 64: return select_bits<64>(bits, a, st);
-    default: return select_bits<128>(bits, a, st);
-  }
+  return axr::select_impl("axr_select_signs", q, k, v, n_layers, n_seq, n_tok, Hq, Hkv, d, bits, candidates, n_cand,
+                          causal, mse_out, best_out, nullptr, 0, workspace, ws_bytes, stream);
+}
+
+extern "C" axr_status axr_select_signs_per_layer(const float* q, const uint16_t* k, const uint16_t* v, int n_layers,
+                                                 int n_seq, int n_tok, int Hq, int Hkv, int d, int bits,
+                                                 const int8_t* candidates, int n_cand, int causal,
+                                                 double* mse_layers_out, int32_t* best_layers_out,
+                                                 double* mse_parts_out, void* workspace, size_t ws_bytes,
+                                                 void* stream) {
+  return axr::select_impl("axr_select_signs_per_layer", q, k, v, n_layers, n_seq, n_tok, Hq, Hkv, d, bits,
+                          candidates, n_cand, causal, mse_layers_out, best_layers_out, mse_parts_out, 1, workspace,
+                          ws_bytes, stream);
 }

@@ -133,11 +133,10 @@ __device__ __forceinline__ void mbar_init(uint64_t* mbar, uint32_t count) {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-// Wait for the phase of parity `parity` to complete; gives up after a bounded number of polls (about a second)
-// and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity) {
+// Wait for the phase of parity `parity` to complete; gives up after `polls` try_wait polls and returns false.
+__device__ __forceinline__ bool mbar_wait_polls(uint64_t* mbar, uint32_t parity, int polls) {
   const uint32_t mb = static_cast<uint32_t>(__cvta_generic_to_shared(mbar));
-  for (int it = 0; it < (1 << 20); ++it) {
+  for (int it = 0; it < polls; ++it) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
@@ -147,6 +146,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity) {
     if (done) return true;
   }
   return false;
+}
+
+// Wait for the phase of parity `parity` to complete; gives up after a bounded number of polls (about a second)
+// and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t* mbar, uint32_t parity) {
+  return mbar_wait_polls(mbar, parity, 1 << 20);
 }
 
 // ---- tables and operands ----------------------------------------------------------------------------------------

@@ -334,3 +334,208 @@ def select_signs(q, k, v, candidates, bits, causal=True, workspace=None):
                                      1 if causal else 0, _ptr(mse), _ptr(best), _ptr(ws), ws.numel(), _stream())
     _abi.check(st, "axr_select_signs")
     return mse, best
+
+
+def select_signs_per_layer(q, k, v, candidates, bits, causal=True, parts=False, workspace=None):
+    """One sign vector per layer: per-layer MSE of every candidate (the mean over that layer's sequences, heads,
+    positions and coordinates) and each layer's first argmin.  Returns (mse [Ly, C] float64, best [Ly] int32) and,
+    with parts, also the MSE of each (layer, sequence) [Ly, S, C] float64, as CUDA tensors."""
+    _need_cuda("q", q, torch.float32)
+    _need_cuda("k", k, torch.float16)
+    _need_cuda("v", v, torch.float16)
+    _need_cuda("candidates", candidates, torch.int8)
+    Ly, S, Hq, N, d = q.shape
+    Hkv = k.shape[2]
+    if tuple(k.shape) != (Ly, S, Hkv, N, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("k, v must be [Ly, S, Hkv, N, d]")
+    C = candidates.shape[0]
+    if tuple(candidates.shape) != (C, d):
+        raise ValueError("candidates must be [C, d]")
+    mse = torch.empty((Ly, C), dtype=torch.float64, device=q.device)
+    best = torch.empty(Ly, dtype=torch.int32, device=q.device)
+    mparts = torch.empty((Ly, S, C), dtype=torch.float64, device=q.device) if parts else None
+    nbytes = select_workspace_bytes(Ly, S, N, Hq, Hkv, d, C)
+    ws = _workspace(nbytes, q.device, workspace)
+    st = _abi.lib().axr_select_signs_per_layer(_ptr(q), _ptr(k), _ptr(v), Ly, S, N, Hq, Hkv, d, bits,
+                                               _ptr(candidates), C, 1 if causal else 0, _ptr(mse), _ptr(best),
+                                               _ptr(mparts), _ptr(ws), ws.numel(), _stream())
+    _abi.check(st, "axr_select_signs_per_layer")
+    return (mse, best, mparts) if parts else (mse, best)
+
+
+def device_status(clear: bool = False) -> int:
+    """The current device's status word (synchronizes the device): AXR_STATUS_WAIT_TIMEOUT (1) if a kernel's bounded
+    wait gave up since the word was last cleared (its outputs hold NaN), else 0.  clear resets it."""
+    flags = ctypes.c_uint(0)
+    st = _abi.lib().axr_device_status(ctypes.byref(flags), 1 if clear else 0)
+    if st not in (0, 3):
+        _abi.check(st, "axr_device_status")
+    if st == 3 and not (flags.value & _abi.STATUS_WAIT_TIMEOUT):
+        _abi.check(st, "axr_device_status")
+    return int(flags.value)
+
+
+def _paged_dims(q, kcodes, knorms, block_table, bits):
+    _need_cuda("q", q, torch.float32)
+    _need_cuda("kcodes", kcodes, torch.uint8)
+    _need_cuda("knorms", knorms, torch.float16)
+    _need_cuda("block_table", block_table, torch.int32)
+    if q.dim() != 3 or kcodes.dim() != 4 or knorms.dim() != 3 or block_table.dim() != 2:
+        raise ValueError("q [B,Hq,d], kcodes [blocks,Hkv,bt,R], knorms [blocks,Hkv,bt], block_table [B,max_blocks]")
+    B, Hq, d = q.shape
+    nb, Hkv, bt, R = kcodes.shape
+    if R != row_bytes(d, bits) or tuple(knorms.shape) != (nb, Hkv, bt) or block_table.shape[0] != B:
+        raise ValueError("pool shapes do not match q, d, bits and the block table")
+    return B, Hq, Hkv, d, bt, block_table.shape[1]
+
+
+def _paged_values(v, vcodes, vnorms, kcodes, knorms, d):
+    if (v is None) == (vcodes is None):
+        raise ValueError("pass exactly one of v or vcodes")
+    if v is not None:
+        _need_cuda("v", v, torch.float16)
+        if tuple(v.shape) != tuple(kcodes.shape[:3]) + (d,):
+            raise ValueError("v must be [blocks, Hkv, bt, d]")
+        return _abi.V_F16, _ptr(v), None
+    _need_cuda("vcodes", vcodes, torch.uint8)
+    _need_cuda("vnorms", vnorms, torch.float16)
+    if vcodes.shape != kcodes.shape or vnorms.shape != knorms.shape:
+        raise ValueError("vcodes / vnorms must have the key pools' shapes")
+    return _abi.V_QUANT, _ptr(vcodes), _ptr(vnorms)
+
+
+def attend_decode_paged(q, kcodes, knorms, signs, bits, block_table, seq_lens=None, T=None, v=None, vcodes=None,
+                        vnorms=None, scale=None, out=None, workspace=None):
+    """axr_attend_decode over paged pools: kcodes [blocks, Hkv, bt, R], knorms [blocks, Hkv, bt], values v [blocks,
+    Hkv, bt, d] float16 or vcodes/vnorms shaped like the key pools; block_table [B, max_blocks] int32 maps logical
+    block j of batch row b to its pool block.  T (default max_blocks * bt) bounds seq_lens.  Returns out [B, Hq, d]."""
+    B, Hq, Hkv, d, bt, mb = _paged_dims(q, kcodes, knorms, block_table, bits)
+    _need_cuda("signs", signs, torch.int8)
+    T = mb * bt if T is None else int(T)
+    seq_lens = _lens(seq_lens, B)
+    vkind, vptr, vnptr = _paged_values(v, vcodes, vnorms, kcodes, knorms, d)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    _need_cuda("out", out, torch.float32)
+    ws = _workspace(attend_workspace_bytes(B, Hq, Hkv, T, d), q.device, workspace)
+    st = _abi.lib().axr_attend_decode_paged(_ptr(q), _ptr(kcodes), _ptr(knorms), vkind, vptr, vnptr, _ptr(block_table),
+                                            mb, bt, _ptr(seq_lens), B, Hq, Hkv, T, d, bits, _ptr(signs), scale,
+                                            _ptr(out), _ptr(ws), ws.numel(), _stream())
+    _abi.check(st, "axr_attend_decode_paged")
+    return out
+
+
+def decode_step_paged(q, k_new, v_new, kcodes, knorms, signs, bits, block_table, seq_lens=None, T=None, v=None,
+                      vcodes=None, vnorms=None, scale=None, out=None, workspace=None):
+    """axr_decode_step over paged pools: k_new, v_new (float16 [B, Hkv, d]) are written at position seq_lens[b] - 1
+    through the block table, then attention runs over [0, seq_lens[b]).  The pools are updated in place."""
+    B, Hq, Hkv, d, bt, mb = _paged_dims(q, kcodes, knorms, block_table, bits)
+    _need_cuda("signs", signs, torch.int8)
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        _need_cuda(name, t, torch.float16)
+        if tuple(t.shape) != (B, Hkv, d):
+            raise ValueError(f"{name} must be a contiguous [B, Hkv, d] float16 tensor")
+    T = mb * bt if T is None else int(T)
+    seq_lens = _lens(seq_lens, B)
+    vkind, vptr, vnptr = _paged_values(v, vcodes, vnorms, kcodes, knorms, d)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    _need_cuda("out", out, torch.float32)
+    ws = _workspace(attend_workspace_bytes(B, Hq, Hkv, T, d), q.device, workspace)
+    st = _abi.lib().axr_decode_step_paged(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(kcodes), _ptr(knorms), vkind, vptr,
+                                          vnptr, _ptr(block_table), mb, bt, _ptr(seq_lens), B, Hq, Hkv, T, d, bits,
+                                          _ptr(signs), scale, _ptr(out), _ptr(ws), ws.numel(), _stream())
+    _abi.check(st, "axr_decode_step_paged")
+    return out
+
+
+# ---- LOOKAT product quantization ------------------------------------------------------------------------------------
+
+def pq_train(x, codebooks, iters, workspace=None):
+    """Lloyd k-means of one head's keys x [n, d] (float16/float32), per subspace, from the initial centroids in
+    codebooks [m, K, d/m] float32, which are updated in place and returned."""
+    _need_cuda("x", x)
+    _need_cuda("codebooks", codebooks, torch.float32)
+    if x.dtype not in (torch.float16, torch.float32):
+        raise TypeError("x must be float16 or float32")
+    m, K, ds = codebooks.shape
+    d = x.shape[-1]
+    if m * ds != d:
+        raise ValueError("codebooks do not match d")
+    n = x.numel() // d
+    nbytes = int(_abi.lib().axr_pq_train_workspace_bytes(d, m, K))
+    ws = _workspace(nbytes, x.device, workspace)
+    dt = _abi.F16 if x.dtype == torch.float16 else _abi.F32
+    st = _abi.lib().axr_pq_train(_ptr(x), dt, n, d, m, K, int(iters), _ptr(codebooks), _ptr(ws), ws.numel(),
+                                 _stream())
+    _abi.check(st, "axr_pq_train")
+    return codebooks
+
+
+def pq_encode(x, codebooks, head_period=None, codes=None, dst_rows=None):
+    """Indices (uint8 [..., m]) of the nearest centroids of x [..., d]; codebooks [heads, m, K, d/m] float32, vector
+    r using set (r / head_period) % heads (default head_period: x.shape[-2] for a [B, Hkv, T, d] cache, i.e. the
+    head axis is x.shape[-3])."""
+    _need_cuda("x", x)
+    _need_cuda("codebooks", codebooks, torch.float32)
+    if codebooks.dim() == 3:
+        codebooks = codebooks.unsqueeze(0)
+    H, m, K, ds = codebooks.shape
+    d = x.shape[-1]
+    n = x.numel() // d
+    if head_period is None:
+        head_period = x.shape[-2] if (H > 1 and x.dim() >= 3) else max(n, 1)
+    if dst_rows is None:
+        if codes is None:
+            codes = torch.empty(x.shape[:-1] + (m,), dtype=torch.uint8, device=x.device)
+    else:
+        _need_cuda("dst_rows", dst_rows, torch.int64)
+        if codes is None:
+            raise ValueError("dst_rows needs the destination codes buffer")
+    _need_cuda("codes", codes, torch.uint8)
+    dt = _abi.F16 if x.dtype == torch.float16 else _abi.F32
+    st = _abi.lib().axr_pq_encode(_ptr(x), dt, n, d, m, K, _ptr(codebooks), H, int(head_period), _ptr(dst_rows),
+                                  _ptr(codes), _stream())
+    _abi.check(st, "axr_pq_encode")
+    return codes
+
+
+def pq_score(q, codes, codebooks, scale=1.0, seq_lens=None, T=None, out=None):
+    """ADC scores [B, Hq, T]: q [B, Hq, d] float32, codes [B, Hkv, Tcap, m] uint8, codebooks [Hkv, m, K, d/m]."""
+    _need_cuda("q", q, torch.float32)
+    _need_cuda("codes", codes, torch.uint8)
+    _need_cuda("codebooks", codebooks, torch.float32)
+    B, Hq, d = q.shape
+    _, Hkv, Tcap, m = codes.shape
+    K = codebooks.shape[2]
+    T = Tcap if T is None else int(T)
+    seq_lens = _lens(seq_lens, B)
+    if out is None:
+        out = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    st = _abi.lib().axr_pq_score(_ptr(q), _ptr(codes), _ptr(codebooks), _ptr(seq_lens), B, Hq, Hkv, T, Tcap, d, m, K,
+                                 float(scale), _ptr(out), _stream())
+    _abi.check(st, "axr_pq_score")
+    return out
+
+
+def pq_attend_decode(q, codes, codebooks, v, scale=None, seq_lens=None, T=None, out=None, workspace=None):
+    """Decode attention over product-quantized keys and float16 values v [B, Hkv, Tcap, d]."""
+    _need_cuda("q", q, torch.float32)
+    _need_cuda("codes", codes, torch.uint8)
+    _need_cuda("codebooks", codebooks, torch.float32)
+    _need_cuda("v", v, torch.float16)
+    B, Hq, d = q.shape
+    _, Hkv, Tcap, m = codes.shape
+    K = codebooks.shape[2]
+    T = Tcap if T is None else int(T)
+    seq_lens = _lens(seq_lens, B)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    ws = _workspace(attend_workspace_bytes(B, Hq, Hkv, T, d), q.device, workspace)
+    st = _abi.lib().axr_pq_attend_decode(_ptr(q), _ptr(codes), _ptr(codebooks), _ptr(v), _ptr(seq_lens), B, Hq, Hkv,
+                                         T, Tcap, d, m, K, scale, _ptr(out), _ptr(ws), ws.numel(), _stream())
+    _abi.check(st, "axr_pq_attend_decode")
+    return out

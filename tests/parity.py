@@ -5,8 +5,9 @@
 * Norms: the fp16 bits are exact, except where the fp64 norm lies within a few fp32 ulps of an fp16 rounding
   midpoint (the kernel rounds its fp32 norm, the oracle its fp64 norm).
 * Scores: |s_gpu - s_oracle| <= 1e-6 + 1e-5 * A_t, with A_t = scale * n16_t * sum_j |q~_j c_{idx_t,j}| (fp32
-  summation error is bounded by the sum of the absolute terms, not by |s|); the strict |s|-relative reading is
-  reported alongside.
+  summation error is bounded by the sum of the absolute terms, not by |s|); the strict |s|-relative reading
+  (1e-6 + 1e-5 |s|) is counted per test, printed in the session summary and held below STRICT_FRACTION of the
+  scores compared.
 * Attention outputs: per (batch, head) ||o_gpu - o_oracle|| / ||o_oracle|| <= 2e-3.
 """
 
@@ -36,7 +37,7 @@ def check_indices(gpu_codes, x, signs, d, bits):
         k = np.maximum(gi, oi)
         dist = np.abs(uu - t[k - 1])
         assert np.all(dist < BOUNDARY), f"index mismatch {dist.max():.3e} away from a threshold"
-    assert nm < MISMATCH_FRACTION * idx.size + 1, f"{nm} index mismatches of {idx.size}"
+    assert nm < MISMATCH_FRACTION * idx.size, f"{nm} index mismatches of {idx.size}"
     return nm, idx.size
 
 
@@ -65,14 +66,31 @@ def abs_score_scale(q, codes, n16, signs, bits, scale):
     return abs(scale) * np.asarray(n16, np.float64) * lut[np.arange(d)[None, :], idx].sum(-1)
 
 
-def check_scores(gpu, want, A):
+# Scores that fail the strict |s|-relative reading (1e-6 + 1e-5 |s|), pooled per test: the gate is the A_t bound
+# above, but the strict count is recorded (printed in the session summary) and bounded by STRICT_FRACTION.
+STRICT_FRACTION = 1e-2
+STRICT_LOG: dict = {}
+
+
+def check_scores(gpu, want, A, tag=None):
     gpu = np.asarray(gpu, np.float64)
+    want = np.asarray(want, np.float64)
     err = np.abs(gpu - want)
     bound = SCORE_ABS + SCORE_REL * A
     bad = err > bound
     assert not bad.any(), f"{int(bad.sum())} scores out of tolerance; worst ratio {np.max(err / bound):.3g}"
     strict = err > SCORE_ABS + SCORE_REL * np.abs(want)
-    return float(np.max(err / bound)), int(strict.sum())
+    ns, n = int(strict.sum()), int(strict.size)
+    key = tag or _current_test()
+    old = STRICT_LOG.get(key, (0, 0))
+    STRICT_LOG[key] = (old[0] + ns, old[1] + n)
+    assert ns <= STRICT_FRACTION * n, f"{ns} of {n} scores fail the strict |s|-relative reading"
+    return float(np.max(err / bound)), ns
+
+
+def _current_test():
+    import os
+    return os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
 
 
 def check_outputs(gpu, want):
@@ -82,3 +100,19 @@ def check_outputs(gpu, want):
     rel = np.where(den > 0, num / np.where(den > 0, den, 1), num)
     assert np.all(rel <= OUT_REL_L2), f"max relative L2 error {rel.max():.3e}"
     return float(rel.max())
+
+
+def boundary_candidates(k, candidates, bits, radius=BOUNDARY):
+    """Candidates (sign vectors) under which some key coordinate's unit value lies within `radius` of a decision
+    threshold: there the kernel's fp32 decision may legitimately differ from the oracle's fp64 one (reading of the
+    index criterion above), and at small d one such index moves a selector MSE far beyond its rounding tolerance.
+    Returns a boolean mask over the candidates."""
+    k = np.asarray(k)
+    d = k.shape[-1]
+    _, t = oracle.codebook(d, bits)
+    rows = k.reshape(-1, d)
+    out = np.zeros(len(candidates), bool)
+    for i, s in enumerate(candidates):
+        _, _, _, u = oracle.quantize_rows(rows, s, bits)
+        out[i] = bool(np.any(np.abs(u[..., None] - t) < radius))
+    return out

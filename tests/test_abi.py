@@ -159,3 +159,43 @@ def test_select_argument_errors(L):
     assert call(Ly=0) == 1
     assert call(wsb=ws - 1) == 4
     assert call(ws=None) == 4
+
+
+def test_select_per_layer_argument_errors(L):
+    ws = L.axr_select_workspace_bytes(2, 2, 64, 16, 2, 128, 8)
+    # the per-(candidate, layer, sequence) sums are part of the workspace
+    assert ws >= 8 * 2 * 2 * 8 and ws == L.axr_select_workspace_bytes(2, 2, 64, 16, 2, 128, 8)
+    call = lambda **kw: L.axr_select_signs_per_layer(FAKE, FAKE, FAKE, kw.get("Ly", 2), 2, 64, kw.get("Hq", 16), 2,
+                                                     kw.get("d", 128), kw.get("bits", 4), FAKE, 8, 1, FAKE, FAKE,
+                                                     kw.get("parts", None), kw.get("ws", FAKE), kw.get("wsb", ws),
+                                                     None)
+    assert call(d=32) == 2
+    assert call(bits=0) == 2
+    assert call(Hq=15) == 1
+    assert call(Ly=0) == 1
+    assert call(parts=FAKE + 4) == 1  # f64 parts need 8-byte alignment
+    assert call(wsb=ws - 1) == 4
+    assert call(ws=None) == 4
+
+
+def test_status_argument_errors(L):
+    """Host-side rejections of the status entry points (no CUDA call is made)."""
+    assert L.axr_device_status(None, 0) == 1 and b"null" in L.axr_last_error()
+    for polls in (0, -1, (1 << 20) + 1):
+        assert L.axr_selftest_wait_timeout(polls, None) == 1
+
+
+def test_paged_argument_errors_host(L):
+    """Rejections made on the host before any launch (block size, table reach, null table, tiled values)."""
+    call = lambda **kw: L.axr_attend_decode_paged(FAKE, FAKE, FAKE, kw.get("vk", 1), FAKE, FAKE, kw.get("tab", FAKE),
+                                                  kw.get("mb", 4), kw.get("bt", 64), None, 2, 8, 2, kw.get("T", 256),
+                                                  128, 4, FAKE, 0.088, FAKE, FAKE, 1 << 20, None)
+    assert call(bt=48) == 1 and b"power of two" in L.axr_last_error()
+    assert call(bt=8) == 1
+    assert call(T=257) == 1 and b"exceeds" in L.axr_last_error()
+    assert call(tab=None) == 1
+    assert call(tab=FAKE + 2) == 1
+    assert call(vk=2) == 1
+    step = L.axr_decode_step_paged(FAKE, None, FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE, 4, 64, None, 2, 8, 2, 256, 128,
+                                   4, FAKE, 0.088, FAKE, FAKE, 1 << 20, None)
+    assert step == 1

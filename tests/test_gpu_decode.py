@@ -47,6 +47,7 @@ SMALL += [(64, 4, g, False) for g in (1, 2, 8)]
 SCORE_CASES = [(d, b, g, m) for m in ("tensor", "mma") for d, b, g in sorted({(d, b, g) for d, b, g, _ in SMALL})]
 SCORE_CASES += [(d, b, g, m) for m in ("factored", "table") for d, b, g in [(128, 4, 4), (64, 3, 4), (128, 2, 8),
                                                                              (128, 1, 1)]]
+SCORE_CASES += [(d, b, g, "table") for d, b, g in [(128, 2, 4), (128, 4, 1), (64, 1, 8), (128, 3, 8), (64, 2, 2)]]
 
 
 # the attend kernels follow the gather mode: "mma" (the default) scores keys through warp-level MMAs, "factored" on
@@ -54,6 +55,9 @@ SCORE_CASES += [(d, b, g, m) for m in ("factored", "table") for d, b, g in [(128
 ATTEND_CASES = [(d, b, g, vq, "mma") for d, b, g, vq in SMALL]
 ATTEND_CASES += [(d, b, g, vq, "factored") for d, b, g, vq in [(128, 4, 4, True), (128, 4, 4, False), (64, 3, 4, True),
                                                                 (128, 2, 8, False), (128, 1, 1, True)]]
+# the literal table (fp16 values): fields of 8 bits at b <= 2, 6 at b = 3, 8 or 4 at b = 4
+ATTEND_CASES += [(d, b, g, False, "table") for d, b, g in [(128, 4, 4), (128, 4, 2), (128, 2, 4), (128, 2, 8), (64, 3, 4),
+                                                           (128, 1, 8), (64, 1, 1)]]
 
 
 @pytest.fixture
@@ -375,3 +379,50 @@ def test_long_context_kv_quantized_full_size():
 def test_sweep_rows_sampled(B, T, bits, d):
     w = W.sweep_case(B, T, bits, d)
     _full_size(w, [(0, 0), (B - 1, 31)])
+
+
+def _sweep_device(w, samples):
+    """A decode-sweep row at its full size with inputs drawn on the device by the benchmark's own generators (one
+    batch row at a time, as the benchmark does; the host could not hold B=64 x T=131072 in numpy).  The attend
+    runs in the benchmark's launch configuration; each sampled (batch row, query head) is recomputed by the oracle
+    from that unit's inputs copied back to the host: indices and norms of the GPU writer, scores of the GPU scorer
+    on the oracle's codes, and the attention output."""
+    B, Hq, Hkv, T, d, bits, G = w.B, w.Hq, w.Hkv, w.T, w.d, w.bits, w.G
+    dev = torch.device("cuda")
+    st = cuda(W.sign_vector(d, w.seed + 4))
+    s = st.cpu().numpy()
+    k = torch.empty((B, Hkv, T, d), dtype=torch.float16, device=dev)
+    v = torch.empty((B, Hkv, T, d), dtype=torch.float16, device=dev)
+    for b in range(B):
+        k[b] = W.lognormal_rows_device((Hkv, T, d), w.seed + 7919 * b, dev)
+        v[b] = W.lognormal_rows_device((Hkv, T, d), w.seed + 2 + 7919 * b, dev)
+    q = W.normal_device((B, Hq, d), w.seed + 3, dev, dtype=torch.float32)
+    kc, kn = ops.write_keys(k, st, bits)
+    out = ops.attend_decode(q, kc, kn, st, bits, v=v).cpu().numpy()
+    scale = 1.0 / math.sqrt(d)
+    qh = q.cpu().numpy()
+    for b, h in samples:
+        hk = h // G
+        kh, vh = k[b, hk].cpu().numpy(), v[b, hk].cpu().numpy()
+        parity.check_indices(kc[b, hk].cpu().numpy(), kh, s, d, bits)
+        parity.check_norms(kn[b, hk].cpu().numpy(), kh)
+        okc, okn = oracle.write(kh, s, bits)
+        want = oracle.decode_attention(qh[b:b + 1, h:h + 1], okc[None, None], okn[None, None], s, bits, scale,
+                                       v=vh[None, None])
+        parity.check_outputs(out[b:b + 1, h:h + 1], want)
+        sc = ops.score(q[b:b + 1, hk * G:(hk + 1) * G].contiguous(), cuda(okc[None, None]), cuda(okn[None, None]),
+                       st, bits, scale=scale).cpu().numpy()[0, h - hk * G]
+        want_s = oracle.score_lut(qh[b, h], okc, okn, s, bits, scale)
+        A = parity.abs_score_scale(qh[b, h].astype(np.float64), okc, okn, s, bits, scale)
+        parity.check_scores(sc, want_s, A)
+    del k, v, kc, kn
+    torch.cuda.empty_cache()
+
+
+# With test_sweep_rows_sampled every (b, d) pair of the sweep appears at least once, the largest row
+# (B=64, T=131072, b=4, d=128: 21.6 GB of cache) included.
+@pytest.mark.parametrize("B,T,bits,d", [(64, 131072, 4, 128), (8, 4096, 1, 128), (64, 32768, 2, 64),
+                                        (8, 131072, 3, 64)])
+def test_sweep_rows_sampled_device_inputs(B, T, bits, d):
+    w = W.sweep_case(B, T, bits, d)
+    _sweep_device(w, [(0, 0), (B // 2, 13), (B - 1, 31)])

@@ -72,18 +72,27 @@ def test_dst_rows_scatter_into_cache():
 
 def test_single_head_config_write_then_score():
     """Single head, d=128, b=2, 1024 fp32 keys x lognormal(0,0.5) norms: write on the GPU, then LUT scores on the
-    GPU, against the oracle's brute-force dequantize-then-dot on the oracle's own codes."""
+    GPU.  The scores are checked twice, whatever the index parity found: the GPU scorer on the oracle's own codes
+    against the oracle's brute-force dequantize-then-dot, and the GPU scorer on the GPU's codes against the
+    oracle's brute force on those same codes."""
     w = W.SINGLE_HEAD
     inp = W.decode_inputs(w)
     k = inp["k"][0, 0]  # [T, d] fp32
     q = inp["q"]        # [1, 1, d]
     s = inp["signs"]
-    codes, norms = ops.write_keys(cuda(k), cuda(s), w.bits)
-    nm, _ = parity.check_indices(codes.cpu().numpy(), k, s, w.d, w.bits)
+    st = cuda(s)
+    codes, norms = ops.write_keys(cuda(k), st, w.bits)
+    parity.check_indices(codes.cpu().numpy(), k, s, w.d, w.bits)
     parity.check_norms(norms.cpu().numpy(), k)
-    sc = ops.score(cuda(q), codes.view(1, 1, w.T, -1), norms.view(1, 1, w.T), cuda(s), w.bits, scale=1.0)
     oc, on = oracle.write(k, s, w.bits)
+    # the scorer on the oracle's codes
+    sc = ops.score(cuda(q), cuda(oc[None, None]), cuda(on[None, None]), st, w.bits, scale=1.0)
     want = oracle.score_bruteforce(q[0, 0], oc, on, s, w.bits)
     A = parity.abs_score_scale(q[0, 0].astype(np.float64), oc, on, s, w.bits, 1.0)
-    if nm == 0:
-        parity.check_scores(sc.cpu().numpy()[0, 0], want, A)
+    parity.check_scores(sc.cpu().numpy()[0, 0], want, A)
+    # the scorer on the GPU's own codes
+    gc, gn = codes.cpu().numpy(), norms.cpu().numpy()
+    sc2 = ops.score(cuda(q), codes.view(1, 1, w.T, -1), norms.view(1, 1, w.T), st, w.bits, scale=1.0)
+    want2 = oracle.score_bruteforce(q[0, 0], gc, gn, s, w.bits)
+    A2 = parity.abs_score_scale(q[0, 0].astype(np.float64), gc, gn, s, w.bits, 1.0)
+    parity.check_scores(sc2.cpu().numpy()[0, 0], want2, A2)
