@@ -164,3 +164,48 @@ def test_kmeans_mean_without_division_is_caught(monkeypatch):
     _patch_lk(monkeypatch, "pq_kmeans", bad_kmeans)
     with pytest.raises(AssertionError):
         TL.test_kmeans_matches_scikit_learn_lloyd()
+
+
+# ---- PoT oracle --------------------------------------------------------------------------------------------------------
+
+import oracle.pot as PT  # noqa: E402
+import tests.test_oracle_pot as TP  # noqa: E402
+
+
+def test_log_domain_rounding_is_caught(monkeypatch):
+    """Midpoints at the geometric mean of two levels (nearest in log2) instead of the arithmetic mean."""
+    def bad_thresholds(E, M):
+        lv = PT.pot_levels(E, M)
+        return np.sqrt(lv[:-1] * lv[1:]).astype(np.float32)
+    monkeypatch.setattr(PT, "pot_thresholds", bad_thresholds)
+    with pytest.raises(AssertionError):
+        TP.test_relative_error_of_nearest_level(3, 0, 1 / 3)
+
+
+def test_dropped_sign_flip_is_caught(monkeypatch):
+    real = PT.pot_score_int
+
+    def bad_score_int(Q, codes, E, M):  # the key's sign bit ignored
+        return real(Q, np.asarray(codes) & ((1 << (E + M)) - 1), E, M)
+    monkeypatch.setattr(PT, "pot_score_int", bad_score_int)
+    monkeypatch.setattr(oracle, "pot_score_int", bad_score_int)
+    with pytest.raises(AssertionError):
+        TP.test_shift_accumulate_is_the_exact_dot_product(3, 0)
+
+
+def test_short_headroom_is_caught(monkeypatch):
+    def bad_score_int(Q, codes, E, M):  # head-room one short: the largest level's shift is lost
+        e_max = (1 << E) - 1
+        codes = np.asarray(codes, dtype=np.int64)
+        rank = codes & ((1 << (E + M)) - 1)
+        neg = (codes >> (E + M)) & 1
+        e = e_max - (rank >> M)
+        mu = rank & ((1 << M) - 1)
+        F = e_max + M - 1
+        Qa = np.abs(np.asarray(Q, dtype=np.int64))
+        mag = (Qa[None, :] << np.maximum(F - e, 0)) + mu * (Qa[None, :] << np.maximum(F - e - M, 0))
+        return np.sum(np.sign(np.asarray(Q))[None, :] * np.where(neg == 1, -1, 1) * mag, axis=-1)
+    monkeypatch.setattr(PT, "pot_score_int", bad_score_int)
+    monkeypatch.setattr(oracle, "pot_score_int", bad_score_int)
+    with pytest.raises(AssertionError):
+        TP.test_shift_accumulate_is_the_exact_dot_product(3, 0)
