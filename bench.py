@@ -317,6 +317,56 @@ def _sweep(args, dev, time_calls):
     return rows
 
 
+def _codecs(w, dev, time_calls, signs, kc, kn, q, wsp):
+    """LOOKAT and PoT decode paths (and the AXELRAM literal table) at the workload's shape over fp16 values: mean ms
+    per call (L2 flushed before each), algorithmic HBM bytes (codes + per-token scale + fp16 values, or codes +
+    scale + fp32 scores for the scorers) and the fraction of the measured copy peak."""
+    import torch
+    from kv_cache_quantized_b200 import ops
+    B, Hq, Hkv, T, d, G = w.B, w.Hq, w.Hkv, w.T, w.d, w.G
+    peak = _peaks()[0]
+    units = B * Hkv * T
+    v = _gen_rows(W.normal_device, (B, Hkv, T, d), w.seed + 11, dev)
+    k = _gen_rows(W.lognormal_rows_device, (B, Hkv, T, d), w.seed + 12, dev)
+    out = torch.empty((B, Hq, d), dtype=torch.float32, device=dev)
+    res = {}
+
+    def rec(name, ms, per_unit):
+        gb = per_unit * units / (ms / 1e3) / 1e9
+        res[name] = {"ms": ms, "bytes_per_token_head": per_unit, "achieved_gbs": gb, "frac": gb / peak,
+                     "keys_heads_per_s": B * T * Hq / (ms / 1e3)}
+
+    # LOOKAT: codebooks by k-means on a slice of the keys (setup, not timed), codes written on the GPU
+    m, K = 8, 256
+    cbs = torch.empty((Hkv, m, K, d // m), dtype=torch.float32, device=dev)
+    for h in range(Hkv):
+        x = k[0, h, :65536].contiguous()
+        init = x[torch.arange(K, device=dev) * (x.shape[0] // K)].view(K, m, d // m).transpose(0, 1).contiguous()
+        cbs[h] = ops.pq_train(x, init.float(), 4)
+    pcodes = ops.pq_encode(k, cbs)
+    rec("lookat_attend", time_calls(lambda: ops.pq_attend_decode(q, pcodes, cbs, v, out=out, workspace=wsp)),
+        m + 2 * d)
+    rec("lookat_score", time_calls(lambda: ops.pq_score(q, pcodes, cbs, scale=1.0 / math.sqrt(d))), m + 4 * G)
+    del pcodes
+    # PoT, 4-bit codes (E = 3, M = 0)
+    pc, pa = ops.pot_write(k, 3, 0)
+    R = ops.pot_row_bytes(d, 3, 0)
+    rec("pot_attend", time_calls(lambda: ops.pot_attend_decode(q, pc, pa, v, 3, 0, out=out, workspace=wsp)),
+        R + 2 + 2 * d)
+    rec("pot_score", time_calls(lambda: ops.pot_score(q, pc, pa, 3, 0, scale=1.0 / math.sqrt(d))), R + 2 + 4 * G)
+    del pc, pa
+    # the AXELRAM literal table read over fp16 values, and the default read path on the same cache
+    ops.set_gather("table")
+    rec("axelram_table_attend_f16v", time_calls(lambda: ops.attend_decode(q, kc, kn, signs, w.bits, v=v, out=out,
+                                                                          workspace=wsp)), w.d * w.bits // 8 + 2 + 2 * d)
+    ops.set_gather("mma")
+    rec("axelram_mma_attend_f16v", time_calls(lambda: ops.attend_decode(q, kc, kn, signs, w.bits, v=v, out=out,
+                                                                        workspace=wsp)), w.d * w.bits // 8 + 2 + 2 * d)
+    del v, k
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_axr(args, w):
     import torch
     import torch.distributed as dist
@@ -439,7 +489,7 @@ def run_axr(args, w):
     scorer = {}
     if not args.no_scorer:
         sc_out = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
-        for mode in ("mma", "tensor", "factored", "table"):
+        for mode in ("mma", "direct", "tensor", "factored", "table"):
             ops.set_gather(mode)
             for _ in range(3):
                 ops.score(q, kc, kn, signs, bits, scale=1.0 / math.sqrt(d), out=sc_out)
@@ -471,6 +521,11 @@ def run_axr(args, w):
                  "value": B * T * Hq / (ms / 1e3), "unit": UNIT, "achieved_gbs": dbytes / (ms / 1e3) / 1e9,
                  "frac": dbytes / (ms / 1e3) / 1e9 / _peaks()[0], "algorithmic_bytes": dbytes}
         del kd, vd
+
+    # the other codecs through the same reducer, at this shape with fp16 values: LOOKAT product-quantized keys
+    # (m = 8 one-byte indices, K = 256) and power-of-two shift-accumulate keys (E = 3, M = 0: 4 bits), scores alone
+    # and decode attention; the AXELRAM literal-table read (AXR_GATHER_TABLE) over the same fp16 values beside them
+    codecs = _codecs(w, dev, time_calls, signs, kc, kn, q, wsp) if not args.no_codecs else None
 
     # the decode sweep (--sweep): the LUT attend with fp16 values next to the dense fp16 kernel, per shape
     sweep = _sweep(args, dev, time_calls) if args.sweep else None
@@ -516,6 +571,8 @@ def run_axr(args, w):
     }
     if sweep is not None:
         line["sweep"] = sweep
+    if codecs is not None:
+        line["codecs"] = codecs
     return line
 
 
@@ -645,6 +702,7 @@ def main(argv=None):
     ap.add_argument("--variants", action="store_true",
                     help="also time the attend over the tiled value layout (MMA and tcgen05 value products)")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense fp16 bandwidth reference")
+    ap.add_argument("--no-codecs", action="store_true", help="skip the LOOKAT / PoT / literal-table measurements")
     ap.add_argument("--sweep", action="store_true",
                     help="also run the decode sweep (B x T x bits x d, fp16 V) against the dense fp16 kernel")
     args = ap.parse_args(argv)

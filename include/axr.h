@@ -165,7 +165,11 @@ AXR_API axr_status axr_score(const float* q, const uint8_t* kcodes, const uint16
  *                        the row factors (split the same way) the other operand, and tcgen05.mma accumulates the
  *                        G sums per token in fp32;
  *   AXR_GATHER_MMA       the same hi/lo operands as warp-level MMAs (mma.sync, operands in registers): one table
- *                        lookup gives a token's hi and lo registers for two coordinates.
+ *                        lookup gives a token's hi and lo registers for two coordinates;
+ *   AXR_GATHER_DIRECT    the AXR_GATHER_MMA arithmetic with every lane's code slice loaded from global memory
+ *                        straight into registers (coalesced, several groups in flight per warp; no staging tile,
+ *                        no block barrier): shared memory serves the table lookups alone.  The decode entry
+ *                        points treat it as AXR_GATHER_MMA.
  * axr_attend_decode reads the key table in factored form; with tiled values the value product runs as warp-level
  * MMAs, or, in AXR_GATHER_TENSOR mode, both products run as tcgen05 MMAs.  Errors: AXR_EINVAL for an unknown mode.
  */
@@ -173,7 +177,8 @@ typedef enum axr_gather {
   AXR_GATHER_FACTORED = 0,
   AXR_GATHER_TABLE = 1,
   AXR_GATHER_TENSOR = 2,
-  AXR_GATHER_MMA = 3
+  AXR_GATHER_MMA = 3,
+  AXR_GATHER_DIRECT = 4
 } axr_gather;
 AXR_API axr_status axr_set_gather(axr_gather mode);
 AXR_API axr_gather axr_get_gather(void);
@@ -322,6 +327,39 @@ AXR_API axr_status axr_pq_attend_decode(const float* q, const uint8_t* codes, co
                                         const uint16_t* v, const int32_t* seq_lens, int B, int Hq, int Hkv, int T,
                                         int Tcap, int d, int m, int K, float scale, float* out, void* workspace,
                                         size_t ws_bytes, void* stream);
+
+/*
+ * Power-of-two shift-accumulate keys (the arxivdaily page of the shift-accumulate attention paper): a second codec
+ * through the same split-T reducer.  The page gives no formulas; the reading implemented here:
+ *   write: alpha = max_j |k_j| (fp16, exact); u = k / alpha (fp32); |u_j| to the nearest magnitude level
+ *     2^-e (1 + mu / 2^M) in linear value (a value on a midpoint goes up; e in [0, 2^E - 1], mu in [0, 2^M - 1]);
+ *     code = sign << (E + M) | l with l = (e_max - e) 2^M + mu the level's rank from the smallest; 1 + E + M bits per
+ *     coordinate packed LSB-first (rows of d (1 + E + M) / 8 bytes), alpha per row.
+ *   scores: the query in fixed point, Q_j = rint(q_j / s_q), s_q = max |q| / 32767 (fp32); S = sum_j sigma_j
+ *     ((Q_j << (F - e_j)) + mu_j (Q_j << (F - e_j - M))) with head-room F = e_max + M, an exact integer; the score is
+ *     scale * s_q * alpha * 2^-F * S.
+ *   attend: r_t = rint(float(S) * (s_q * (scale * log2 e) * alpha_t) * 2^-F) (fp32, in that order) is an integer
+ *     log2 weight; out = sum_t 2^(r_t - R) v_t / sum_t 2^(r_t - R), R = max_t r_t -- every weight and every rescale
+ *     (the running maximum, the split merge) an exact power of two.  fp16 values.
+ * Formats (E, M): (1, 0), (2, 0), (3, 0), (1, 1), (2, 1); d in {64, 128}; G in {1, 2, 4, 8}.
+ *   axr_pot_write: x [dev] [n_vec, d] fp16 (8-byte aligned rows); dst_rows [dev] int64 or NULL; codes [dev] out;
+ *     alpha [dev] out fp16 per row.
+ *   axr_pot_score: q [dev] [B, Hq, d] f32; codes [dev] [B, Hkv, Tcap, row] (16-byte aligned); alpha [dev]
+ *     [B, Hkv, Tcap] fp16; S_out [dev] out [B, Hq, T] int32 and/or scores [dev] out [B, Hq, T] f32 (either NULL;
+ *     past len_b: S = 0 and score -inf).
+ *   axr_pot_attend_decode: v [dev] [B, Hkv, Tcap, d] fp16; out [dev] [B, Hq, d] f32; workspace as
+ *     axr_attend_decode (axr_attend_workspace_bytes).
+ * Errors: AXR_EINVAL (pointers, sizes, alignment), AXR_EUNSUPPORTED (d, format, G), AXR_EWORKSPACE, AXR_ECUDA.
+ */
+AXR_API axr_status axr_pot_write(const uint16_t* x, int64_t n_vec, int d, int E, int M, const int64_t* dst_rows,
+                                 uint8_t* codes, uint16_t* alpha, void* stream);
+AXR_API axr_status axr_pot_score(const float* q, const uint8_t* codes, const uint16_t* alpha, const int32_t* seq_lens,
+                                 int B, int Hq, int Hkv, int T, int Tcap, int d, int E, int M, float scale,
+                                 int32_t* S_out, float* scores, void* stream);
+AXR_API axr_status axr_pot_attend_decode(const float* q, const uint8_t* codes, const uint16_t* alpha,
+                                         const uint16_t* v, const int32_t* seq_lens, int B, int Hq, int Hkv, int T,
+                                         int Tcap, int d, int E, int M, float scale, float* out, void* workspace,
+                                         size_t ws_bytes, void* stream);
 
 /* Bytes of workspace for axr_select_signs with these sizes. */
 AXR_API size_t axr_select_workspace_bytes(int n_layers, int n_seq, int n_tok, int Hq, int Hkv, int d, int n_cand);

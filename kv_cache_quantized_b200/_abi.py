@@ -15,7 +15,7 @@ LIB_PATH = os.path.join(_HERE, "libaxr.so")
 STATUS = {0: "AXR_OK", 1: "AXR_EINVAL", 2: "AXR_EUNSUPPORTED", 3: "AXR_ECUDA", 4: "AXR_EWORKSPACE"}
 F32, F16 = 0, 1
 V_F16, V_QUANT, V_QUANT_TILED = 0, 1, 2
-GATHER_FACTORED, GATHER_TABLE, GATHER_TENSOR, GATHER_MMA = 0, 1, 2, 3
+GATHER_FACTORED, GATHER_TABLE, GATHER_TENSOR, GATHER_MMA, GATHER_DIRECT = 0, 1, 2, 3, 4
 STATUS_WAIT_TIMEOUT = 1
 
 _p = ctypes.c_void_p
@@ -50,6 +50,9 @@ SIGNATURES = {
     "axr_pq_encode": (_i, [_p, _i, _i64, _i, _i, _i, _p, _i, _i, _p, _p, _p]),
     "axr_pq_score": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p]),
     "axr_pq_attend_decode": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
+    "axr_pot_write": (_i, [_p, _i64, _i, _i, _i, _p, _p, _p, _p]),
+    "axr_pot_score": (_i, [_p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p]),
+    "axr_pot_attend_decode": (_i, [_p, _p, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _sz, _p]),
     "axr_set_gather": (_i, [_i]),
     "axr_device_status": (_i, [_p, _i]),
     "axr_selftest_wait_timeout": (_i, [_i, _p]),

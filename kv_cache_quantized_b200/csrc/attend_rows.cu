@@ -1,55 +1,14 @@
-// Launcher of the row-layout decode kernel with MMA key scores (attend_rows.cuh).
-#include "attend_rows.cuh"
-#include "launch.h"
+// Launcher of the row-layout decode kernel (attend_rows.cuh) for contiguous caches; paged pools go to the
+// instances of attend_rows_paged.cu.
+#include "attend_rows_dispatch.cuh"
 
 namespace axr {
-namespace {
 
-// The C entry point a launch serves, for error messages: decode steps carry the new token.
-const char* entry_name(const DecodeArgs& a) { return a.knew != nullptr ? "axr_decode_step" : "axr_attend_decode"; }
-
-template <int D, int BITS, int G, bool VQ>
-axr_status launch(const DecodeArgs& a, cudaStream_t st) {
-  using S = RowsPlan<D, BITS, G, VQ>;
-  auto k1 = attend_rows_kernel<D, BITS, G, VQ>;
-  const char* what = entry_name(a);
-  axr_status rs = ensure_smem(k1, S::bytes, what);
-  if (rs != AXR_OK) return rs;
-  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent blocks loop over the items
-  const long resident = static_cast<long>(S::MIN_BLOCKS) * kSmCount;
-  k1<<<static_cast<unsigned>(items < resident ? items : resident), kDecThreads, S::bytes, st>>>(a);
-  launch_reduce<D, VQ>(a, st);
-  return check_launch(what);
-}
-
-template <int D, int BITS>
-axr_status by_g(int G, bool vq, const DecodeArgs& a, cudaStream_t st) {
-  switch (G) {
-    case 1: return vq ? launch<D, BITS, 1, true>(a, st) : launch<D, BITS, 1, false>(a, st);
-    case 2: return vq ? launch<D, BITS, 2, true>(a, st) : launch<D, BITS, 2, false>(a, st);
-    case 4: return vq ? launch<D, BITS, 4, true>(a, st) : launch<D, BITS, 4, false>(a, st);
-    case 8: return vq ? launch<D, BITS, 8, true>(a, st) : launch<D, BITS, 8, false>(a, st);
-  }
-  return set_error(AXR_EUNSUPPORTED, "%s: G=%d", entry_name(a), G);
-}
-
-template <int D>
-axr_status by_bits(int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st) {
-  switch (bits) {
-    case 1: return by_g<D, 1>(G, vq, a, st);
-    case 2: return by_g<D, 2>(G, vq, a, st);
-    case 3: return by_g<D, 3>(G, vq, a, st);
-    case 4: return by_g<D, 4>(G, vq, a, st);
-  }
-  return set_error(AXR_EUNSUPPORTED, "%s: bits=%d", entry_name(a), bits);
-}
-
-}  // namespace
+axr_status attend_rows_paged_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st);
 
 axr_status attend_rows_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st) {
-  if (d == 64) return by_bits<64>(bits, G, vq, a, st);
-  if (d == 128) return by_bits<128>(bits, G, vq, a, st);
-  return set_error(AXR_EUNSUPPORTED, "%s: d=%d", entry_name(a), d);
+  if (a.block_table) return attend_rows_paged_launch(d, bits, G, vq, a, st);
+  return rows_detail::dispatch<false>(d, bits, G, vq, a, st);
 }
 
 }  // namespace axr

@@ -86,7 +86,7 @@ struct RowsPlan {
   static_assert(bytes <= 227 * 1024, "shared memory of one block");
 };
 
-template <int D, int BITS, int G, bool VQ>
+template <int D, int BITS, int G, bool VQ, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, RowsPlan<D, BITS, G, VQ>::MIN_BLOCKS)
 attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
   using P = RowsPlan<D, BITS, G, VQ>;
@@ -140,7 +140,7 @@ attend_rows_kernel(const __grid_constant__ DecodeArgs a) {
     const int start = split * a.chunk;
     const int end = min(start + a.chunk, len);
     const int ntiles = end > start ? (end - start + TT - 1) / TT : 0;
-    const RowMap rm = row_map(a, b, hk);  // cache row of each token (contiguous or through the block table)
+    const RowMap<PAGED> rm = row_map<PAGED>(a, b, hk);  // cache row of each token (contiguous or paged)
     const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
 
     fence_proxy_async();  // the merge region's generic writes come before the bulk copies that reuse it

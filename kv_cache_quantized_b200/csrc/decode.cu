@@ -146,7 +146,7 @@ axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, con
   // fp16 values in AXR_GATHER_TABLE mode: the literal table in shared memory, values on the CUDA cores
   if (mode == kGatherTable && !vq) return table_attend_launch(d, bits, G, a, as_stream(stream));
   // row-layout values: keys scored through warp-level MMAs in AXR_GATHER_MMA mode, else on CUDA cores
-  if (mode == kGatherMma) {
+  if (mode == kGatherMma || mode == kGatherDirect) {
     // fp16 values: one warp per token range through scores, softmax and the value product (no block barrier);
     // quantized values: scoring and value warps one tile apart
     if (!vq && attend_fused_supported(d, bits)) return attend_fused_launch(d, bits, G, vq, a, as_stream(stream));
@@ -231,6 +231,7 @@ extern "C" axr_status axr_set_gather(axr_gather mode) {
   else if (mode == AXR_GATHER_TABLE) g_gather.store(kGatherTable);
   else if (mode == AXR_GATHER_TENSOR) g_gather.store(kGatherTensor);
   else if (mode == AXR_GATHER_MMA) g_gather.store(kGatherMma);
+  else if (mode == AXR_GATHER_DIRECT) g_gather.store(kGatherDirect);
   else return set_error(AXR_EINVAL, "axr_set_gather: unknown mode %d", (int)mode);
   return set_error(AXR_OK, "");
 }
@@ -240,5 +241,6 @@ extern "C" axr_gather axr_get_gather(void) {
   return m == axr::kGatherTable      ? AXR_GATHER_TABLE
          : m == axr::kGatherFactored ? AXR_GATHER_FACTORED
          : m == axr::kGatherMma      ? AXR_GATHER_MMA
+         : m == axr::kGatherDirect   ? AXR_GATHER_DIRECT
                                      : AXR_GATHER_TENSOR;
 }

@@ -26,7 +26,7 @@ constexpr int kDecThreads = 256;
 constexpr int kDecWarps = kDecThreads / kWarp;
 constexpr float kLog2e = 1.4426950408889634f;
 
-enum Gather { kGatherFactored = 0, kGatherTable = 1, kGatherTensor = 2, kGatherMma = 3 };
+enum Gather { kGatherFactored = 0, kGatherTable = 1, kGatherTensor = 2, kGatherMma = 3, kGatherDirect = 4 };
 
 struct DecodeArgs {
   const float* q;            // [B, Hq, D]
@@ -56,26 +56,31 @@ struct DecodeArgs {
 
 // Cache row of token t of one (batch row, KV head).  Contiguous caches [B, Hkv, Tcap] number the rows
 // (b Hkv + hk) Tcap + t; paged pools [num_blocks, Hkv, bt] number them (block_table[b][t / bt] Hkv + hk) bt + t % bt,
-// so the bt tokens of one (block, KV head) are contiguous.
+// so the bt tokens of one (block, KV head) are contiguous.  PAGED is a compile-time choice, so the contiguous
+// kernels carry none of the paging arithmetic.
+template <bool PAGED>
 struct RowMap {
-  const int32_t* table;  // the batch row's block table, or null (contiguous)
+  const int32_t* table;  // paged: the batch row's block table
   size_t base;           // contiguous: (b Hkv + hk) Tcap; paged: hk bt
   size_t stride;         // paged: Hkv bt, the rows of one block
   int shift;             // paged: log2 bt
   __device__ __forceinline__ size_t operator()(int t) const {
-    if (!table) return base + static_cast<size_t>(t);
-    return static_cast<size_t>(__ldg(table + (t >> shift))) * stride + base +
-           static_cast<size_t>(t & ((1 << shift) - 1));
+    if constexpr (!PAGED) return base + static_cast<size_t>(t);
+    else
+      return static_cast<size_t>(__ldg(table + (t >> shift))) * stride + base +
+             static_cast<size_t>(t & ((1 << shift) - 1));
   }
   // rows from t to the end of t's block (contiguous caches: unbounded)
   __device__ __forceinline__ int run(int t) const {
-    return table ? (1 << shift) - (t & ((1 << shift) - 1)) : (1 << 30);
+    if constexpr (!PAGED) return 1 << 30;
+    else return (1 << shift) - (t & ((1 << shift) - 1));
   }
 };
 
-__device__ __forceinline__ RowMap row_map(const DecodeArgs& a, int b, int hk) {
-  RowMap m;
-  if (a.block_table) {
+template <bool PAGED>
+__device__ __forceinline__ RowMap<PAGED> row_map(const DecodeArgs& a, int b, int hk) {
+  RowMap<PAGED> m;
+  if constexpr (PAGED) {
     m.table = a.block_table + static_cast<size_t>(b) * a.max_blocks;
     m.shift = a.block_shift;
     m.base = static_cast<size_t>(hk) << a.block_shift;
@@ -128,7 +133,8 @@ __device__ __forceinline__ void stage_norms(__half* dst, const __half* src, int 
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
 // stage_norms for rows [t0, t0 + n) of one (batch row, KV head) through its row map (blocks hold >= 8 tokens, so an
 // 8-token chunk never straddles two)
-__device__ __forceinline__ void stage_norms_map(__half* dst, const __half* norms, const RowMap& rm, int t0, int n,
+template <class Map>
+__device__ __forceinline__ void stage_norms_map(__half* dst, const __half* norms, const Map& rm, int t0, int n,
                                                 int c) {
   const int tok0 = 8 * c;
   if (c < 16 && tok0 < n) cp_async16_zfill(dst + tok0, norms + rm(t0 + tok0), min(16, 2 * (n - tok0)));
@@ -152,8 +158,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* mbar, uint32_t b
 // Bulk copies of the rows [t0, t0 + n) of one (batch row, KV head), RB bytes each (a multiple of 16), into dst: one
 // copy per run of rows contiguous in global memory (one for a contiguous cache, one per block for a paged pool),
 // all completing on `mbar`, which the caller has armed with the total.
-template <int RB>
-__device__ __forceinline__ void copy_rows_bulk(uint8_t* dst, const uint8_t* src, const RowMap& rm, int t0, int n,
+template <int RB, class Map>
+__device__ __forceinline__ void copy_rows_bulk(uint8_t* dst, const uint8_t* src, const Map& rm, int t0, int n,
                                                uint64_t* mbar) {
   for (int o = 0; o < n;) {
     const int seg = min(n - o, rm.run(t0 + o));
@@ -163,11 +169,11 @@ __device__ __forceinline__ void copy_rows_bulk(uint8_t* dst, const uint8_t* src,
 }
 
 // The same rows as CH-byte cp.async chunks spread over a role's 128 threads (RB a multiple of CH).
-template <int CH, int RB>
-__device__ __forceinline__ void copy_rows_async(uint8_t* dst, const uint8_t* src, const RowMap& rm, int t0, int n,
+template <int CH, int RB, class Map>
+__device__ __forceinline__ void copy_rows_async(uint8_t* dst, const uint8_t* src, const Map& rm, int t0, int n,
                                                 int rtid) {
   const int bytes = n * RB;
-  if (!rm.table) {
+  if (rm.run(t0) >= n) {  // one contiguous run
     const uint8_t* s = src + rm(t0) * RB;
     for (int o = rtid * CH; o < bytes; o += 128 * CH) cp_async<CH>(dst + o, s + o);
   } else {
@@ -667,8 +673,9 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
 }
 
 // Merge of the splits for one (batch, query head) per block, D threads.  With quantized values the merged vector
-// is still in the rotated domain and is mapped back once: out = s .* H(o).
-template <int D, bool VQ>
+// is still in the rotated domain and is mapped back once: out = s .* H(o).  EXACT: the splits' maxima are integers
+// (a log2 domain of integers), and every rescale is the exact power of two 2^(m_s - M).
+template <int D, bool VQ, bool EXACT = false>
 __global__ void __launch_bounds__(D) attend_reduce_kernel(const __grid_constant__ DecodeArgs a) {
   __shared__ float vec[D];
   const int bh = blockIdx.x, j = threadIdx.x;
@@ -682,7 +689,9 @@ __global__ void __launch_bounds__(D) attend_reduce_kernel(const __grid_constant_
   float Ls = 0.f, acc = 0.f;
   if (M != -INFINITY) {
     for (int s = 0; s < a.splits; ++s) {
-      const float w = (m[s] == -INFINITY) ? 0.f : exp2f(m[s] - M);
+      const float w = (m[s] == -INFINITY) ? 0.f
+                      : EXACT             ? ldexpf(1.f, static_cast<int>(m[s] - M))
+                                          : exp2f(m[s] - M);
       Ls = fmaf(w, l[s], Ls);
       acc = fmaf(w, o[static_cast<size_t>(s) * D + j], acc);
     }

@@ -21,7 +21,7 @@ axr_status ensure_smem(K kernel, size_t bytes, const char* what) {
 // decode kernel's blocks retire and wait (griddepcontrol.wait) for that grid's completion and memory flush before
 // reading the partials, so the launch latency overlaps the decode kernel's tail.  Without programmatic launches in
 // the stream (e.g. an older driver) the wait returns at once and ordinary stream order holds.
-template <int D, bool VQ>
+template <int D, bool VQ, bool EXACT = false>
 void launch_reduce(const DecodeArgs& a, cudaStream_t st) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.Hq));
@@ -33,7 +33,7 @@ void launch_reduce(const DecodeArgs& a, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, attend_reduce_kernel<D, VQ>, a);
+  cudaLaunchKernelEx(&cfg, attend_reduce_kernel<D, VQ, EXACT>, a);
 }
 
 // Row-layout cache, one warp per token range through scores, softmax and the value product, all as warp-level MMAs
@@ -52,7 +52,7 @@ axr_status attend_partial_launch(int d, int bits, int G, bool vq, bool dense, co
 // Tiled value layout, d = 128 (attend_tiled.cu): tcgen05 kernel if tensor, else warp-level MMAs.
 axr_status attend_tiled_launch(int bits, int G, bool tensor, const DecodeArgs& a, cudaStream_t st);
 
-// Scores only (score.cu): mode is one of kGatherTable, kGatherFactored, kGatherMma.
+// Scores only (score.cu): mode is one of kGatherFactored, kGatherMma, kGatherDirect (kGatherTable: lut.cu).
 axr_status score_launch(int d, int bits, int G, int mode, const DecodeArgs& a, cudaStream_t st);
 
 // The literal table in shared memory (lut.cu): multi-coordinate fields, G-wide entries; scores, and attend over

@@ -54,7 +54,7 @@ axr_status launch_score(LutArgs a, cudaStream_t st, const char* what) {
 template <int D, int BITS, int W, int NI, int G, int KIND>
 axr_status launch_attend(LutArgs a, float* out, const int8_t* signs, cudaStream_t st, const char* what) {
   using P = LutPlan<D, W, NI, G>;
-  auto k = lut_attend_kernel<D, BITS, W, NI, G, KIND>;
+  auto k = table_attend_kernel<D, G, LutScorer<D, BITS, W, NI, G, KIND>>;
   axr_status rs = lut_smem(k, P::attend_bytes, what);
   if (rs != AXR_OK) return rs;
   const SplitPlan sp = lut_plan(a.B, a.Hkv, a.T, P::attend_bytes);

@@ -13,9 +13,12 @@
 //  * LOOKAT (product quantization with asymmetric distance computation): W = 8 and one field per subspace; entry k
 //    of table i is q^(i) . C_i[k], C_i the subspace's codebook (K <= 256 centroids).
 //
-// Kernels: scores only (lut_score_kernel), and decode attention over fp16 values (lut_attend_kernel: the scores feed
-// a per-warp online softmax and the value product on the CUDA cores; the splits are merged by attend_reduce_kernel).
+// Kernels: scores only (lut_score_kernel), and decode attention over fp16 values (table_attend_kernel with the
+// LutScorer policy: the scores feed a per-warp online softmax and the value product on the CUDA cores; the splits
+// are merged by attend_reduce_kernel).
 #pragma once
+
+#include <type_traits>
 
 #include "decode.cuh"
 
@@ -54,9 +57,8 @@ struct LutPlan {
   static constexpr size_t OFF_QS = TAB;                  // [G][D] row factors
   static constexpr size_t OFF_CENT = OFF_QS + (size_t)G * D * 4;
   static constexpr size_t OFF_MERGE = OFF_CENT + 16 * 4;  // attend: [8 warps][G][D + 2]
-  static constexpr int WARPS = kLutThreads / kWarp;
   static constexpr size_t score_bytes = OFF_MERGE;
-  static constexpr size_t attend_bytes = OFF_MERGE + (size_t)WARPS * G * (D + 2) * 4;
+  static constexpr size_t attend_bytes = OFF_MERGE + (size_t)(kLutThreads / kWarp) * G * (D + 2) * 4;
 };
 
 // Cache row of token t: [B, Hkv, Tcap] numbering.
@@ -236,19 +238,42 @@ __global__ void __launch_bounds__(kLutThreads) lut_score_kernel(const __grid_con
   }
 }
 
-// Decode attention over fp16 values: tiles of 256 tokens, thread t scores token t of the tile; warp w keeps the
-// online softmax of its 32 tokens of every tile (max in log2 units) and the value product over them, each lane
-// holding D / 32 coordinates of every head.  At the end of an item the warps merge into the split's partial.
+// The literal-table scorer as a policy of table_attend_kernel: the item's table is built in shared memory, a token's
+// scores are the gathered entries times its norm (AXELRAM), in log2 units (mult holds scale * log2(e)).
 template <int D, int BITS, int W, int NI, int G, int KIND>
-__global__ void __launch_bounds__(kLutThreads) lut_attend_kernel(const __grid_constant__ LutArgs a) {
+struct LutScorer {
   using P = LutPlan<D, W, NI, G>;
+  static constexpr bool EXACT = false;           // scores are real numbers; rescales through exp2
+  static constexpr size_t SMEM = P::OFF_MERGE;   // bytes before the merge region
+  __device__ static void build(const LutArgs& a, int b, int hk, uint8_t* smem) {
+    lut_build<D, BITS, W, NI, G, KIND>(a, b, hk, smem);
+  }
+  __device__ static void score(const LutArgs& a, const uint8_t* smem, size_t row0, int t, bool valid,
+                               float (&z)[G]) {
+    uint32_t w[P::NW];
+    lut_load_row<P::RB>(a.codes + (row0 + t) * P::RB, w);
+    lut_gather<W, NI, G>(reinterpret_cast<const float*>(smem), w, z);
+    const float n = KIND == kLutAxelram ? (valid ? __half2float(a.norms[row0 + t]) : 0.f) : 1.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) z[h] = valid ? z[h] * n : -INFINITY;
+  }
+};
+
+// Decode attention over fp16 values: tiles of 256 tokens, thread t scores token t of the tile through the scorer S;
+// warp w keeps the online softmax of its 32 tokens of every tile (max in log2 units) and the value product over
+// them, each lane holding D / 32 coordinates of every head.  At the end of an item the warps merge into the split's
+// partial (the layout of attend_reduce_kernel).  With S::EXACT the scores are integers in the log2 domain: every
+// weight and every rescale is an exact power of two (ldexp), never a rounded exponential.
+template <int D, int G, class S>
+__global__ void __launch_bounds__(kLutThreads) table_attend_kernel(const __grid_constant__ LutArgs a) {
   constexpr int DPL = D / kWarp;  // coordinates per lane
+  constexpr int WARPS = kLutThreads / kWarp;
   static_assert(DPL == 2 || DPL == 4, "d = 64 or 128");
   extern __shared__ __align__(16) uint8_t smem[];
-  const float* tab = reinterpret_cast<const float*>(smem);
-  float* merge = reinterpret_cast<float*>(smem + P::OFF_MERGE);  // [warp][G][D + 2]: o, then m, l
+  float* merge = reinterpret_cast<float*>(smem + S::SMEM);  // [warp][G][D + 2]: o, then m, l
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int items = a.B * a.Hkv * a.splits;
+  auto pow2 = [](float x) { return S::EXACT ? ldexpf(1.f, static_cast<int>(x)) : exp2f(x); };
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
     const int split = item % a.splits;
     const int hk = (item / a.splits) % a.Hkv;
@@ -265,12 +290,51 @@ __global__ void __launch_bounds__(kLutThreads) lut_attend_kernel(const __grid_co
       }
       continue;
     }
-    lut_build<D, BITS, W, NI, G, KIND>(a, b, hk, smem);
     const size_t row0 = lut_row(a, b, hk, 0);
-    const uint8_t* rows = a.codes + row0 * P::RB;
-    const __half* nrm = KIND == kLutAxelram ? a.norms + row0 : nullptr;
     const __half* vrow = a.v + row0 * D + lane * DPL;
+    // value rows of the warp's 32 tokens of a tile travel in batches of 8 through two register buffers: each is
+    // refilled as soon as it is consumed, with the tile's next batch or the first batches of the warp's next tile
+    // (which do not wait for that tile's scores), so 16 rows stay in flight
+    using VRaw = typename std::conditional<DPL == 4, uint2, unsigned int>::type;
+    VRaw va[8], vb[8];
+    auto load8 = [&](VRaw (&buf)[8], int wt0, int nw, int k0) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int tok = wt0 + min(k0 + k, nw - 1);
+        buf[k] = __ldg(reinterpret_cast<const VRaw*>(vrow + static_cast<size_t>(tok) * D));
+      }
+    };
     float m_run[G], l_lane[G], o[G][DPL];
+    auto pv8 = [&](const VRaw (&buf)[8], int k0, int nw, const float (&p)[G]) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (k0 + k >= nw) break;
+        float2 vv[DPL / 2];
+        if constexpr (DPL == 4) {
+          const uint2 u = reinterpret_cast<const uint2&>(buf[k]);
+          vv[0] = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+          vv[1] = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+        } else {
+          const unsigned int u = reinterpret_cast<const unsigned int&>(buf[k]);
+          vv[0] = __half22float2(*reinterpret_cast<const __half2*>(&u));
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float pk = __shfl_sync(0xffffffffu, p[h], k0 + k);
+#pragma unroll
+          for (int c = 0; c < DPL / 2; ++c) {
+            o[h][2 * c] = fmaf(pk, vv[c].x, o[h][2 * c]);
+            o[h][2 * c + 1] = fmaf(pk, vv[c].y, o[h][2 * c + 1]);
+          }
+        }
+      }
+    };
+    {
+      const int wt0 = start + warp * kWarp, nw = min(kWarp, end - wt0);
+      if (nw > 0) load8(va, wt0, nw, 0);
+      if (nw > 8) load8(vb, wt0, nw, 8);
+    }
+    S::build(a, b, hk, smem);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       m_run[h] = -INFINITY;
@@ -281,57 +345,36 @@ __global__ void __launch_bounds__(kLutThreads) lut_attend_kernel(const __grid_co
     for (int t0 = start; t0 < end; t0 += kLutThreads) {
       const int t = t0 + tid;
       float z[G];
-      {
-        uint32_t w[P::NW];
-        lut_load_row<P::RB>(rows + static_cast<size_t>(t < end ? t : start) * P::RB, w);
-        lut_gather<W, NI, G>(tab, w, z);
-        const float n = KIND == kLutAxelram ? (t < end ? __half2float(nrm[t]) : 0.f) : 1.f;
-#pragma unroll
-        for (int h = 0; h < G; ++h) z[h] = t < end ? z[h] * n : -INFINITY;
-      }
+      S::score(a, smem, row0, t < end ? t : start, t < end, z);
       float p[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float mx = warp_max(z[h]);
         const float m_new = fmaxf(m_run[h], mx);
-        const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m_run[h] - m_new);
-        p[h] = (z[h] == -INFINITY) ? 0.f : exp2f(z[h] - m_new);
+        // nothing has accumulated while the running max is -inf; otherwise m_new >= m_run is finite
+        const float alpha = (m_run[h] == -INFINITY) ? 0.f : pow2(m_run[h] - m_new);
+        p[h] = (z[h] == -INFINITY) ? 0.f : pow2(z[h] - m_new);
         l_lane[h] = l_lane[h] * alpha + p[h];
         m_run[h] = m_new;
 #pragma unroll
         for (int c = 0; c < DPL; ++c) o[h][c] *= alpha;
       }
-      // the value product over the warp's 32 tokens of this tile, eight rows in flight
-      const int wt0 = t0 + warp * kWarp;
-      const int nw = min(kWarp, end - wt0);
-      for (int k0 = 0; k0 < nw; k0 += 8) {
-        float2 vv[8][DPL / 2];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const int tok = wt0 + min(k0 + k, nw - 1);
-          const __half* src = vrow + static_cast<size_t>(tok) * D;
-          if constexpr (DPL == 4) {
-            const uint2 u = __ldg(reinterpret_cast<const uint2*>(src));
-            vv[k][0] = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
-            vv[k][1] = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
-          } else {
-            const unsigned int u = __ldg(reinterpret_cast<const unsigned int*>(src));
-            vv[k][0] = __half22float2(*reinterpret_cast<const __half2*>(&u));
-          }
-        }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (k0 + k >= nw) break;
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            const float pk = __shfl_sync(0xffffffffu, p[h], k0 + k);
-#pragma unroll
-            for (int c = 0; c < DPL / 2; ++c) {
-              o[h][2 * c] = fmaf(pk, vv[k][c].x, o[h][2 * c]);
-              o[h][2 * c + 1] = fmaf(pk, vv[k][c].y, o[h][2 * c + 1]);
-            }
-          }
-        }
+      // a tile with a successor is full (every warp has 32 tokens); only the last tile can be partial
+      const int wt0 = t0 + warp * kWarp, nw = min(kWarp, end - wt0);
+      const int nx0 = wt0 + kLutThreads, nxw = min(kWarp, end - nx0);
+      if (nw > 0) pv8(va, 0, nw, p);
+      if (nw > 16) load8(va, wt0, nw, 16);
+      else if (nxw > 0) load8(va, nx0, nxw, 0);
+      if (nw > 8) pv8(vb, 8, nw, p);
+      if (nw > 24) load8(vb, wt0, nw, 24);
+      else if (nxw > 8) load8(vb, nx0, nxw, 8);
+      if (nw > 16) {
+        pv8(va, 16, nw, p);
+        if (nxw > 0) load8(va, nx0, nxw, 0);
+      }
+      if (nw > 24) {
+        pv8(vb, 24, nw, p);
+        if (nxw > 8) load8(vb, nx0, nxw, 8);
       }
     }
     // merge the warps: each publishes o, m and its l; then every (head, coordinate) sums the rescaled parts
@@ -348,17 +391,17 @@ __global__ void __launch_bounds__(kLutThreads) lut_attend_kernel(const __grid_co
       const int h = e / D, j = e % D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w2 = 0; w2 < P::WARPS; ++w2) M = fmaxf(M, merge[(w2 * G + h) * (D + 2) + D]);
-      float s = 0.f, ls = 0.f;
+      for (int w2 = 0; w2 < WARPS; ++w2) M = fmaxf(M, merge[(w2 * G + h) * (D + 2) + D]);
+      float sum = 0.f, ls = 0.f;
 #pragma unroll
-      for (int w2 = 0; w2 < P::WARPS; ++w2) {
+      for (int w2 = 0; w2 < WARPS; ++w2) {
         const float* mw = merge + (w2 * G + h) * (D + 2);
-        const float f = (mw[D] == -INFINITY) ? 0.f : exp2f(mw[D] - M);
-        s = fmaf(f, mw[j], s);
+        const float f = (mw[D] == -INFINITY) ? 0.f : pow2(mw[D] - M);
+        sum = fmaf(f, mw[j], sum);
         ls = fmaf(f, mw[D + 1], ls);
       }
       const size_t part = part0 + static_cast<size_t>(h) * a.splits;
-      a.ws_o[part * D + j] = s;
+      a.ws_o[part * D + j] = sum;
       if (j == 0) {
         a.ws_m[part] = M;
         a.ws_l[part] = ls;

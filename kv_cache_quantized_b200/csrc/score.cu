@@ -1,5 +1,6 @@
 // Launchers of the scores-only kernels on CUDA cores and warp-level MMAs (score_kernel in decode.cuh, score_mma.cuh).
 #include "launch.h"
+#include "score_direct.cuh"
 #include "score_mma.cuh"
 
 namespace axr {
@@ -28,9 +29,40 @@ axr_status launch_mma(const DecodeArgs& a, cudaStream_t st) {
   return check_launch("axr_score");
 }
 
+// Chunk of the direct-load scorer's warp items: a multiple of 16 tokens minimising ceil(items / resident warps) x
+// (chunk + per-item setup), so that the last round of items keeps most warps busy.
+int direct_chunk(int B, int Hkv, int T, long resident_warps) {
+  const long units = static_cast<long>(B) * Hkv;
+  long best_chunk = 256;
+  double best = 1e300;
+  for (long chunk = 256; chunk < T + 16; chunk += 16) {
+    const long items = units * ((T + chunk - 1) / chunk);
+    const long rounds = (items + resident_warps - 1) / resident_warps;
+    const double cost = static_cast<double>(rounds) * static_cast<double>(chunk + 96);
+    if (cost < best - 1e-9) {
+      best = cost;
+      best_chunk = chunk;
+    }
+  }
+  return static_cast<int>(best_chunk);
+}
+
+template <int D, int BITS, int G>
+axr_status launch_direct(DecodeArgs a, cudaStream_t st) {
+  using P = DirectPlan<D, BITS, G>;
+  auto k = score_direct_kernel<D, BITS, G>;
+  axr_status rs = ensure_smem(k, P::bytes, "axr_score");
+  if (rs != AXR_OK) return rs;
+  const long blocks = 2L * kSmCount;  // two resident blocks of 8 warps per SM
+  a.chunk = direct_chunk(a.B, a.Hkv, a.T, blocks * P::WARPS);
+  k<<<static_cast<unsigned>(blocks), P::THREADS, P::bytes, st>>>(a);
+  return check_launch("axr_score");
+}
+
 template <int D, int BITS, int G>
 axr_status launch(int mode, const DecodeArgs& a, cudaStream_t st) {
   if (mode == kGatherMma) return launch_mma<D, BITS, G>(a, st);
+  if (mode == kGatherDirect) return launch_direct<D, BITS, G>(a, st);
   if (mode == kGatherTable) return launch_mode<D, BITS, G, kGatherTable>(a, st);
   if (mode == kGatherFactored) return launch_mode<D, BITS, G, kGatherFactored>(a, st);
   return set_error(AXR_EINVAL, "axr_score: gather mode %d", mode);

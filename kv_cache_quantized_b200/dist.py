@@ -76,3 +76,29 @@ def select_signs_sharded(q, k, v, candidates, bits, causal=True, score_fn=None):
         torch.empty(0, dtype=torch.float64, device=candidates.device)
     mse = gather_candidate_mse(local, n)
     return mse, first_argmin(mse)
+
+
+def select_signs_per_layer_sharded(q, k, v, candidates, bits, causal=True, score_fn=None):
+    """One sign vector per layer with the candidates split across ranks: each rank scores its share of candidates
+    on every layer, one all-gather of the [n_layers, share] MSEs per layer row assembles [n_layers, n_cand] on every
+    rank, and each layer picks the first index of its minimum.
+
+    score_fn(q, k, v, candidates_share, bits, causal) -> [n_layers, share] MSEs; the default runs the library's
+    axr_select_signs_per_layer on this rank's GPU.  Returns (mse [n_layers, n_cand] float64, best [n_layers] list).
+    """
+    if score_fn is None:
+        from . import ops
+
+        def score_fn(q_, k_, v_, c_, b_, causal_):
+            return ops.select_signs_per_layer(q_, k_, v_, c_, b_, causal=causal_)[0]
+    rank, size = world()
+    n = candidates.shape[0]
+    lo, hi = shard_range(n, rank, size)
+    n_layers = q.shape[0] if q is not None else None
+    local = score_fn(q, k, v, candidates[lo:hi].contiguous(), bits, causal) if hi > lo else None
+    if local is None:
+        local = torch.empty((n_layers if n_layers is not None else 0, 0), dtype=torch.float64,
+                            device=candidates.device)
+    rows = [gather_candidate_mse(local[layer], n) for layer in range(local.shape[0])]
+    mse = torch.stack(rows) if rows else torch.empty((0, n), dtype=torch.float64)
+    return mse, [first_argmin(mse[layer]) for layer in range(mse.shape[0])]

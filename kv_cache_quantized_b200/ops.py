@@ -178,7 +178,7 @@ def score(q, kcodes, knorms, signs, bits, scale=1.0, seq_lens=None, T=None, out=
 
 
 GATHER_MODES = {"tensor": _abi.GATHER_TENSOR, "factored": _abi.GATHER_FACTORED, "table": _abi.GATHER_TABLE,
-                "mma": _abi.GATHER_MMA}
+                "mma": _abi.GATHER_MMA, "direct": _abi.GATHER_DIRECT}
 
 
 def set_gather(mode: str) -> None:
@@ -538,4 +538,67 @@ def pq_attend_decode(q, codes, codebooks, v, scale=None, seq_lens=None, T=None, 
     st = _abi.lib().axr_pq_attend_decode(_ptr(q), _ptr(codes), _ptr(codebooks), _ptr(v), _ptr(seq_lens), B, Hq, Hkv,
                                          T, Tcap, d, m, K, scale, _ptr(out), _ptr(ws), ws.numel(), _stream())
     _abi.check(st, "axr_pq_attend_decode")
+    return out
+
+
+# ---- power-of-two shift-accumulate keys -------------------------------------------------------------------------------
+
+def pot_row_bytes(d: int, E: int, M: int) -> int:
+    return d * (1 + E + M) // 8
+
+
+def pot_write(x, E, M, codes=None, alpha=None, dst_rows=None):
+    """PoT codes of float16 rows x [..., d]: (codes uint8 [..., d(1+E+M)/8], alpha float16 [...])."""
+    _need_cuda("x", x, torch.float16)
+    d = x.shape[-1]
+    n = x.numel() // d
+    R = pot_row_bytes(d, E, M)
+    if dst_rows is None:
+        codes = torch.empty(x.shape[:-1] + (R,), dtype=torch.uint8, device=x.device) if codes is None else codes
+        alpha = torch.empty(x.shape[:-1], dtype=torch.float16, device=x.device) if alpha is None else alpha
+    else:
+        _need_cuda("dst_rows", dst_rows, torch.int64)
+        if codes is None or alpha is None:
+            raise ValueError("dst_rows needs the destination codes and alpha buffers")
+    _need_cuda("codes", codes, torch.uint8)
+    _need_cuda("alpha", alpha, torch.float16)
+    st = _abi.lib().axr_pot_write(_ptr(x), n, d, E, M, _ptr(dst_rows), _ptr(codes), _ptr(alpha), _stream())
+    _abi.check(st, "axr_pot_write")
+    return codes, alpha
+
+
+def pot_score(q, codes, alpha, E, M, scale=1.0, seq_lens=None, T=None, integers=False):
+    """PoT scores [B, Hq, T] float32 (and, with integers, the exact shift-accumulated int32 sums S as well)."""
+    _need_cuda("q", q, torch.float32)
+    _need_cuda("codes", codes, torch.uint8)
+    _need_cuda("alpha", alpha, torch.float16)
+    B, Hq, d = q.shape
+    _, Hkv, Tcap, _ = codes.shape
+    T = Tcap if T is None else int(T)
+    seq_lens = _lens(seq_lens, B)
+    out = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    S = torch.empty((B, Hq, T), dtype=torch.int32, device=q.device) if integers else None
+    st = _abi.lib().axr_pot_score(_ptr(q), _ptr(codes), _ptr(alpha), _ptr(seq_lens), B, Hq, Hkv, T, Tcap, d, E, M,
+                                  float(scale), _ptr(S), _ptr(out), _stream())
+    _abi.check(st, "axr_pot_score")
+    return (out, S) if integers else out
+
+
+def pot_attend_decode(q, codes, alpha, v, E, M, scale=None, seq_lens=None, T=None, out=None, workspace=None):
+    """Decode attention over PoT keys (integer-log2 weights) and float16 values v [B, Hkv, Tcap, d]."""
+    _need_cuda("q", q, torch.float32)
+    _need_cuda("codes", codes, torch.uint8)
+    _need_cuda("alpha", alpha, torch.float16)
+    _need_cuda("v", v, torch.float16)
+    B, Hq, d = q.shape
+    _, Hkv, Tcap, _ = codes.shape
+    T = Tcap if T is None else int(T)
+    seq_lens = _lens(seq_lens, B)
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.float32, device=q.device)
+    ws = _workspace(attend_workspace_bytes(B, Hq, Hkv, T, d), q.device, workspace)
+    st = _abi.lib().axr_pot_attend_decode(_ptr(q), _ptr(codes), _ptr(alpha), _ptr(v), _ptr(seq_lens), B, Hq, Hkv, T,
+                                          Tcap, d, E, M, scale, _ptr(out), _ptr(ws), ws.numel(), _stream())
+    _abi.check(st, "axr_pot_attend_decode")
     return out

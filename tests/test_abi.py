@@ -199,3 +199,22 @@ def test_paged_argument_errors_host(L):
     step = L.axr_decode_step_paged(FAKE, None, FAKE, FAKE, FAKE, 1, FAKE, FAKE, FAKE, 4, 64, None, 2, 8, 2, 256, 128,
                                    4, FAKE, 0.088, FAKE, FAKE, 1 << 20, None)
     assert step == 1
+
+
+def test_codec_argument_errors_host(L):
+    """LOOKAT and PoT entry points reject bad sizes and formats on the host, before any CUDA call."""
+    assert L.axr_pq_encode(FAKE, 1, 10, 96, 4, 256, FAKE, 1, 1, None, FAKE, None) == 2      # d
+    assert L.axr_pq_encode(FAKE, 1, 10, 128, 3, 256, FAKE, 1, 1, None, FAKE, None) == 2     # m
+    assert L.axr_pq_encode(FAKE, 1, 10, 128, 4, 257, FAKE, 1, 1, None, FAKE, None) == 2     # K
+    assert L.axr_pq_encode(FAKE, 1, 0, 128, 4, 256, None, 1, 1, None, None, None) == 0      # empty
+    assert L.axr_pq_train(FAKE, 1, 10, 128, 4, 256, 3, FAKE, None, 0, None) == 4            # workspace
+    assert L.axr_pq_train_workspace_bytes(128, 4, 256) >= 128 * 256 * 8
+    assert L.axr_pq_score(FAKE, FAKE, FAKE, None, 2, 6, 4, 100, 100, 128, 4, 256, 0.1, FAKE, None) == 1  # Hq % Hkv
+    assert L.axr_pq_attend_decode(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 100, 100, 128, 4, 256, 0.1, FAKE, None, 0,
+                                  None) == 4
+    assert L.axr_pot_write(FAKE, 10, 128, 3, 1, None, FAKE, FAKE, None) == 2  # 5-bit format
+    assert L.axr_pot_write(FAKE, 10, 128, 0, 0, None, FAKE, FAKE, None) == 2
+    assert L.axr_pot_score(FAKE, FAKE, FAKE, None, 2, 8, 2, 100, 100, 128, 3, 0, 0.1, None, None, None) == 1
+    assert L.axr_pot_score(FAKE, FAKE + 8, FAKE, None, 2, 8, 2, 100, 100, 128, 3, 0, 0.1, FAKE, None, None) == 1
+    assert L.axr_pot_attend_decode(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 100, 100, 128, 2, 1, 0.1, FAKE, FAKE, 16,
+                                   None) == 4

@@ -78,3 +78,36 @@ def test_single_process_identity():
     assert D.first_argmin(mse) == 1
     assert torch.equal(D.gather_candidate_mse(mse, 4), mse)
     assert D.max_over_ranks([1.5]) == [1.5]
+
+
+def _fake_score_layers(q, k, v, cands, bits, causal):
+    # per layer a different deterministic stand-in objective of the candidate's signs
+    w = torch.arange(1, cands.shape[1] + 1, dtype=torch.float64)
+    base = (cands.to(torch.float64) @ w) ** 2
+    return torch.stack([base / (1.0 + layer) + (layer * 7.0) % 5 * cands[:, layer % cands.shape[1]].double()
+                        for layer in range(q.shape[0])])
+
+
+def _worker_layers(rank, size, port, n_cand, out_dir):
+    dist.init_process_group("gloo", rank=rank, world_size=size, init_method=f"tcp://127.0.0.1:{port}")
+    try:
+        rng = np.random.default_rng(1)
+        cands = torch.from_numpy(np.where(rng.random((n_cand, 8)) < 0.5, -1, 1).astype(np.int8))
+        q = torch.zeros((3, 1, 1, 1, 8))
+        mse, best = D.select_signs_per_layer_sharded(q, None, None, cands, 2, score_fn=_fake_score_layers)
+        np.save(os.path.join(out_dir, f"l{rank}.npy"), np.concatenate([mse.numpy().ravel(), best]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("n_cand", [5, 200])
+def test_sharded_per_layer_selection_two_ranks(tmp_path, n_cand):
+    size = 2
+    mp.spawn(_worker_layers, args=(size, _port(), n_cand, str(tmp_path)), nprocs=size, join=True)
+    rng = np.random.default_rng(1)
+    cands = torch.from_numpy(np.where(rng.random((n_cand, 8)) < 0.5, -1, 1).astype(np.int8))
+    want = _fake_score_layers(torch.zeros((3, 1, 1, 1, 8)), None, None, cands, 2, True).numpy()
+    for r in range(size):
+        x = np.load(tmp_path / f"l{r}.npy")
+        assert np.array_equal(x[:3 * n_cand].reshape(3, n_cand), want)
+        assert list(x[3 * n_cand:].astype(int)) == [int(np.argmin(want[layer])) for layer in range(3)]

@@ -44,7 +44,7 @@ SMALL += [(128, 3, g, vq) for g in (1, 2, 8) for vq in (False, True)]
 SMALL += [(64, 4, g, False) for g in (1, 2, 8)]
 
 
-SCORE_CASES = [(d, b, g, m) for m in ("tensor", "mma") for d, b, g in sorted({(d, b, g) for d, b, g, _ in SMALL})]
+SCORE_CASES = [(d, b, g, m) for m in ("tensor", "mma", "direct") for d, b, g in sorted({(d, b, g) for d, b, g, _ in SMALL})]
 SCORE_CASES += [(d, b, g, m) for m in ("factored", "table") for d, b, g in [(128, 4, 4), (64, 3, 4), (128, 2, 8),
                                                                              (128, 1, 1)]]
 SCORE_CASES += [(d, b, g, "table") for d, b, g in [(128, 2, 4), (128, 4, 1), (64, 1, 8), (128, 3, 8), (64, 2, 2)]]
