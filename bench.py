@@ -522,6 +522,29 @@ def run_axr(args, w):
                  "frac": dbytes / (ms / 1e3) / 1e9 / _peaks()[0], "algorithmic_bytes": dbytes}
         del kd, vd
 
+    # the same decode step through paged pools (shuffled block tables) at two block sizes
+    paged = None
+    if not args.no_codecs and w.v_quant:
+        paged = {}
+        for bt in (16, 256):
+            nb = T // bt
+            perm = torch.randperm(B * nb, generator=torch.Generator().manual_seed(bt)).to(dev)
+            table = perm.view(B, nb).to(torch.int32).contiguous()
+
+            def pool(x):  # [B, Hkv, T, ...] -> [B * nb, Hkv, bt, ...] with block (b, j) at table[b, j]
+                y = x.view(B, Hkv, nb, bt, *x.shape[3:]).transpose(1, 2).reshape(B * nb, Hkv, bt, *x.shape[3:])
+                out_ = torch.empty_like(y)
+                out_[perm] = y
+                return out_
+            pk, pn, pvc, pvn = pool(kc), pool(kn), pool(vc), pool(vn)
+            ms = time_calls(lambda: ops.decode_step_paged(q, knew, vnew, pk, pn, signs, bits, table, vcodes=pvc,
+                                                          vnorms=pvn, out=out, workspace=wsp))
+            ab = _bytes_per_key_head(w) * B * Hkv * T
+            paged[f"bt{bt}"] = {"ms": ms, "achieved_gbs": ab / (ms / 1e3) / 1e9,
+                                "frac": ab / (ms / 1e3) / 1e9 / _peaks()[0], "algorithmic_bytes": ab}
+            del pk, pn, pvc, pvn
+        paged["contiguous"] = {"ms": float(np.mean(attend_ms))}
+
     # the other codecs through the same reducer, at this shape with fp16 values: LOOKAT product-quantized keys
     # (m = 8 one-byte indices, K = 256) and power-of-two shift-accumulate keys (E = 3, M = 0: 4 bits), scores alone
     # and decode attention; the AXELRAM literal-table read (AXR_GATHER_TABLE) over the same fp16 values beside them
@@ -573,6 +596,8 @@ def run_axr(args, w):
         line["sweep"] = sweep
     if codecs is not None:
         line["codecs"] = codecs
+    if paged is not None:
+        line["paged_decode_step"] = paged
     return line
 
 

@@ -248,12 +248,17 @@ struct LutScorer {
   __device__ static void build(const LutArgs& a, int b, int hk, uint8_t* smem) {
     lut_build<D, BITS, W, NI, G, KIND>(a, b, hk, smem);
   }
-  __device__ static void score(const LutArgs& a, const uint8_t* smem, size_t row0, int t, bool valid,
-                               float (&z)[G]) {
+  struct Row {  // a token's index row and norm, loaded a tile ahead of its scoring
     uint32_t w[P::NW];
-    lut_load_row<P::RB>(a.codes + (row0 + t) * P::RB, w);
-    lut_gather<W, NI, G>(reinterpret_cast<const float*>(smem), w, z);
-    const float n = KIND == kLutAxelram ? (valid ? __half2float(a.norms[row0 + t]) : 0.f) : 1.f;
+    unsigned short n;
+  };
+  __device__ static void load(const LutArgs& a, size_t row0, int t, Row& r) {
+    lut_load_row<P::RB>(a.codes + (row0 + t) * P::RB, r.w);
+    r.n = KIND == kLutAxelram ? __ldg(reinterpret_cast<const unsigned short*>(a.norms) + row0 + t) : 0;
+  }
+  __device__ static void score(const LutArgs& a, const uint8_t* smem, const Row& r, bool valid, float (&z)[G]) {
+    lut_gather<W, NI, G>(reinterpret_cast<const float*>(smem), r.w, z);
+    const float n = KIND == kLutAxelram ? __half2float(__ushort_as_half(r.n)) : 1.f;
 #pragma unroll
     for (int h = 0; h < G; ++h) z[h] = valid ? z[h] * n : -INFINITY;
   }
@@ -334,6 +339,8 @@ __global__ void __launch_bounds__(kLutThreads) table_attend_kernel(const __grid_
       if (nw > 0) load8(va, wt0, nw, 0);
       if (nw > 8) load8(vb, wt0, nw, 8);
     }
+    typename S::Row row;  // this thread's token of the current tile, loaded one tile ahead
+    S::load(a, row0, min(start + tid, end - 1), row);
     S::build(a, b, hk, smem);
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -345,7 +352,8 @@ __global__ void __launch_bounds__(kLutThreads) table_attend_kernel(const __grid_
     for (int t0 = start; t0 < end; t0 += kLutThreads) {
       const int t = t0 + tid;
       float z[G];
-      S::score(a, smem, row0, t < end ? t : start, t < end, z);
+      S::score(a, smem, row, t < end, z);
+      if (t0 + kLutThreads < end) S::load(a, row0, min(t + kLutThreads, end - 1), row);  // the next tile's
       float p[G];
 #pragma unroll
       for (int h = 0; h < G; ++h) {

@@ -93,11 +93,18 @@ struct PotScorer {
     __syncthreads();
   }
 
-  // S[h] = sum_j sigma_j Q[h][j] (2^M + mu_j) 2^(l_j >> M) for the token at row
-  __device__ static void integer_scores(const LutArgs& a, const uint8_t* smem, size_t row, int (&S)[G]) {
-    const int* Qs = reinterpret_cast<const int*>(smem + OFF_Q);
+  struct Row {  // a token's code row and alpha, loaded a tile ahead of its scoring
     uint32_t w[NW];
-    lut_load_row<RB>(a.codes + row * RB, w);
+    unsigned short alpha;
+  };
+  __device__ static void load(const LutArgs& a, size_t row0, int t, Row& r) {
+    lut_load_row<RB>(a.codes + (row0 + t) * RB, r.w);
+    r.alpha = __ldg(reinterpret_cast<const unsigned short*>(a.norms) + row0 + t);
+  }
+
+  // S[h] = sum_j sigma_j Q[h][j] (2^M + mu_j) 2^(l_j >> M) for the token whose code words are w
+  __device__ static void integer_scores(const uint8_t* smem, const uint32_t (&w)[NW], int (&S)[G]) {
+    const int* Qs = reinterpret_cast<const int*>(smem + OFF_Q);
 #pragma unroll
     for (int h = 0; h < G; ++h) S[h] = 0;
 #pragma unroll
@@ -121,12 +128,11 @@ struct PotScorer {
   }
 
   // exponent r_t (integer, as a float) in the log2 domain, -inf for an invalid token
-  __device__ static void score(const LutArgs& a, const uint8_t* smem, size_t row0, int t, bool valid,
-                               float (&z)[G]) {
+  __device__ static void score(const LutArgs& a, const uint8_t* smem, const Row& r, bool valid, float (&z)[G]) {
     const float* cq = reinterpret_cast<const float*>(smem + OFF_C);
     int S[G];
-    integer_scores(a, smem, row0 + t, S);
-    const float al = __half2float(a.norms[row0 + t]);
+    integer_scores(smem, r.w, S);
+    const float al = __half2float(__ushort_as_half(r.alpha));
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       const float c = __fmul_rn(cq[h], al);
@@ -163,8 +169,10 @@ __global__ void __launch_bounds__(kLutThreads) pot_score_kernel(const __grid_con
     const size_t row0 = lut_row(a, b, hk, 0);
     for (int t = start + threadIdx.x; t < vend; t += kLutThreads) {
       int S[G];
-      Sc::integer_scores(a, smem, row0 + t, S);
-      const float al = __half2float(a.norms[row0 + t]);
+      typename Sc::Row r;
+      Sc::load(a, row0, t, r);
+      Sc::integer_scores(smem, r.w, S);
+      const float al = __half2float(__ushort_as_half(r.alpha));
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const size_t o = o0 + static_cast<size_t>(h) * a.T + t;
