@@ -39,11 +39,12 @@ NOMINAL_HBM_GBS = 8000.0  # the HBM bandwidth the target is stated against (abou
 UNIT = "keys·heads/s"
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM traffic (read + write bytes) per launch of the timed decode kernel, from an ncu capture of dram__bytes_read.sum
-# and dram__bytes_write.sum on the same workload at B=4 (half the units), scaled by the units processed.  Valid for
-# the kernel version that capture was taken on; a workload without an entry reports null.
+# DRAM traffic (read + write bytes) per launch of the timed decode kernel: an ncu counters-only capture
+# (dram__bytes_read.sum, dram__bytes_write.sum, three launches) of the same workload at B=4 (half the units) read
+# 138.582 MB and wrote 1.457 MB per launch on average; scaled by the units processed.  Valid for the kernel version
+# that capture was taken on; a workload without an entry reports null.
 TRAFFIC = {
-    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.560768e6 + 3.692800e6),
+    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.581845e6 + 1.457408e6),
 }
 
 WORKLOADS = {
