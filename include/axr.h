@@ -371,7 +371,10 @@ AXR_API size_t axr_select_workspace_bytes(int n_layers, int n_seq, int n_tok, in
  * softmax attention (computed once in fp64) and o_quant the same attention with every key written through
  * axr_write_keys' path with signs s^(c) (values unquantized).  Softmax scale 1/sqrt(d); causal != 0 lets
  * position i see keys 0..i only.
- *   q [dev] [n_layers, n_seq, Hq, n_tok, d] f32;  k, v [dev] [n_layers, n_seq, Hkv, n_tok, d] fp16;
+ *   q [dev] [n_layers, n_seq, Hq, n_tok, d] f32;  k, v [dev] [n_layers, n_seq, Hkv, n_tok, d] fp16 (q and v
+ *   16-byte aligned for d >= 64, where the candidate attention runs on the tensor cores: q and the reconstructed keys
+ *   as hi and lo fp16 planes, three products a step, the weights split the same way against the fp16 values, fp32
+ *   accumulation; d = 8 runs in fp32 on the CUDA cores);
  *   candidates [dev] [n_cand, d] int8 (+-1);  mse_out [dev] out [n_cand] f64;
  *   best_out [dev] out, one int32: the first index of the minimum of mse_out;
  *   workspace [dev] >= axr_select_workspace_bytes(...) bytes, 16-aligned.

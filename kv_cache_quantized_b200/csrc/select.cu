@@ -8,13 +8,15 @@
 //      sign flip, Walsh-Hadamard, threshold count, fp16 norm) and is reconstructed in the original domain,
 //      k^ = s .* H(n16 * c[idx]) -- for a prefill-shaped calibration set this is the cheap direction (one transform
 //      per key instead of one per query), and q . k^ equals the table score exactly up to rounding;
-//   3. fp32 tiled attention with k^, squared error against o_ref accumulated in fp64 per (candidate, layer,
-//      sequence);
+//   3. attention with k^, squared error against o_ref accumulated in fp64 per (candidate, layer, sequence): on the
+//      tensor cores for d = 64 and 128 (select_tc.cuh: hi/lo fp16 planes of q and k^, three products per step, fp32
+//      accumulation), on the CUDA cores in fp32 for d = 8;
 //   4. mse = sum / count, best = first index of the minimum: over every layer (one sign vector for the model), or
 //      per layer (one sign vector per layer, axr_select_signs_per_layer).
 #include <cmath>
 
 #include "axr_host.h"
+#include "select_tc.cuh"
 
 namespace axr {
 namespace {
@@ -28,7 +30,7 @@ struct SelArgs {
   const __half* v;      // [Ly, S, Hkv, N, D]
   const int8_t* cand;   // [C, D]
   double* oref;         // [Ly, S, Hq, N, D]
-  float* khat;          // [chunk, Ly, S, Hkv, N, D]
+  float* khat;          // [chunk, Ly, S, Hkv, N, D] f32 (d = 8), or the hi then lo fp16 planes of it (d >= 64)
   double* acc;          // [C, Ly, S] squared-error sums
   double* mse;          // [C], or [Ly, C] per layer
   int32_t* best;        // [1], or [Ly] per layer
@@ -42,7 +44,7 @@ struct SelArgs {
 
 // ---- step 2: write path + reconstruction, one warp per key row ----------------------------------------------------
 
-template <int D, int BITS>
+template <int D, int BITS, bool PLANES>
 __global__ void __launch_bounds__(256) requantize_kernel(const __grid_constant__ SelArgs a) {
   constexpr int VPL = WarpVec<D>::VPL;
   constexpr int LANES = WarpVec<D>::LANES;
@@ -80,8 +82,20 @@ __global__ void __launch_bounds__(256) requantize_kernel(const __grid_constant__
     }
     fwht_warp<D>(v, lane);
     if (active) {
+      if constexpr (PLANES) {  // hi and lo fp16 planes for the tensor-core attention
+        __half* kh = reinterpret_cast<__half*>(a.khat);
+        __half* kl = kh + total * D;
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) a.khat[r * D + lane * VPL + i] = v[i] * nrm * sg[i];
+        for (int i = 0; i < VPL; ++i) {
+          const float x = v[i] * nrm * sg[i];
+          const __half hi = __float2half_rn(x);
+          kh[r * D + lane * VPL + i] = hi;
+          kl[r * D + lane * VPL + i] = __float2half_rn(x - __half2float(hi));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < VPL; ++i) a.khat[r * D + lane * VPL + i] = v[i] * nrm * sg[i];
+      }
     }
   }
 }
@@ -311,6 +325,10 @@ axr_status run_select(SelArgs a, int per_layer, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kref, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RC::smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(kq, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)FC::smem);
   if (e != cudaSuccess) return set_error(AXR_ECUDA, "axr_select_signs: %s", cudaGetErrorString(e));
+  if (e == cudaSuccess && D >= 64)
+    e = cudaFuncSetAttribute(select_attn_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SelTcPlan<D>::bytes);
+  if (e != cudaSuccess) return set_error(AXR_ECUDA, "axr_select_signs: %s", cudaGetErrorString(e));
   e = cudaMemsetAsync(a.acc, 0, sizeof(double) * a.C * a.Ly * a.S, st);
   if (e != cudaSuccess) return set_error(AXR_ECUDA, "axr_select_signs: %s", cudaGetErrorString(e));
   const int qtiles = (a.N + RC::BQ - 1) / RC::BQ;
@@ -326,8 +344,17 @@ axr_status run_select(SelArgs a, int per_layer, cudaStream_t st) {
     size_t warps = rows * a.nc;
     size_t blocks = (warps + 7) / 8;
     if (blocks > static_cast<size_t>(kSmCount) * 32) blocks = static_cast<size_t>(kSmCount) * 32;
-    requantize_kernel<D, BITS><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
-    kq<<<dim3(qtiles, a.Hq, a.Ly * a.S * a.nc), kSelThreads, FC::smem, st>>>(a);
+    if constexpr (D >= 64) {
+      requantize_kernel<D, BITS, true><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
+      const __half* kh = reinterpret_cast<const __half*>(a.khat);
+      const __half* kl = kh + rows * a.nc * D;
+      select_attn_tc_kernel<D><<<dim3(qtiles, a.Hq, a.Ly * a.S * a.nc), SelTcPlan<D>::THREADS,
+                                  SelTcPlan<D>::bytes, st>>>(a.q, kh, kl, a.v, a.oref, a.acc, a.Ly, a.S, a.Hq,
+                                                             a.Hkv, a.N, a.c0, a.causal);
+    } else {
+      requantize_kernel<D, BITS, false><<<static_cast<unsigned>(blocks), 256, 0, st>>>(a);
+      kq<<<dim3(qtiles, a.Hq, a.Ly * a.S * a.nc), kSelThreads, FC::smem, st>>>(a);
+    }
     rs = check_launch("axr_select_signs (candidates)");
     if (rs != AXR_OK) return rs;
   }
@@ -357,8 +384,8 @@ axr_status select_impl(const char* w, const float* q, const uint16_t* k, const u
   if (d != 8 && d != 64 && d != 128) return set_error(AXR_EUNSUPPORTED, "%s: d=%d not in {8,64,128}", w, d);
   if (bits < 1 || bits > 4) return set_error(AXR_EUNSUPPORTED, "%s: bits=%d outside 1..4", w, bits);
   if (!q || !k || !v || !candidates || !mse_out || !best_out) return set_error(AXR_EINVAL, "%s: null pointer", w);
-  if (!aligned(q, 4) || !aligned(k, 2) || !aligned(v, 2) || !aligned(mse_out, 8) || !aligned(best_out, 4) ||
-      (parts_out && !aligned(parts_out, 8)))
+  if (!aligned(q, d >= 64 ? 16 : 4) || !aligned(k, 2) || !aligned(v, d >= 64 ? 16 : 2) || !aligned(mse_out, 8) ||
+      !aligned(best_out, 4) || (parts_out && !aligned(parts_out, 8)))
     return set_error(AXR_EINVAL, "%s: misaligned pointer", w);
   const SelLayout L = sel_layout(n_layers, n_seq, n_tok, Hq, Hkv, d, n_cand);
   if (!workspace || ws_bytes < L.total)

@@ -42,4 +42,7 @@ def test_algorithmic_bytes_per_key_head():
     w = W.LONG_CONTEXT
     units = w.B * w.Hkv * w.T
     assert units * bench._bytes_per_key_head(w) == 276_824_064
-    assert np.isclose(bench.TRAFFIC[w.name] / (units * bench._bytes_per_key_head(w)), 1.028, atol=0.01)
+    # the measured DRAM traffic of the decode kernel is the algorithmic bytes plus the partials and the new tokens'
+    # writes: at least the algorithmic bytes, and no re-reads beyond a percent or two
+    ratio = bench.TRAFFIC[w.name] / (units * bench._bytes_per_key_head(w))
+    assert 1.0 <= ratio <= 1.02, ratio
