@@ -509,7 +509,31 @@ def run_axr(args, w):
                             "achieved_gbs_codes_norms": cbytes / (ms / 1e3) / 1e9,
                             "algorithmic_bytes_codes_norms": cbytes}
         ops.set_gather("mma")
-        del sc_out
+        # the literal table where byte-indexed multi-coordinate tables apply (b <= 2: 8 or 4 coordinates per
+        # 8-bit field), against the factored MMA read of the same codes, at this shape
+        klow = _gen_rows(W.lognormal_rows_device, (B, Hkv, T, d), seed + 21, dev)
+        for lb in (1, 2):
+            lc, ln = ops.write_keys(klow, signs, lb)
+            for mode in ("mma", "table"):
+                ops.set_gather(mode)
+                for _ in range(3):
+                    ops.score(q, lc, ln, signs, lb, scale=1.0 / math.sqrt(d), out=sc_out)
+                evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                       for _ in range(args.steps)]
+                for a_, b2 in evs:
+                    flush.zero_()
+                    a_.record(stream)
+                    ops.score(q, lc, ln, signs, lb, scale=1.0 / math.sqrt(d), out=sc_out)
+                    b2.record(stream)
+                torch.cuda.synchronize()
+                ms = float(np.mean([a_.elapsed_time(b2) for a_, b2 in evs]))
+                sbytes = (d * lb // 8 + 2 + 4 * w.G) * B * Hkv * T
+                scorer[f"{mode}_b{lb}"] = {"ms": ms, "achieved_gbs": sbytes / (ms / 1e3) / 1e9, "algorithmic_bytes": sbytes,
+                                           "achieved_gbs_codes_norms": (d * lb // 8 + 2) * B * Hkv * T / (ms / 1e3) / 1e9,
+                                           "algorithmic_bytes_codes_norms": (d * lb // 8 + 2) * B * Hkv * T}
+            del lc, ln
+        ops.set_gather("mma")
+        del sc_out, klow
 
     # the build's own dense fp16 decode kernel on the same shape (fp16 K and V), the bandwidth reference
     dense = None
@@ -637,6 +661,9 @@ def run_select(args):
     import torch
     from kv_cache_quantized_b200 import ops
     c = W.QWEN3B_SELECT
+    if args.batch is not None:  # fewer layers (small ncu cases)
+        import dataclasses
+        c = dataclasses.replace(c, layers=args.batch, name=c.name.replace("_l36_", f"_l{args.batch}_"))
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     shape_q = (c.layers, c.seqs, c.Hq, c.tokens, c.d)
@@ -738,7 +765,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["select"], default="long_context")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU time budget of the oracle baseline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch size (small ncu cases)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size, or the selector's layer count (small ncu cases)")
     ap.add_argument("--no-scorer", action="store_true", help="skip the separate axr_score measurement")
     ap.add_argument("--variants", action="store_true",
                     help="also time the attend over the tiled value layout (MMA and tcgen05 value products)")
