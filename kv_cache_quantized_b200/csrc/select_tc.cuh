@@ -9,27 +9,36 @@
 // with fp32 accumulation, the online softmax in fp32 (FA2 order: rows held by quads of lanes) and the squared error
 // against the fp64 reference summed in fp64.
 //
-// Block: 4 warps, 16 query rows each (64 rows); key tiles of 64.  Q (hi, lo), K^ (hi, lo) and V tiles sit in shared
-// memory with rows padded by 16 bytes, so the ldmatrix reads of 8 rows fall in 8 different 16-byte bank groups.
+// Block: 4 warps, 16 query rows each (64 rows); key tiles of 32, double-buffered: the cp.async copies of tile k + 1
+// are in flight while tile k is computed.  Q (hi, lo), K^ (hi, lo) and V tiles sit in shared memory with rows padded
+// by 16 bytes, so the ldmatrix reads of 8 rows fall in 8 different 16-byte bank groups.
 #pragma once
 
 #include "axr_common.cuh"
 
 namespace axr {
 
-template <int D>
-struct SelTcPlan {
-  static constexpr int BQ = 64, BK = 64, WARPS = 4, THREADS = 32 * WARPS;
-  static constexpr int RS = D * 2 + 16;                // padded row stride in bytes (fp16 rows)
-  static constexpr size_t TILE = (size_t)BQ * RS;      // one 64-row tile
-  static constexpr size_t OFF_QH = 0, OFF_QL = TILE, OFF_KH = 2 * TILE, OFF_KL = 3 * TILE, OFF_V = 4 * TILE;
-  static constexpr size_t bytes = 5 * TILE;
-  static constexpr int KT = D / 16;                    // k-tiles of the score MMA
-  static constexpr int NO = D / 8;                     // n-tiles of the output
-};
-
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+template <int D>
+struct SelTcPlan {
+  static constexpr int BQ = 64, BK = 32, WARPS = 4, THREADS = 32 * WARPS;
+  static constexpr int RS = D * 2 + 16;                // padded row stride in bytes (fp16 rows)
+  static constexpr size_t QTILE = (size_t)BQ * RS;     // the 64-row query tile (one plane)
+  static constexpr size_t KTILE = (size_t)BK * RS;     // a 32-row key or value tile (one plane)
+  static constexpr size_t STAGE = 3 * KTILE;           // K^ hi, K^ lo, V
+  static constexpr size_t OFF_QH = 0, OFF_QL = QTILE, OFF_ST = 2 * QTILE;  // [2] stages follow the queries
+  static constexpr size_t bytes = 2 * QTILE + 2 * STAGE;
+  static constexpr int KT = D / 16;                    // k-tiles of the score MMA
+  static constexpr int NO = D / 8;                     // n-tiles of the output
+  static constexpr int NS = BK / 8;                    // n-tiles of the scores (keys)
+};
+
+// 16-byte global -> shared copy; src_bytes = 0 fills the destination with zeros
+__device__ __forceinline__ void cp16(void* dst, const void* src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes));
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -75,6 +84,7 @@ select_attn_tc_kernel(const float* __restrict__ q, const __half* __restrict__ kh
                       int Ly, int S, int Hq, int Hkv, int N, int c0, int causal) {
   using P = SelTcPlan<D>;
   constexpr int BQ = P::BQ, BK = P::BK, RS = P::RS, KT = P::KT, NO = P::NO;
+  static_assert(BK % 16 == 0, "key tiles of whole 16-key MMA steps");
   extern __shared__ __align__(16) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
@@ -108,8 +118,6 @@ select_attn_tc_kernel(const float* __restrict__ q, const __half* __restrict__ kh
   const int b_row = 8 * (lane >> 4) + (lane & 7), b_col = ((lane >> 3) & 1) * 8;
   const int v_row = 8 * ((lane >> 3) & 1) + (lane & 7), v_col = (lane >> 4) * 8;
   const uint32_t sQH = smem_addr(smem + P::OFF_QH), sQL = smem_addr(smem + P::OFF_QL);
-  const uint32_t sKH = smem_addr(smem + P::OFF_KH), sKL = smem_addr(smem + P::OFF_KL);
-  const uint32_t sV = smem_addr(smem + P::OFF_V);
 
   float o[NO][4];
 #pragma unroll
@@ -120,27 +128,36 @@ select_attn_tc_kernel(const float* __restrict__ q, const __half* __restrict__ kh
   const int row_lo = q0 + 16 * warp + g, row_hi = row_lo + 8;
 
   const int kend = causal ? min(N, q0 + BQ) : N;
-  for (int k0 = 0; k0 < kend; k0 += BK) {
-    __syncthreads();  // the previous tiles are consumed (and, the first time, the Q tile is written)
-    for (int e = tid; e < BK * D / 8; e += P::THREADS) {  // 16-byte chunks of K^ hi, lo and V rows
-      const int r = e / (D / 8), c8 = e % (D / 8);
-      uint4 xh = make_uint4(0u, 0u, 0u, 0u), xl = xh, xv = xh;
-      if (k0 + r < N) {
-        const size_t off = (krow0 + k0 + r) * D + 8 * c8;
-        xh = *reinterpret_cast<const uint4*>(kh + kcand * D + off);
-        xl = *reinterpret_cast<const uint4*>(kl + kcand * D + off);
-        xv = *reinterpret_cast<const uint4*>(v + off);
+  const int ntiles = (kend + BK - 1) / BK;
+  // cp.async copies of key tile `kt` (rows past N zero-filled) into stage kt % 2; one commit group per tile
+  auto issue = [&](int kt) {
+    if (kt < ntiles) {
+      uint8_t* st = smem + P::OFF_ST + static_cast<size_t>(kt & 1) * P::STAGE;
+      for (int e = tid; e < BK * D / 8; e += P::THREADS) {
+        const int r = e / (D / 8), c8 = e % (D / 8);
+        const int row = min(kt * BK + r, N - 1);
+        const int nb = kt * BK + r < N ? 16 : 0;
+        const size_t off = (krow0 + row) * D + 8 * c8;
+        cp16(st + r * RS + 16 * c8, kh + kcand * D + off, nb);
+        cp16(st + P::KTILE + r * RS + 16 * c8, kl + kcand * D + off, nb);
+        cp16(st + 2 * P::KTILE + r * RS + 16 * c8, v + off, nb);
       }
-      *reinterpret_cast<uint4*>(smem + P::OFF_KH + r * RS + 16 * c8) = xh;
-      *reinterpret_cast<uint4*>(smem + P::OFF_KL + r * RS + 16 * c8) = xl;
-      *reinterpret_cast<uint4*>(smem + P::OFF_V + r * RS + 16 * c8) = xv;
     }
-    __syncthreads();
+    asm volatile("cp.async.commit_group;\n" ::);
+  };
+  issue(0);
+  for (int kt = 0; kt < ntiles; ++kt) {
+    const int k0 = kt * BK;
+    issue(kt + 1);
+    asm volatile("cp.async.wait_group 1;\n" ::);  // tile kt has landed (tile kt + 1 may be in flight)
+    __syncthreads();  // ... for every thread's copies; and, the first time, the Q tile is written
+    const uint32_t sKH = smem_addr(smem + P::OFF_ST + static_cast<size_t>(kt & 1) * P::STAGE);
+    const uint32_t sKL = sKH + P::KTILE, sV = sKH + 2 * P::KTILE;
 
-    // ---- S = Q K^T for the warp's 16 rows x 64 keys (8 n-tiles), three products per step
-    float s[8][4];
+    // ---- S = Q K^T for the warp's 16 rows x 32 keys (4 n-tiles), three products per step
+    float s[P::NS][4];
 #pragma unroll
-    for (int n = 0; n < 8; ++n)
+    for (int n = 0; n < P::NS; ++n)
 #pragma unroll
       for (int i = 0; i < 4; ++i) s[n][i] = 0.f;
 #pragma unroll
@@ -150,7 +167,7 @@ select_attn_tc_kernel(const float* __restrict__ q, const __half* __restrict__ kh
       ldsm_x4(sQH + aoff, ah[0], ah[1], ah[2], ah[3]);
       ldsm_x4(sQL + aoff, al[0], al[1], al[2], al[3]);
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {  // pairs of n-tiles (16 keys)
+      for (int np = 0; np < P::NS / 2; ++np) {  // pairs of n-tiles (16 keys)
         uint32_t bh[4], bl[4];
         const uint32_t boff = (16 * np + b_row) * RS + (16 * kk + b_col) * 2;
         ldsm_x4(sKH + boff, bh[0], bh[1], bh[2], bh[3]);
@@ -168,7 +185,7 @@ select_attn_tc_kernel(const float* __restrict__ q, const __half* __restrict__ kh
     // ---- online softmax (log2 units): lane (g, t) holds rows g, g + 8, keys 8 n + 2 t + {0, 1}
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-    for (int n = 0; n < 8; ++n)
+    for (int n = 0; n < P::NS; ++n)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int key = k0 + 8 * n + 2 * t + (i & 1);
@@ -188,7 +205,7 @@ select_attn_tc_kernel(const float* __restrict__ q, const __half* __restrict__ kh
     }
     float rs[2] = {0.f, 0.f};
 #pragma unroll
-    for (int n = 0; n < 8; ++n)
+    for (int n = 0; n < P::NS; ++n)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float mm = m_run[i >> 1];
@@ -207,18 +224,18 @@ select_attn_tc_kernel(const float* __restrict__ q, const __half* __restrict__ kh
       o[n][0] *= alpha[0]; o[n][1] *= alpha[0]; o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
     }
 
-    // ---- O += P V: P from the score accumulators (keys 16 kt + {0..15}), split hi / lo; V by ldmatrix.trans
+    // ---- O += P V: P from the score accumulators (keys 16 kq + {0..15}), split hi / lo; V by ldmatrix.trans
 #pragma unroll
-    for (int kt = 0; kt < 4; ++kt) {
+    for (int kq = 0; kq < BK / 16; ++kq) {
       uint32_t ph[4], pl[4];
-      split_h2(s[2 * kt][0], s[2 * kt][1], ph[0], pl[0]);
-      split_h2(s[2 * kt][2], s[2 * kt][3], ph[1], pl[1]);
-      split_h2(s[2 * kt + 1][0], s[2 * kt + 1][1], ph[2], pl[2]);
-      split_h2(s[2 * kt + 1][2], s[2 * kt + 1][3], ph[3], pl[3]);
+      split_h2(s[2 * kq][0], s[2 * kq][1], ph[0], pl[0]);
+      split_h2(s[2 * kq][2], s[2 * kq][3], ph[1], pl[1]);
+      split_h2(s[2 * kq + 1][0], s[2 * kq + 1][1], ph[2], pl[2]);
+      split_h2(s[2 * kq + 1][2], s[2 * kq + 1][3], ph[3], pl[3]);
 #pragma unroll
       for (int np = 0; np < NO / 2; ++np) {  // pairs of output n-tiles (16 coordinates)
         uint32_t b[4];
-        ldsm_x4_t(sV + (16 * kt + v_row) * RS + (16 * np + v_col) * 2, b[0], b[1], b[2], b[3]);
+        ldsm_x4_t(sV + (16 * kq + v_row) * RS + (16 * np + v_col) * 2, b[0], b[1], b[2], b[3]);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
           mma16816(o[2 * np + j], ph[0], ph[1], ph[2], ph[3], b[2 * j], b[2 * j + 1]);
@@ -226,7 +243,9 @@ select_attn_tc_kernel(const float* __restrict__ q, const __half* __restrict__ kh
         }
       }
     }
+    __syncthreads();  // every warp is done with this stage before tile kt + 2 is copied into it
   }
+  asm volatile("cp.async.wait_group 0;\n" ::);
 
   // ---- squared error against the fp64 reference: lane (g, t) holds rows g, g + 8, coordinates 8 n + 2 t + {0, 1}
   double err = 0.0;
