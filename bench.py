@@ -542,7 +542,7 @@ def run_axr(args, w):
         vd = _gen_rows(W.normal_device, (B, Hkv, T, d), seed + 8, dev)
         ms = time_calls(lambda: ops.dense_decode(q, kd, vd, out=out, workspace=wsp))
         dbytes = 4 * d * B * Hkv * T
-        dense = {"kernel": "attend_partial_kernel<DENSE> + attend_reduce_kernel (axr_dense_decode)", "ms": ms,
+        dense = {"kernel": "dense_stream_kernel + attend_reduce_kernel (axr_dense_decode)", "ms": ms,
                  "value": B * T * Hq / (ms / 1e3), "unit": UNIT, "achieved_gbs": dbytes / (ms / 1e3) / 1e9,
                  "frac": dbytes / (ms / 1e3) / 1e9 / _peaks()[0], "algorithmic_bytes": dbytes}
         del kd, vd

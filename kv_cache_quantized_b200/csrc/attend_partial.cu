@@ -1,14 +1,14 @@
 // Launcher of the CUDA-core row-layout decode kernel (attend_partial_kernel in decode.cuh): quantized keys through
-// the factored gather, or fp16 keys for the dense bandwidth reference.
+// the factored gather.
 #include "launch.h"
 
 namespace axr {
 namespace {
 
-template <int D, int BITS, int G, bool VQ, bool DENSE>
+template <int D, int BITS, int G, bool VQ>
 axr_status launch(const DecodeArgs& a, cudaStream_t st, const char* what) {
-  using S = DecPlan<D, BITS, G, VQ, DENSE>;
-  auto k1 = attend_partial_kernel<D, BITS, G, VQ, DENSE>;
+  using S = DecPlan<D, BITS, G, VQ>;
+  auto k1 = attend_partial_kernel<D, BITS, G, VQ>;
   axr_status rs = ensure_smem(k1, S::bytes, what);
   if (rs != AXR_OK) return rs;
   const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // persistent blocks loop over the items
@@ -22,10 +22,10 @@ axr_status launch(const DecodeArgs& a, cudaStream_t st, const char* what) {
 template <int D, int BITS>
 axr_status by_g(int G, bool vq, const DecodeArgs& a, cudaStream_t st, const char* w) {
   switch (G) {
-    case 1: return vq ? launch<D, BITS, 1, true, false>(a, st, w) : launch<D, BITS, 1, false, false>(a, st, w);
-    case 2: return vq ? launch<D, BITS, 2, true, false>(a, st, w) : launch<D, BITS, 2, false, false>(a, st, w);
-    case 4: return vq ? launch<D, BITS, 4, true, false>(a, st, w) : launch<D, BITS, 4, false, false>(a, st, w);
-    case 8: return vq ? launch<D, BITS, 8, true, false>(a, st, w) : launch<D, BITS, 8, false, false>(a, st, w);
+    case 1: return vq ? launch<D, BITS, 1, true>(a, st, w) : launch<D, BITS, 1, false>(a, st, w);
+    case 2: return vq ? launch<D, BITS, 2, true>(a, st, w) : launch<D, BITS, 2, false>(a, st, w);
+    case 4: return vq ? launch<D, BITS, 4, true>(a, st, w) : launch<D, BITS, 4, false>(a, st, w);
+    case 8: return vq ? launch<D, BITS, 8, true>(a, st, w) : launch<D, BITS, 8, false>(a, st, w);
   }
   return set_error(AXR_EUNSUPPORTED, "%s: G=%d", w, G);
 }
@@ -41,23 +41,11 @@ axr_status by_bits(int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t s
   return set_error(AXR_EUNSUPPORTED, "%s: bits=%d", w, bits);
 }
 
-template <int D>
-axr_status dense_g(int G, const DecodeArgs& a, cudaStream_t st, const char* w) {
-  switch (G) {
-    case 1: return launch<D, 1, 1, false, true>(a, st, w);
-    case 2: return launch<D, 1, 2, false, true>(a, st, w);
-    case 4: return launch<D, 1, 4, false, true>(a, st, w);
-    case 8: return launch<D, 1, 8, false, true>(a, st, w);
-  }
-  return set_error(AXR_EUNSUPPORTED, "%s: G=%d", w, G);
-}
-
 }  // namespace
 
-axr_status attend_partial_launch(int d, int bits, int G, bool vq, bool dense, const DecodeArgs& a, cudaStream_t st,
+axr_status attend_partial_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st,
                                  const char* what) {
   if (d != 64 && d != 128) return set_error(AXR_EUNSUPPORTED, "%s: d=%d", what, d);
-  if (dense) return d == 64 ? dense_g<64>(G, a, st, what) : dense_g<128>(G, a, st, what);
   return d == 64 ? by_bits<64>(bits, G, vq, a, st, what) : by_bits<128>(bits, G, vq, a, st, what);
 }
 

@@ -152,7 +152,7 @@ axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, con
     if (!vq && attend_fused_supported(d, bits)) return attend_fused_launch(d, bits, G, vq, a, as_stream(stream));
     return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));
   }
-  return attend_partial_launch(d, bits, G, vq, false, a, as_stream(stream), w);
+  return attend_partial_launch(d, bits, G, vq, a, as_stream(stream), w);
 }
 }  // namespace
 
@@ -218,11 +218,12 @@ extern "C" axr_status axr_dense_decode(const float* q, const uint16_t* k, const 
     return e == cudaSuccess ? set_error(AXR_OK, "") : set_error(AXR_ECUDA, "%s: %s", w, cudaGetErrorString(e));
   }
   DecodeArgs a = base_args(B, Hq, Hkv, T, Tcap, seq_lens, q, scale * kLog2e);
+  const SplitPlan p = plan_splits_dense(B, Hkv, T);
+  a.splits = p.splits; a.chunk = p.chunk;
   st = carve_workspace(a, d, workspace, ws_bytes, w);
   if (st != AXR_OK) return st;
   a.kdense = reinterpret_cast<const __half*>(k); a.v = v; a.out = out;
-  const int G = Hq / Hkv;
-  return attend_partial_launch(d, 1, G, false, true, a, as_stream(stream), w);
+  return dense_launch(d, Hq / Hkv, a, as_stream(stream), w);
 }
 
 extern "C" axr_status axr_set_gather(axr_gather mode) {

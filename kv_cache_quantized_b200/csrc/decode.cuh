@@ -32,7 +32,7 @@ struct DecodeArgs {
   const float* q;            // [B, Hq, D]
   const uint8_t* kcodes;     // [B, Hkv, Tcap, R]
   const __half* knorms;      // [B, Hkv, Tcap]
-  const __half* kdense;      // [B, Hkv, Tcap, D] (dense reference only)
+  const __half* kdense;      // [B, Hkv, Tcap, D] fp16 keys (the dense kernel only)
   const void* v;             // fp16 [B, Hkv, Tcap, D] or codes [B, Hkv, Tcap, R]
   const __half* vnorms;      // [B, Hkv, Tcap] (quantized V)
   const int32_t* seq_lens;   // [B] or null
@@ -322,7 +322,7 @@ constexpr int kTT = 128;     // tokens per tile of the scorer
 constexpr int kStages = 3;   // cp.async pipeline depth (two tiles in flight while one is processed)
 constexpr int kDecReps = 16; // pair-table copies in the decode kernel
 
-template <int D, int BITS, int G, bool VQ, bool DENSE>
+template <int D, int BITS, int G, bool VQ>
 struct DecPlan {
   static constexpr int TT = 128;                          // tokens per tile
   static constexpr int KW = 4;                            // scoring warps; value warps follow them
@@ -330,7 +330,7 @@ struct DecPlan {
   static constexpr int WT = TT / KW;                      // tokens per scoring warp per tile
   static constexpr int L = 1 << BITS;
   static constexpr int R = D * BITS / 8;
-  static constexpr int KROW = DENSE ? 2 * D : R;          // bytes per key row
+  static constexpr int KROW = R;                          // bytes per key row
   static constexpr int VROW = VQ ? R : 2 * D;             // bytes per value row
   static constexpr int KCH = (KROW % 16 == 0) ? 16 : 8;   // cp.async chunk sizes
   static constexpr int VCH = (VROW % 16 == 0) ? 16 : 8;
@@ -342,7 +342,7 @@ struct DecPlan {
   static constexpr int TPR = D / 8;                       // value lanes per token row (8 coordinates each)
   static constexpr int RPW = kWarp / TPR;                 // value rows per warp step
   static constexpr int NVG = KW * RPW;                    // value lane groups, summed at the end
-  static constexpr int TAB = DENSE ? 0 : PairTable<BITS, kDecReps>::FLOATS;
+  static constexpr int TAB = PairTable<BITS, kDecReps>::FLOATS;
   static constexpr size_t OFF_K = 0;                                         // [kStages][STAGE_K]
   static constexpr size_t OFF_V = OFF_K + kStages * (size_t)STAGE_K;         // [kStages][STAGE_V]
   static constexpr size_t STAGES_END = OFF_V + kStages * (size_t)STAGE_V;
@@ -367,10 +367,10 @@ __device__ __forceinline__ void role_copy_async(uint8_t* dst, const uint8_t* src
   for (int o = rtid * CH; o < bytes; o += 128 * CH) cp_async<CH>(dst + o, src + o);
 }
 
-template <int D, int BITS, int G, bool VQ, bool DENSE>
-__global__ void __launch_bounds__(kDecThreads, DecPlan<D, BITS, G, VQ, DENSE>::MIN_BLOCKS)
+template <int D, int BITS, int G, bool VQ>
+__global__ void __launch_bounds__(kDecThreads, DecPlan<D, BITS, G, VQ>::MIN_BLOCKS)
 attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
-  using P = DecPlan<D, BITS, G, VQ, DENSE>;
+  using P = DecPlan<D, BITS, G, VQ>;
   constexpr int J = P::J, HG = P::HG, TT = P::TT, WT = P::WT, KW = P::KW, RPW = P::RPW, TPR = P::TPR;
   extern __shared__ __align__(16) uint8_t smem[];
   float* tab = reinterpret_cast<float*>(smem + P::OFF_TAB);
@@ -389,7 +389,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
 
   if (tid < 16) cent[tid] = a.cb.c[tid];
   __syncthreads();
-  if constexpr (!DENSE) build_pair_table<BITS, kDecReps>(cent, tab);
+  build_pair_table<BITS, kDecReps>(cent, tab);
 
   const int items = a.B * a.Hkv * a.splits;
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
@@ -404,11 +404,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
     const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
 
     __syncthreads();  // the previous item is finished with the row factors, the stages and the merge region
-    if constexpr (DENSE) {
-      for (int e = tid; e < G * D; e += kDecThreads) qs[e] = qg[e] * a.mult;  // fp16 keys: untransformed query
-    } else {
-      transform_queries<D, G>(qg, a.signs, a.mult, qs);
-    }
+    transform_queries<D, G>(qg, a.signs, a.mult, qs);
     __syncthreads();
 
     if (scorer) {
@@ -417,7 +413,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
       const int tk0 = warp * WT + ((tid >> 3) & 3) * 4;  // first token of this lane group, round 0
       const bool writer_lo = (sl & 1) == 0;
       const uint32_t rep_off = rep_offset<BITS, kDecReps>(lane);
-      const uint8_t* ksrc = DENSE ? reinterpret_cast<const uint8_t*>(a.kdense) : a.kcodes;
+      const uint8_t* ksrc = a.kcodes;
       float2 qp[HG][J / 2];
       if constexpr (P::PASSES == 1) {
 #pragma unroll
@@ -433,7 +429,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int t = start + tk0 + 16 * r + kord;
-        kn_next[r] = (!DENSE && ntiles > 0 && t < end) ? __half2float(a.knorms[kv_row0 + t]) : 1.f;
+        kn_next[r] = (ntiles > 0 && t < end) ? __half2float(a.knorms[kv_row0 + t]) : 1.f;
         vn_next[r] = (VQ && ntiles > 0 && t < end) ? __half2float(a.vnorms[kv_row0 + t]) : 1.f;
       }
       auto issue_k = [&](int tile) {
@@ -461,7 +457,7 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
           vn_cur[r] = vn_next[r];
           const int t = t0 + TT + tk0 + 16 * r + kord;  // my tokens of the next tile
           if (it + 1 < ntiles && t < end) {
-            if constexpr (!DENSE) kn_next[r] = __half2float(a.knorms[kv_row0 + t]);
+            kn_next[r] = __half2float(a.knorms[kv_row0 + t]);
             if constexpr (VQ) vn_next[r] = __half2float(a.vnorms[kv_row0 + t]);
           }
         }
@@ -484,24 +480,8 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               const int tt = tk + (k ^ kord);
-              if constexpr (DENSE) {
-                const __half2* kh = reinterpret_cast<const __half2*>(st + tt * P::KROW + 2 * J * sl);
-                float2 s2[HG];
-#pragma unroll
-                for (int h = 0; h < HG; ++h) s2[h] = make_float2(0.f, 0.f);
-#pragma unroll
-                for (int i = 0; i < J / 2; ++i) {
-                  const float2 kf = __half22float2(kh[i]);
-#pragma unroll
-                  for (int h = 0; h < HG; ++h) s2[h] = fma2(qp[h][i], kf, s2[h]);
-                }
-#pragma unroll
-                for (int h = 0; h < HG; ++h) v[k][h] = s2[h].x + s2[h].y;
-              } else {
-                const uint64_t bits = load_slice<D, BITS, J>(st + tt * P::KROW, sl);
-                factored_slice<BITS, J, HG, kDecReps>(bits, reinterpret_cast<const uint8_t*>(tab), rep_off, qp,
-                                                      v[k]);
-              }
+              const uint64_t bits = load_slice<D, BITS, J>(st + tt * P::KROW, sl);
+              factored_slice<BITS, J, HG, kDecReps>(bits, reinterpret_cast<const uint8_t*>(tab), rep_off, qp, v[k]);
             }
 #pragma unroll
             for (int h = 0; h < HG; ++h) {

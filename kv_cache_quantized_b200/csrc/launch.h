@@ -44,10 +44,13 @@ axr_status attend_fused_launch(int d, int bits, int G, bool vq, const DecodeArgs
 // Row-layout cache, quantized keys scored through warp-level MMAs (attend_rows.cu); vq: values quantized.
 axr_status attend_rows_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st);
 
-// Row-layout cache on CUDA cores (attend_partial.cu): quantized keys through the factored gather, or fp16 keys
-// (dense; bits ignored).
-axr_status attend_partial_launch(int d, int bits, int G, bool vq, bool dense, const DecodeArgs& a, cudaStream_t st,
+// Row-layout cache on CUDA cores (attend_partial.cu): quantized keys through the factored gather.
+axr_status attend_partial_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st,
                                  const char* what);
+
+// Unquantized fp16 keys and values (dense.cu): the dense bandwidth reference, one streaming worker per warp; the
+// arguments carry the plan_splits_dense split plan.
+axr_status dense_launch(int d, int G, const DecodeArgs& a, cudaStream_t st, const char* what);
 
 // Tiled value layout, d = 128 (attend_tiled.cu): tcgen05 kernel if tensor, else warp-level MMAs.
 axr_status attend_tiled_launch(int bits, int G, bool tensor, const DecodeArgs& a, cudaStream_t st);

@@ -15,12 +15,9 @@
 #pragma once
 
 #include "axr_common.cuh"
+#include "warp_mma.cuh"
 
 namespace axr {
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
 
 template <int D>
 struct SelTcPlan {
@@ -35,44 +32,6 @@ struct SelTcPlan {
   static constexpr int NO = D / 8;                     // n-tiles of the output
   static constexpr int NS = BK / 8;                    // n-tiles of the scores (keys)
 };
-
-// 16-byte global -> shared copy; src_bytes = 0 fills the destination with zeros
-__device__ __forceinline__ void cp16(void* dst, const void* src, int src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_addr(dst)), "l"(src), "r"(src_bytes));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t pack_h2(float lo_elem, float hi_elem) {
-  const __half2 h = __floats2half2_rn(lo_elem, hi_elem);
-  return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// hi and lo fp16 planes of two values, packed as half2 words
-__device__ __forceinline__ void split_h2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  const __half h0 = __float2half_rn(x0), h1 = __float2half_rn(x1);
-  const __half2 hh = __halves2half2(h0, h1);
-  hi = *reinterpret_cast<const uint32_t*>(&hh);
-  lo = pack_h2(x0 - __half2float(h0), x1 - __half2float(h1));
-}
 
 // One block: query rows [q0, q0 + 64) of head h of (layer, sequence) ls for candidate ci of the chunk.
 //   q     [Ly, S, Hq, N, D] f32;  kh, kl [chunk][Ly, S, Hkv, N, D] fp16 hi / lo planes of the reconstructed keys;

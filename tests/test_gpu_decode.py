@@ -267,18 +267,45 @@ def test_decode_step_many_items(vq):
     assert bool(torch.all(num <= 2.0 ** -11 * den)), float((num / den).max())
 
 
-def test_dense_matches_oracle_attention():
-    B, Hkv, G, T, Tcap, d = 3, 2, 4, 2100, 2200, 128
-    k = W.lognormal_rows((B, Hkv, T, d), 800, dtype=np.float16)
-    v = W.normal((B, Hkv, T, d), 801, np.float16)
-    q = W.normal((B, Hkv * G, d), 802, np.float32)
-    lens = np.array([T, 5, 1500], np.int32)
-    out = ops.dense_decode(cuda(q), cuda(padded(k, Tcap)), cuda(padded(v, Tcap)), seq_lens=cuda(lens),
-                           T=T).cpu().numpy()
+@pytest.mark.parametrize("d,G,Hkv", [(128, 4, 2), (64, 8, 1), (128, 1, 3), (64, 2, 2), (128, 8, 1)])
+def test_dense_matches_oracle_attention(d, G, Hkv):
+    """The dense fp16 kernel (per-warp streaming workers) against the oracle's attention on the same fp16 cache:
+    every (d, G) family, rows of 0, 1, 5 and ragged lengths (tails inside a 32-token tile, chunks split over
+    several workers), and garbage past each row's length that must not be read."""
+    B, T, Tcap = 5, 2100, 2200
+    k = W.lognormal_rows((B, Hkv, T, d), 800 + d + G, dtype=np.float16)
+    v = W.normal((B, Hkv, T, d), 801 + d + G, np.float16)
+    q = W.normal((B, Hkv * G, d), 802 + d + G, np.float32)
+    lens = np.array([T, 5, 1500, 0, 1], np.int32)
+    kp, vp = padded(k, Tcap, fill=np.nan), padded(v, Tcap, fill=np.nan)
+    for b in range(B):  # positions past the row's length hold NaN: a read of one would show in the output
+        kp[b, :, lens[b]:] = np.nan
+        vp[b, :, lens[b]:] = np.nan
+    out = ops.dense_decode(cuda(q), cuda(kp), cuda(vp), seq_lens=cuda(lens), T=T).cpu().numpy()
     for b in range(B):
         Tb = lens[b]
+        if Tb == 0:
+            assert np.all(out[b] == 0)
+            continue
         want = oracle.attention(q[b][:, None, :], k[b, :, :Tb], v[b, :, :Tb], causal=False)[:, 0, :]
         parity.check_outputs(out[b], want)
+
+
+def test_dense_full_size_sampled():
+    """The long-context shape (B=8, T=32768, 32/8 heads, d=128) through the dense kernel, in the launch
+    configuration the benchmark times; sampled (batch row, KV head) pairs against the oracle."""
+    B, Hkv, G, T, d = 8, 8, 4, 32768, 128
+    dev = torch.device("cuda", 0)
+    k = W.lognormal_rows_device((B, Hkv, T, d), 810, dev)
+    v = W.normal_device((B, Hkv, T, d), 811, dev, dtype=torch.float16)
+    q = W.normal_device((B, Hkv * G, d), 812, dev, dtype=torch.float32)
+    out = ops.dense_decode(q, k, v).cpu().numpy()
+    for b, hk in [(0, 0), (3, 5), (7, 7)]:
+        kk = k[b, hk].cpu().numpy()
+        vv = v[b, hk].cpu().numpy()
+        qq = q[b, hk * G:(hk + 1) * G].cpu().numpy()
+        want = oracle.attention(qq[:, None, :], kk[None], vv[None], causal=False)[:, 0, :]
+        parity.check_outputs(out[b, hk * G:(hk + 1) * G], want)
 
 
 def test_split_count_invariance():
