@@ -43,6 +43,14 @@ L2_BYTES = 126 * 1024 * 1024
 # (dram__bytes_read.sum, dram__bytes_write.sum, three launches) of the same workload at B=4 (half the units) read
 # 138.582 MB and wrote 1.457 MB per launch on average; scaled by the units processed.  Valid for the kernel version
 # that capture was taken on; a workload without an entry reports null.
+def _step_kernel(w) -> str:
+    """The decode kernel the library runs for a contiguous decode step of this workload: the streaming kernel for
+    fp16 values, and for quantized values at eight query heads per KV head or more than 296 (batch row, KV head)
+    units; the row kernel otherwise."""
+    stream = (not w.v_quant) or w.Hq // w.Hkv == 8 or w.B * w.Hkv > 296
+    return "attend_stream_kernel" if stream else "attend_rows_kernel"
+
+
 TRAFFIC = {
     "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.581845e6 + 1.457408e6),
 }
@@ -599,7 +607,7 @@ def run_axr(args, w):
                    "values": "quantized b=%d" % bits if w.v_quant else "fp16", "parallelism": f"replicas x{ws}",
                    "l2": "flushed between steps (256 MiB write outside the per-step events)"},
         "hbm_gbs": alg_bytes * ws * args.steps / (step_ms / 1e3) / 1e9,
-        "roofline": {"bound": "hbm", "kernel": "attend_rows_kernel (with the new token's write) + "
+        "roofline": {"bound": "hbm", "kernel": f"{_step_kernel(w)} (with the new token's write) + "
                      "attend_reduce_kernel (one axr_decode_step call)", "achieved": achieved,
                      "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,

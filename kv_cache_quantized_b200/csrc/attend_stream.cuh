@@ -1,0 +1,392 @@
+// Decode attention over quantized keys, and fp16 or quantized values, as a pure stream: the dense kernel's skeleton
+// (dense_stream.cuh) with the keys scored from their codes.
+//
+// AXELRAM Key Points (1st, 2nd items): a token's score is the gather-sum of q~_j c_k at its stored indices times its
+// stored norm; the table is read in factored form on mma.sync exactly as mma_score.cuh does it (one MMA per 8 tokens
+// and 16 coordinates carries the four products of the hi/lo fp16 planes of both factors; fp32 accumulation).  Lane
+// (g, t) then holds head t's scores of tokens g and g + 8 of each 16-token group.  The value product is
+//   O^T (d x heads) += V^T (d x tokens) P^T (tokens x heads):
+//   fp16 values: A = V^T, read with ldmatrix.trans from the 128-byte-swizzled TMA boxes of the value rows; B = P^T
+//       as hi and lo fp16 planes (fp32-level weights, so that the result does not depend on where the splits fall),
+//       gathered from the score lanes with four shuffles per 16 tokens;
+//   quantized values: A = V^T from the hi-only copies of the key/value pair table (one lookup of a code byte gives
+//       the fp16 pair (v_2p, v_2p+1) of a token; two byte permutes of the pairs of tokens k and k + 1 give two A
+//       registers, as in attend_rows.cuh); B = P^T times the value norm and 1 / sqrt(D), fp16 (the table's hi plane
+//       holds the centroids to 2^-11); the product stays in the rotated domain and the merge applies the one inverse
+//       transform.
+//
+// Every warp is an independent worker over (batch row, KV head, split) items with a ring of NS stages of its own: a
+// stage holds TW tokens' value rows (fp16: D / 64 tiled TMA boxes; quantized: one bulk copy of code rows) and key
+// code rows (one bulk copy).  No barrier spans two
+// warps.  A decode step's new token is written by the warp whose item holds it, before that item's copies.
+#pragma once
+
+#include <cuda.h>
+
+#include "append.cuh"
+#include "dense_stream.cuh"
+#include "mma_score.cuh"
+
+namespace axr {
+
+template <int D, int BITS, int G, bool VQ>
+struct StreamPlan {
+  static constexpr int TW = 32;                          // tokens per warp tile
+  static constexpr int NS = 2;                           // stages per warp
+  static constexpr int WARPS = VQ ? 12 : 8;              // warps per block (one block per SM)
+  static constexpr int THREADS = 32 * WARPS;
+  static constexpr int R = D * BITS / 8;                 // bytes of a key code row
+  static constexpr int BOXC = 64;                        // value coordinates per TMA box
+  static constexpr int NBX = D / BOXC;                   // value boxes per row
+  static constexpr size_t BOX = (size_t)TW * 128;
+  static constexpr size_t VPLANE = VQ ? (size_t)TW * R : NBX * BOX;  // value rows of a stage (first: 1024-aligned)
+  static constexpr size_t KPLANE = (size_t)TW * R;       // key code rows of a stage
+  static constexpr size_t STAGE = (VPLANE + KPLANE + 1023) / 1024 * 1024;
+  static constexpr size_t SCRATCH = ((size_t)G * D * 4 + D + 1023) / 1024 * 1024;  // queries + index scratch
+  static constexpr size_t WARP_BYTES = NS * STAGE > SCRATCH ? NS * STAGE : SCRATCH;
+  static constexpr size_t OFF_TAB = WARPS * WARP_BYTES;
+  static constexpr size_t TAB_BYTES = VQ ? (size_t)PairTableKV<BITS>::BYTES : (size_t)HiLoTable16<BITS>::BYTES;
+  static constexpr size_t OFF_MBAR = OFF_TAB + TAB_BYTES;
+  static constexpr size_t bytes = 1024 + OFF_MBAR + (size_t)WARPS * NS * 8;  // + the alignment slack
+  static constexpr int NT = MmaB<D, G>::NT;              // n-tiles of heads (2: heads 4..7)
+  static constexpr int MTV = D / 16;                     // m-tiles of the value product (16 coordinates)
+  static constexpr int NBV = R / 8;                      // quantized values: bytes of lane g's run of a row
+  static constexpr int NWV = (NBV + 3) / 4 + 1;          // its words, plus a zero word
+  static_assert(R % 16 == 0, "key code rows of whole 16-byte chunks (one bulk copy per tile)");
+  static_assert(TW == 32, "two 16-token groups per tile");
+  static_assert(bytes <= 227 * 1024, "shared memory of one block");
+};
+
+// vmap: the TMA map of the fp16 value cache (fp16 values only).
+template <int D, int BITS, int G, bool VQ>
+__global__ void __launch_bounds__(StreamPlan<D, BITS, G, VQ>::THREADS, 1)
+attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap vmap) {
+  using P = StreamPlan<D, BITS, G, VQ>;
+  constexpr int TW = P::TW, NS = P::NS, R = P::R, NT = P::NT, MTV = P::MTV, VPL = WarpVec<D>::VPL;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  uint8_t* ring = smem + static_cast<size_t>(warp) * P::WARP_BYTES;
+  const uint8_t* tab = smem + P::OFF_TAB;
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + P::OFF_MBAR) + warp * NS;
+
+  {  // the pair table, once per block: hi/lo key copies (and hi-only value copies with quantized values)
+    __shared__ float gamma_s[16];
+    if (threadIdx.x < 16) gamma_s[threadIdx.x] = a.cb.gamma[threadIdx.x];
+    if (lane == 0)
+      for (int s = 0; s < NS; ++s) tc::mbar_init(mbar + s, 1);
+    __syncthreads();
+    if constexpr (VQ) build_pair_table_kv<BITS>(gamma_s, smem + P::OFF_TAB);
+    else build_hilo_table16<BITS>(gamma_s, smem + P::OFF_TAB);
+    __syncthreads();
+  }
+  // the split merge, launched as this grid's programmatic dependent, may be scheduled from now on
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+
+  // the lane's key copy in the pair table, and (quantized values) its hi-only value copy
+  const uint32_t repk = static_cast<uint32_t>(lane & 15) << (VQ ? 3 : 4);
+  const uint32_t repv = 128u + (static_cast<uint32_t>(lane) << 2);
+  // quantized values: lanes with odd t fetch token k + 1 before k (rows of both parities in every half-warp: no bank
+  // conflicts), so their byte permutes take the two pairs the other way round
+  const int tf = t & 1;
+  const uint32_t sel_lo = tf ? 0x1054u : 0x5410u, sel_hi = tf ? 0x3276u : 0x7632u;
+  const int a_row = (lane & 7) + 8 * (lane >> 4), a_col = 8 * ((lane >> 3) & 1);  // ldmatrix.trans rows of V^T
+  const float rd = rsqrtf(static_cast<float>(D));
+  // items are dealt across the blocks first (item blockIdx.x + gridDim.x (warp + WARPS k)), so that a launch with
+  // fewer items than workers still spreads them over every SM
+  const int workers = gridDim.x * P::WARPS;
+  const int first = blockIdx.x + gridDim.x * warp;
+  const int items = a.B * a.Hkv * a.splits;
+  uint32_t seq = 0;  // tiles this warp has consumed: stage seq % NS, phase parity (seq / NS) & 1
+  bool failed = false;
+
+  for (int item = first; item < items && !failed; item += workers) {
+    const int split = item % a.splits;
+    const int hk = (item / a.splits) % a.Hkv;
+    const int b = item / (a.splits * a.Hkv);
+    const int len = row_len(a, b);
+    const int start = split * a.chunk;
+    const int end = min(start + a.chunk, len);
+    const int ntiles = end > start ? (end - start + TW - 1) / TW : 0;
+    const size_t row0 = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
+    const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
+    // the ring is idle between items: it holds the transformed queries and the write path's index scratch
+    float* qs = reinterpret_cast<float*>(ring);
+    uint8_t* scratch = ring + static_cast<size_t>(G) * D * 4;
+
+    if (a.knew != nullptr && len > 0 && start <= len - 1 && len - 1 < end) {
+      // decode step: this item holds the new token (position len - 1): write its key and value through the write
+      // path before any of the item's copies is issued
+      append_row<D, BITS, VQ>(a, b, hk, row0 + len - 1, 0, lane, scratch);
+      append_row<D, BITS, VQ>(a, b, hk, row0 + len - 1, 1, lane, scratch);
+      __threadfence();                                           // the stores reach the device-wide view ...
+      asm volatile("fence.proxy.async.global;\n" ::: "memory");  // ... and the async proxy of the copies
+    }
+
+    // q~_h = mult H (s .* q_h) / sqrt(D) for the G heads, then the key MMA's B fragments (head-scaled hi/lo planes)
+    for (int h = 0; h < G; ++h) {
+      float v[VPL];
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int j = lane * VPL + i;
+        v[i] = qg[h * D + j] * sign_of(a.signs[j]);
+      }
+      fwht_warp<D>(v, lane);
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) qs[h * D + lane * VPL + i] = v[i] * (a.mult * rd);
+    }
+    MmaB<D, G> QB;
+    {
+      float scl[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) scl[h] = tc::head_scale<D>(qg + h * D, a.mult);
+      __syncwarp();
+      mma_b_build<D, G>(qs, scl, lane, QB);
+    }
+    // this lane's scratch accesses come before the async proxy's copies into the ring, for every lane
+    fence_proxy_async();
+    __syncwarp();
+
+    auto issue = [&](int i) {
+      if (lane == 0) {
+        const int s = static_cast<int>((seq + i) % NS);
+        uint8_t* st = ring + static_cast<size_t>(s) * P::STAGE;
+        const int t0 = start + i * TW;
+        const int n = min(TW, end - t0);
+        if constexpr (VQ) {
+          mbar_arrive_expect_tx(mbar + s, static_cast<uint32_t>(2 * n * R));
+          bulk_copy_g2s(st, static_cast<const uint8_t*>(a.v) + (row0 + t0) * R, static_cast<uint32_t>(n * R),
+                        mbar + s);
+        } else {
+          mbar_arrive_expect_tx(mbar + s, static_cast<uint32_t>(P::VPLANE + n * R));
+#pragma unroll
+          for (int bx = 0; bx < P::NBX; ++bx)
+            tma_load_2d(st + bx * P::BOX, &vmap, bx * P::BOXC, static_cast<int>(row0) + t0, mbar + s);
+        }
+        bulk_copy_g2s(st + P::VPLANE, a.kcodes + (row0 + t0) * R, static_cast<uint32_t>(n * R), mbar + s);
+      }
+    };
+    for (int i = 0; i < NS && i < ntiles; ++i) issue(i);
+
+    // O^T: (coordinate 16 mt + g (+ 8), head 2 t (+ 1)); quantized values: coordinates 2 (MTV g + mt) (+ 1)
+    float acc[MTV][4];
+#pragma unroll
+    for (int mt = 0; mt < MTV; ++mt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+    float m_run[NT], l_lane[NT];  // head 4 nt + t
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) { m_run[nt] = -INFINITY; l_lane[nt] = 0.f; }
+
+    // key (and value) norms of this lane's tokens (16 m + g + 8 i of a tile) times 1 / sqrt(D), one tile ahead;
+    // L2-only loads, since a decode step writes one of them in this launch
+    auto load_norms = [&](int i, float (&kn)[2][2], float (&vn)[2][2]) {
+      const int t0 = start + i * TW;
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int tok = t0 + 16 * m + g + 8 * e;
+          const bool in = i < ntiles && tok < end;
+          kn[m][e] = in ? __half2float(__ldcg(a.knorms + row0 + tok)) * rd : 0.f;
+          if constexpr (VQ) vn[m][e] = in ? __half2float(__ldcg(a.vnorms + row0 + tok)) * rd : 0.f;
+          else vn[m][e] = 1.f;
+        }
+    };
+    float kn_next[2][2], vn_next[2][2];
+    load_norms(0, kn_next, vn_next);
+
+    for (int i = 0; i < ntiles; ++i) {
+      const int s = static_cast<int>((seq + i) % NS);
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(mbar + s, ((seq + i) / NS) & 1))) {
+        // a wait gave up: stop issuing and let this warp's copies in flight land (bounded again) before exiting
+        failed = true;
+        for (int j = i; j < i + NS && j < ntiles; ++j) tc::mbar_wait(mbar + (seq + j) % NS, ((seq + j) / NS) & 1);
+        break;
+      }
+      uint8_t* st = ring + static_cast<size_t>(s) * P::STAGE;
+      const uint32_t sV = smem_u32(st);
+      const int t0 = start + i * TW;
+      float kn[2][2], vn[2][2];
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) { kn[m][e] = kn_next[m][e]; vn[m][e] = vn_next[m][e]; }
+      load_norms(i + 1, kn_next, vn_next);
+      if (!VQ && t0 + TW > end) {
+        // the row ends inside this tile: zero the value rows past it (whatever the cache holds there); the key
+        // rows past it are stale codes, valid table indices, whose scores are masked
+        uint4* vz = reinterpret_cast<uint4*>(st);
+        const int r0 = end - t0;
+        for (int e = lane; e < (TW - r0) * 8 * P::NBX; e += 32) {
+          const int bx = e / ((TW - r0) * 8), rem = e % ((TW - r0) * 8);
+          vz[(bx * P::BOX + (r0 + rem / 8) * 128) / 16 + rem % 8] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+      }
+
+      // ---- scores of the tile's two 16-token groups (times s_h): z[m][nt][i] is token 16 m + g + 8 i, head 4 nt + t
+      float z[2][NT][2];
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+        mma_scores16<D, BITS, G, false, VQ>(st + P::VPLANE, 16 * m, tab, repk, QB, lane, z[m]);
+
+      // ---- online softmax per head (log2 units), over the lanes g of each t
+      float alpha[NT];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const bool head = 4 * nt + t < G;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const bool valid = head && t0 + 16 * m + g + 8 * e < end;
+            z[m][nt][e] = valid ? z[m][nt][e] * QB.inv[nt] * kn[m][e] : -INFINITY;
+            mx = fmaxf(mx, z[m][nt][e]);
+          }
+#pragma unroll
+        for (int msk = 4; msk < 32; msk <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, msk));
+        const float m_new = fmaxf(m_run[nt], mx);
+        alpha[nt] = (m_new == -INFINITY) ? 1.f : exp2f(m_run[nt] - m_new);
+        float ps = 0.f;
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float p = (z[m][nt][e] == -INFINITY) ? 0.f : exp2f(z[m][nt][e] - m_new);
+            z[m][nt][e] = p;
+            ps += p;
+          }
+        l_lane[nt] = l_lane[nt] * alpha[nt] + ps;
+        m_run[nt] = m_new;
+      }
+      // rescale the accumulators (columns: heads 2 t and 2 t + 1) when some head's running max moved
+      bool moved = false;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) moved |= alpha[nt] != 1.f;
+      if (__any_sync(0xffffffffu, moved)) {
+        float al[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int h = 2 * t + c;  // held by lanes t' = h % 4 in n-tile h / 4
+          float x = __shfl_sync(0xffffffffu, alpha[0], h & 3);
+          if constexpr (NT > 1) {
+            const float y = __shfl_sync(0xffffffffu, alpha[NT - 1], h & 3);
+            x = h >= 4 ? y : x;
+          }
+          al[c] = x;
+        }
+#pragma unroll
+        for (int mt = 0; mt < MTV; ++mt) {
+          acc[mt][0] *= al[0]; acc[mt][1] *= al[1];
+          acc[mt][2] *= al[0]; acc[mt][3] *= al[1];
+        }
+      }
+
+      // ---- O^T += V^T P^T per 16-token group: B = P^T (tokens 2 t, 2 t + 1 | + 8, + 9; head g)
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        float pv[2][2];  // [b register][token of the pair]
+#pragma unroll
+        for (int e = 0; e < 2; ++e)
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int src = 4 * (2 * t + u) + (g & 3);  // the lane holding token 2 t + u (+ 8 e) of head g % 4 (+ 4)
+            float x = __shfl_sync(0xffffffffu, z[m][0][e] * vn[m][e], src);
+            if constexpr (NT > 1) {
+              const float y = __shfl_sync(0xffffffffu, z[m][NT - 1][e] * vn[m][e], src);
+              x = g >= 4 ? y : x;
+            } else {
+              x = g < G ? x : 0.f;
+            }
+            pv[e][u] = x;
+          }
+        if constexpr (VQ) {
+          // the weights p n^V / sqrt(D) in fp16; A = V^T from the value codes of tokens k0, k0 + 1, k0 + 8, k0 + 9
+          const uint32_t b0 = pack_h2(pv[0][0], pv[0][1]), b1 = pack_h2(pv[1][0], pv[1][1]);
+          const int k0 = 16 * m + 2 * t;
+          uint32_t w[4][P::NWV];
+          load_run<R, P::NBV, false>(st, (k0 + tf) * R + g * P::NBV, w[0]);
+          load_run<R, P::NBV, false>(st, (k0 + 1 - tf) * R + g * P::NBV, w[1]);
+          load_run<R, P::NBV, false>(st, (k0 + 8 + tf) * R + g * P::NBV, w[2]);
+          load_run<R, P::NBV, false>(st, (k0 + 9 - tf) * R + g * P::NBV, w[3]);
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+#pragma unroll
+            for (int x = (P::NBV + 3) / 4; x < P::NWV; ++x) w[r][x] = 0u;
+#pragma unroll
+          for (int mt = 0; mt < MTV; ++mt) {
+            uint32_t x[4];  // hi fp16 pairs (v_2p, v_2p+1) of the four tokens, p = MTV g + mt
+#pragma unroll
+            for (int r = 0; r < 4; ++r) x[r] = *reinterpret_cast<const uint32_t*>(tab + kv_off<BITS>(w[r], mt, repv));
+            mma16816(acc[mt], __byte_perm(x[0], x[1], sel_lo), __byte_perm(x[0], x[1], sel_hi),
+                     __byte_perm(x[2], x[3], sel_lo), __byte_perm(x[2], x[3], sel_hi), b0, b1);
+          }
+        } else {
+          uint32_t bh0, bl0, bh1, bl1;
+          split_h2(pv[0][0], pv[0][1], bh0, bl0);
+          split_h2(pv[1][0], pv[1][1], bh1, bl1);
+#pragma unroll
+          for (int mt = 0; mt < MTV; ++mt) {
+            uint32_t va[4];
+            ldsm_x4_t(sV + swz<TW>(16 * m + a_row, 16 * mt + a_col), va[0], va[1], va[2], va[3]);
+            mma16816(acc[mt], va[0], va[1], va[2], va[3], bh0, bh1);
+            mma16816(acc[mt], va[0], va[1], va[2], va[3], bl0, bl1);
+          }
+        }
+      }
+
+      // the stage is free once every lane's reads (and zeroing writes) of it are done: each lane orders its own
+      // accesses before the async proxy's, then the warp syncs, then lane 0 refills it with tile i + NS
+      fence_proxy_async();
+      __syncwarp();
+      if (i + NS < ntiles) issue(i + NS);
+    }
+    if (failed) break;
+    seq += static_cast<uint32_t>(ntiles);
+
+    // ---- the item's partials
+    const size_t part0 = (static_cast<size_t>(b) * a.Hq + hk * G) * a.splits + split;  // head h adds h * splits
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      float l = l_lane[nt];
+#pragma unroll
+      for (int msk = 4; msk < 32; msk <<= 1) l += __shfl_xor_sync(0xffffffffu, l, msk);
+      const int h = 4 * nt + t;
+      if (g == 0 && h < G) {
+        a.ws_m[part0 + static_cast<size_t>(h) * a.splits] = m_run[nt];
+        a.ws_l[part0 + static_cast<size_t>(h) * a.splits] = l;
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int h = 2 * t + c;
+      if (h < G) {
+        float* dst = a.ws_o + (part0 + static_cast<size_t>(h) * a.splits) * D;
+#pragma unroll
+        for (int mt = 0; mt < MTV; ++mt) {
+          const int r0 = VQ ? 2 * (MTV * g + mt) : 16 * mt + g, r1 = VQ ? r0 + 1 : r0 + 8;
+          dst[r0] = acc[mt][c];
+          dst[r1] = acc[mt][2 + c];
+        }
+      }
+    }
+    __syncwarp();  // every lane is done with this item's ring before the next item's scratch writes
+  }
+
+  if (failed) {
+    // poison every partial this warp owns (the merge then yields NaN) and record the failure in the status word
+    for (int item = first; item < items; item += workers) {
+      const int split = item % a.splits;
+      const int hk = (item / a.splits) % a.Hkv;
+      const int b = item / (a.splits * a.Hkv);
+      if (lane < G) a.ws_m[(static_cast<size_t>(b) * a.Hq + hk * G + lane) * a.splits + split] =
+          __int_as_float(0x7fc00000);
+    }
+    if (lane == 0 && a.status) atomicOr(a.status, 1u);
+  }
+}
+
+}  // namespace axr

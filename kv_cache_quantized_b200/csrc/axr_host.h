@@ -63,18 +63,27 @@ inline SplitPlan plan_splits(int B, int Hkv, int T, long resident = kResident, i
   return p;
 }
 
-// The dense fp16 kernel's plan: one worker per warp (4 per SM), 32-token tiles, chunks of at least 8 tiles, and a
-// setup of about one tile (the worker's copy ring fills before its first tile).
+// The plan of the streaming kernels (per-warp workers over 32-token tiles): chunks of at least 2 tiles, and a setup
+// of about two tiles (a worker transforms its queries and fills its copy ring before its first tile), so that small
+// problems spread over many workers.  The dense fp16 kernel runs 4 workers per SM, the kernel for quantized keys
+// over fp16 values 8.
+constexpr int kStreamTile = 32;
 constexpr int kDenseWorkers = 4 * kSmCount;
-constexpr int kDenseTile = 32;
-inline SplitPlan plan_splits_dense(int B, int Hkv, int T) {
-  return plan_splits(B, Hkv, T, kDenseWorkers, kDenseTile, 8, 1.0);
+constexpr int kAttendStreamWorkers = 8 * kSmCount;   // fp16 values
+constexpr int kAttendStreamWorkersQ = 12 * kSmCount; // quantized values
+inline SplitPlan plan_splits_stream(int B, int Hkv, int T, int workers) {
+  return plan_splits(B, Hkv, T, workers, kStreamTile, 2, 2.0);
 }
 
 inline size_t attend_ws_bytes(int B, int Hq, int Hkv, int T, int d) {
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || T <= 0 || d <= 0) return 0;
-  const SplitPlan p = plan_splits(B, Hkv, T), pd = plan_splits_dense(B, Hkv, T);
-  const size_t parts = static_cast<size_t>(B) * Hq * (p.splits > pd.splits ? p.splits : pd.splits);
+  // the largest split count of the plans (the kernels that may run on this workspace)
+  int splits = plan_splits(B, Hkv, T).splits;
+  for (int workers : {kDenseWorkers, kAttendStreamWorkers, kAttendStreamWorkersQ}) {
+    const int s = plan_splits_stream(B, Hkv, T, workers).splits;
+    splits = s > splits ? s : splits;
+  }
+  const size_t parts = static_cast<size_t>(B) * Hq * splits;
   size_t bytes = parts * static_cast<size_t>(d) * sizeof(float) + 2 * parts * sizeof(float);
   return (bytes + 255) / 256 * 256;
 }

@@ -127,14 +127,27 @@ axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, con
   const Codebook* cb = codebook_for(d, bits);
   if (!cb) return set_error(AXR_EINVAL, "%s: codebook unavailable", w);
   DecodeArgs a = base_args(B, Hq, Hkv, T, Tcap, seq_lens, q, scale * kLog2e);
+  const int mode = g_gather.load();
+  // row-layout values on a contiguous cache, keys through warp-level MMAs (attend and decode step): the streaming
+  // kernel for fp16 values; for quantized values where it measured faster than attend_rows (eight query heads per
+  // KV head, or more (batch row, KV head) units than attend_rows has resident blocks), else attend_rows, which is
+  // ahead at four query heads per KV head and few units (the long-context step: 120 against 127 us)
+  const bool stream_vq = vkind == AXR_V_QUANT && (Hq / Hkv == 8 || static_cast<long>(B) * Hkv > kResident);
+  const bool stream_path = (vkind == AXR_V_F16 || stream_vq) && !paged && attend_stream_supported(d, bits) &&
+                           (step || mode == kGatherMma || mode == kGatherDirect);
+  if (stream_path) {
+    const SplitPlan p =
+        plan_splits_stream(B, Hkv, T, vkind == AXR_V_QUANT ? kAttendStreamWorkersQ : kAttendStreamWorkers);
+    a.splits = p.splits; a.chunk = p.chunk;
+  }
   st = carve_workspace(a, d, workspace, ws_bytes, w);
   if (st != AXR_OK) return st;
   a.kcodes = kcodes; a.knorms = reinterpret_cast<const __half*>(knorms); a.signs = signs; a.out = out;
   a.v = v; a.vnorms = reinterpret_cast<const __half*>(vnorms); a.cb = *cb;
   a.knew = reinterpret_cast<const __half*>(knew); a.vnew = reinterpret_cast<const __half*>(vnew);
   const int G = Hq / Hkv;
-  const int mode = g_gather.load();
   const bool vq = vkind == AXR_V_QUANT;
+  if (stream_path) return attend_stream_launch(d, bits, G, vq, a, as_stream(stream), w);
   if (paged) {
     a.block_table = block_table; a.max_blocks = max_blocks; a.block_shift = shift;
   }
@@ -218,7 +231,7 @@ extern "C" axr_status axr_dense_decode(const float* q, const uint16_t* k, const 
     return e == cudaSuccess ? set_error(AXR_OK, "") : set_error(AXR_ECUDA, "%s: %s", w, cudaGetErrorString(e));
   }
   DecodeArgs a = base_args(B, Hq, Hkv, T, Tcap, seq_lens, q, scale * kLog2e);
-  const SplitPlan p = plan_splits_dense(B, Hkv, T);
+  const SplitPlan p = plan_splits_stream(B, Hkv, T, kDenseWorkers);
   a.splits = p.splits; a.chunk = p.chunk;
   st = carve_workspace(a, d, workspace, ws_bytes, w);
   if (st != AXR_OK) return st;

@@ -23,6 +23,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // 2-D map over an fp16 cache viewed as [rows, D]: boxes of `box_rows` rows x 64 coordinates, 128-byte swizzle.
 axr_status encode_cache_map(CUtensorMap* map, const void* base, size_t rows, int D, int box_rows, const char* what) {
   auto fn = encode_fn();
@@ -38,10 +40,12 @@ axr_status encode_cache_map(CUtensorMap* map, const void* base, size_t rows, int
   return AXR_OK;
 }
 
+namespace {
+
 template <int D, int G>
 axr_status launch(const DecodeArgs& a, cudaStream_t st, const char* what) {
   using P = DenseStreamPlan<D, G>;
-  static_assert(P::WARPS * kSmCount == kDenseWorkers && P::TW == kDenseTile, "the split plan's worker model");
+  static_assert(P::WARPS * kSmCount == kDenseWorkers && P::TW == kStreamTile, "the split plan's worker model");
   auto k = dense_stream_kernel<D, G>;
   axr_status rs = ensure_smem(k, P::bytes, what);
   if (rs != AXR_OK) return rs;
@@ -51,9 +55,8 @@ axr_status launch(const DecodeArgs& a, cudaStream_t st, const char* what) {
   CUtensorMap kmap, vmap;
   if ((rs = encode_cache_map(&kmap, a.kdense, rows, D, P::TW, what)) != AXR_OK) return rs;
   if ((rs = encode_cache_map(&vmap, a.v, rows, D, P::TW, what)) != AXR_OK) return rs;
-  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // one per warp worker, dealt round-robin
-  const long blocks = (items + P::WARPS - 1) / P::WARPS;
-  const unsigned grid = static_cast<unsigned>(blocks < kSmCount ? blocks : kSmCount);
+  const long items = static_cast<long>(a.B) * a.Hkv * a.splits;  // one per warp worker, dealt across the blocks
+  const unsigned grid = static_cast<unsigned>(items < kSmCount ? items : kSmCount);
   k<<<grid, P::THREADS, P::bytes, st>>>(a, kmap, vmap);
   launch_reduce<D, false>(a, st);
   return check_launch(what);

@@ -47,12 +47,6 @@ struct DenseStreamPlan {
   static_assert(D % BOXC == 0 && BOX % 1024 == 0, "whole boxes, each aligned for the 128-byte swizzle");
 };
 
-// Workers (warps) the launch provides, for the split plan.
-template <int D, int G>
-constexpr int dense_stream_workers() {
-  return kSmCount * DenseStreamPlan<D, G>::WARPS;
-}
-
 // Tiled TMA load of box (x = first coordinate, y = first cache row) of `map` into shared memory, completing on mbar.
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* mbar) {
   asm volatile(
@@ -93,12 +87,15 @@ dense_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant_
   const __half2 zero2 = __float2half2_rn(0.f);
   const uint32_t zero = *reinterpret_cast<const uint32_t*>(&zero2);
 
+  // items are dealt across the blocks first (item blockIdx.x + gridDim.x (warp + WARPS k)), so that a launch with
+  // fewer items than workers still spreads them over every SM
   const int workers = gridDim.x * P::WARPS;
+  const int first = blockIdx.x + gridDim.x * warp;
   const int items = a.B * a.Hkv * a.splits;
   uint32_t seq = 0;  // tiles this warp has consumed: stage seq % NS, phase parity (seq / NS) & 1
   bool failed = false;
 
-  for (int item = blockIdx.x * P::WARPS + warp; item < items && !failed; item += workers) {
+  for (int item = first; item < items && !failed; item += workers) {
     const int split = item % a.splits;
     const int hk = (item / a.splits) % a.Hkv;
     const int b = item / (a.splits * a.Hkv);
@@ -264,7 +261,7 @@ dense_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant_
 
   if (failed) {
     // poison every partial this warp owns (the merge then yields NaN) and record the failure in the status word
-    for (int item = blockIdx.x * P::WARPS + warp; item < items; item += workers) {
+    for (int item = first; item < items; item += workers) {
       const int split = item % a.splits;
       const int hk = (item / a.splits) % a.Hkv;
       const int b = item / (a.splits * a.Hkv);

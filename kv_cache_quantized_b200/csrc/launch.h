@@ -3,6 +3,8 @@
 // arguments and picks the family.
 #pragma once
 
+#include <cuda.h>
+
 #include "decode.cuh"
 
 namespace axr {
@@ -48,8 +50,19 @@ axr_status attend_rows_launch(int d, int bits, int G, bool vq, const DecodeArgs&
 axr_status attend_partial_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st,
                                  const char* what);
 
+// 2-D TMA map over an fp16 cache viewed as [rows, D]: boxes of `box_rows` rows x 64 coordinates, 128-byte swizzle
+// (dense.cu).
+axr_status encode_cache_map(CUtensorMap* map, const void* base, size_t rows, int D, int box_rows, const char* what);
+
+// Quantized keys over fp16 (vq false) or quantized row-layout values on contiguous caches, as a stream of per-warp
+// workers (attend_stream.cu); decode steps included.  Code rows of whole 16-byte chunks only
+// (attend_stream_supported); the arguments carry the plan_splits_stream split plan for kAttendStreamWorkers.
+bool attend_stream_supported(int d, int bits);
+axr_status attend_stream_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st,
+                                const char* what);
+
 // Unquantized fp16 keys and values (dense.cu): the dense bandwidth reference, one streaming worker per warp; the
-// arguments carry the plan_splits_dense split plan.
+// arguments carry the plan_splits_stream split plan for kDenseWorkers.
 axr_status dense_launch(int d, int G, const DecodeArgs& a, cudaStream_t st, const char* what);
 
 // Tiled value layout, d = 128 (attend_tiled.cu): tcgen05 kernel if tensor, else warp-level MMAs.

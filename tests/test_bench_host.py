@@ -46,3 +46,13 @@ def test_algorithmic_bytes_per_key_head():
     # writes: at least the algorithmic bytes, and no re-reads beyond a percent or two
     ratio = bench.TRAFFIC[w.name] / (units * bench._bytes_per_key_head(w))
     assert 1.0 <= ratio <= 1.02, ratio
+
+
+def test_step_kernel_label_follows_the_library_routing():
+    """The bench line names the decode kernel the library picks for a contiguous step: the row kernel for the
+    long-context step with quantized values (G = 4, 64 units), the streaming kernel for fp16 values."""
+    import dataclasses
+    assert bench._step_kernel(W.LONG_CONTEXT) == "attend_rows_kernel"
+    assert bench._step_kernel(W.LLAMA8B_DECODE) == "attend_stream_kernel"
+    assert bench._step_kernel(dataclasses.replace(W.LONG_CONTEXT, B=64)) == "attend_stream_kernel"
+    assert bench._step_kernel(dataclasses.replace(W.LONG_CONTEXT, Hq=64)) == "attend_stream_kernel"

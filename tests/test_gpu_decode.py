@@ -221,12 +221,14 @@ def test_decode_step(vq, d, bits, G, Tcap):
     parity.check_outputs(out, want)
 
 
+@pytest.mark.parametrize("B,T", [(8, 4096), (40, 512)])
 @pytest.mark.parametrize("vq", [False, True])
-def test_decode_step_many_items(vq):
+def test_decode_step_many_items(vq, B, T):
     """More (batch row, KV head, split) items than resident blocks, ragged rows (one full, one of a single token):
     blocks carry several items, some of them holding a new token.  The step writes each token exactly as
-    axr_write_keys does and gives the output of attend over the completed cache."""
-    B, Hkv, G, T, d, bits = 8, 8, 4, 4096, 128, 4
+    axr_write_keys does and gives the output of attend over the completed cache.  B = 40 gives 320 (batch row,
+    KV head) units: quantized values then take the streaming kernel too."""
+    Hkv, G, d, bits = 8, 4, 128, 4
     Tcap = T + 8
     Hq = Hkv * G
     rng = np.random.default_rng(977)
@@ -265,6 +267,30 @@ def test_decode_step_many_items(vq):
     num = torch.linalg.vector_norm(out - again, dim=-1)
     den = torch.linalg.vector_norm(again, dim=-1)
     assert bool(torch.all(num <= 2.0 ** -11 * den)), float((num / den).max())
+
+
+@pytest.mark.parametrize("d,bits", [(128, 4), (128, 2), (64, 4)])
+def test_attend_many_units_quantized_values(d, bits):
+    """Quantized values over more (batch row, KV head) units than the row kernel keeps resident (B = 40, Hkv = 8):
+    the streaming kernel's quantized-value path, ragged rows, against the oracle on sampled batch rows."""
+    B, Hkv, G, T, Tcap = 40, 8, 4, 300, 320
+    Hq = Hkv * G
+    k = W.lognormal_rows((B, Hkv, T, d), 1200 + d + bits, dtype=np.float16)
+    v = W.lognormal_rows((B, Hkv, T, d), 1201 + d + bits, dtype=np.float16)
+    s = W.sign_vector(d, 1202)
+    q = W.normal((B, Hq, d), 1203, np.float32)
+    lens = np.random.default_rng(1204).integers(1, T + 1, size=B).astype(np.int32)
+    lens[0], lens[1], lens[2] = T, 1, 0
+    kc, kn = oracle.write(k, s, bits)
+    vc, vn = oracle.write(v, s, bits)
+    out = ops.attend_decode(cuda(q), cuda(padded(kc, Tcap)), cuda(padded(kn, Tcap)), cuda(s), bits,
+                            vcodes=cuda(padded(vc, Tcap)), vnorms=cuda(padded(vn, Tcap)), seq_lens=cuda(lens),
+                            T=T).cpu().numpy()
+    assert np.all(out[2] == 0)
+    for b in [0, 1, 5, 17, 39]:
+        want = oracle.decode_attention(q[b:b + 1], kc[b:b + 1], kn[b:b + 1], s, bits, 1.0 / math.sqrt(d),
+                                       vcodes=vc[b:b + 1], vn16=vn[b:b + 1], seq_lens=lens[b:b + 1])
+        parity.check_outputs(out[b:b + 1], want)
 
 
 @pytest.mark.parametrize("d,G,Hkv", [(128, 4, 2), (64, 8, 1), (128, 1, 3), (64, 2, 2), (128, 8, 1)])

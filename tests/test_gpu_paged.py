@@ -73,15 +73,13 @@ def test_paged_attend_matches_oracle_and_contiguous(d, bits, G, bt, vq):
     out = ops.attend_decode_paged(tq, cuda(kcp), cuda(knp), st, bits, tt, seq_lens=tl, T=T, **vargs).cpu().numpy()
     parity.check_outputs(out, want)
     assert np.all(out[1] != 0) and np.all(np.isfinite(out))
-    # the contiguous cache through the library gives the same result (bit for bit for quantized values: the same
-    # kernel and split plan; fp16 values may take another kernel)
+    # the contiguous cache through the library gives the same result up to rounding: it may take the streaming
+    # kernel (other split points).  fp16 values carry fp32-level weights there; quantized values carry fp16 weights
+    # p n^V / sqrt(d) in both kernels, each rounded to half an fp16 ulp (2^-11) against its own split maxima.
     ref = ops.attend_decode(tq, cuda(kc), cuda(kn), st, bits, seq_lens=tl, T=T, **cargs).cpu().numpy()
-    if vq:
-        assert np.array_equal(out, ref)
-    else:
-        num = np.linalg.norm((out - ref).reshape(-1, d), axis=1)
-        den = np.linalg.norm(ref.reshape(-1, d), axis=1)
-        assert np.all(num <= 2.0 ** -11 * den)
+    num = np.linalg.norm((out - ref).reshape(-1, d), axis=1)
+    den = np.linalg.norm(ref.reshape(-1, d), axis=1)
+    assert np.all(num <= (2.0 ** -10 if vq else 2.0 ** -11) * den), float(np.max(num / den))
 
 
 @pytest.mark.parametrize("vq", [False, True])
