@@ -42,7 +42,12 @@ axr_status by_g(int G, bool vq, const DecodeArgs& a, cudaStream_t st, const char
 
 }  // namespace
 
-bool attend_stream_supported(int d, int bits) { return (d == 128 || d == 64) && d * bits % 128 == 0; }
+// Code rows of whole 16-byte chunks, or (d = 64, b = 1, 3: rows of 8 or 24 bytes) an even capacity, so that every
+// (batch row, KV head) starts on a 16-byte boundary and a tile's rows, rounded up to an even count, stay inside it.
+bool attend_stream_supported(int d, int bits, int Tcap) {
+  if (d == 128) return bits >= 1 && bits <= 4;
+  return d == 64 && bits >= 1 && bits <= 4 && (d * bits % 128 == 0 || Tcap % 2 == 0);
+}
 
 axr_status attend_stream_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st,
                                 const char* what) {
@@ -55,7 +60,9 @@ axr_status attend_stream_launch(int d, int bits, int G, bool vq, const DecodeArg
     }
   } else if (d == 64) {
     switch (bits) {
+      case 1: return by_g<64, 1>(G, vq, a, st, what);
       case 2: return by_g<64, 2>(G, vq, a, st, what);
+      case 3: return by_g<64, 3>(G, vq, a, st, what);
       case 4: return by_g<64, 4>(G, vq, a, st, what);
     }
   }

@@ -52,7 +52,7 @@ struct StreamPlan {
   static constexpr int MTV = D / 16;                     // m-tiles of the value product (16 coordinates)
   static constexpr int NBV = R / 8;                      // quantized values: bytes of lane g's run of a row
   static constexpr int NWV = (NBV + 3) / 4 + 1;          // its words, plus a zero word
-  static_assert(R % 16 == 0, "key code rows of whole 16-byte chunks (one bulk copy per tile)");
+  static_assert(R % 8 == 0 && (TW * R) % 16 == 0, "tiles of code rows in whole 16-byte chunks");
   static_assert(TW == 32, "two 16-token groups per tile");
   static_assert(bytes <= 227 * 1024, "shared memory of one block");
 };
@@ -153,18 +153,20 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         const int s = static_cast<int>((seq + i) % NS);
         uint8_t* st = ring + static_cast<size_t>(s) * P::STAGE;
         const int t0 = start + i * TW;
-        const int n = min(TW, end - t0);
+        // the tile's code rows, rounded up to whole 16-byte chunks: with rows of 8 or 24 bytes (d = 64, b = 1, 3)
+        // an odd row count takes one row more, which lies inside the row's capacity (the launcher requires Tcap
+        // even, and a tile that ends at Tcap has an even row count)
+        const uint32_t cb = static_cast<uint32_t>((min(TW, end - t0) * R + 15) / 16 * 16);
         if constexpr (VQ) {
-          mbar_arrive_expect_tx(mbar + s, static_cast<uint32_t>(2 * n * R));
-          bulk_copy_g2s(st, static_cast<const uint8_t*>(a.v) + (row0 + t0) * R, static_cast<uint32_t>(n * R),
-                        mbar + s);
+          mbar_arrive_expect_tx(mbar + s, 2 * cb);
+          bulk_copy_g2s(st, static_cast<const uint8_t*>(a.v) + (row0 + t0) * R, cb, mbar + s);
         } else {
-          mbar_arrive_expect_tx(mbar + s, static_cast<uint32_t>(P::VPLANE + n * R));
+          mbar_arrive_expect_tx(mbar + s, static_cast<uint32_t>(P::VPLANE) + cb);
 #pragma unroll
           for (int bx = 0; bx < P::NBX; ++bx)
             tma_load_2d(st + bx * P::BOX, &vmap, bx * P::BOXC, static_cast<int>(row0) + t0, mbar + s);
         }
-        bulk_copy_g2s(st + P::VPLANE, a.kcodes + (row0 + t0) * R, static_cast<uint32_t>(n * R), mbar + s);
+        bulk_copy_g2s(st + P::VPLANE, a.kcodes + (row0 + t0) * R, cb, mbar + s);
       }
     };
     for (int i = 0; i < NS && i < ntiles; ++i) issue(i);
@@ -179,23 +181,26 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) { m_run[nt] = -INFINITY; l_lane[nt] = 0.f; }
 
-    // key (and value) norms of this lane's tokens (16 m + g + 8 i of a tile) times 1 / sqrt(D), one tile ahead;
-    // L2-only loads, since a decode step writes one of them in this launch
-    auto load_norms = [&](int i, float (&kn)[2][2], float (&vn)[2][2]) {
+    // key (and value) norms of this lane's tokens (16 m + g + 8 i of a tile), one tile ahead, kept as raw fp16 bits
+    // (key | value << 16) until the tile that uses them, so that the loads have a whole tile to land; L2-only
+    // loads, since a decode step writes one of them in this launch
+    auto load_norms = [&](int i, uint32_t (&nr)[2][2]) {
       const int t0 = start + i * TW;
 #pragma unroll
       for (int m = 0; m < 2; ++m)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int tok = t0 + 16 * m + g + 8 * e;
-          const bool in = i < ntiles && tok < end;
-          kn[m][e] = in ? __half2float(__ldcg(a.knorms + row0 + tok)) * rd : 0.f;
-          if constexpr (VQ) vn[m][e] = in ? __half2float(__ldcg(a.vnorms + row0 + tok)) * rd : 0.f;
-          else vn[m][e] = 1.f;
+          uint32_t r = 0u;  // norms 0 past the end (fp16 +0)
+          if (i < ntiles && tok < end) {
+            r = __half_as_ushort(__ldcg(a.knorms + row0 + tok));
+            if constexpr (VQ) r |= static_cast<uint32_t>(__half_as_ushort(__ldcg(a.vnorms + row0 + tok))) << 16;
+          }
+          nr[m][e] = r;
         }
     };
-    float kn_next[2][2], vn_next[2][2];
-    load_norms(0, kn_next, vn_next);
+    uint32_t nr_next[2][2];
+    load_norms(0, nr_next);
 
     for (int i = 0; i < ntiles; ++i) {
       const int s = static_cast<int>((seq + i) % NS);
@@ -208,12 +213,16 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
       uint8_t* st = ring + static_cast<size_t>(s) * P::STAGE;
       const uint32_t sV = smem_u32(st);
       const int t0 = start + i * TW;
-      float kn[2][2], vn[2][2];
+      float kn[2][2], vn[2][2];  // times the centroid scale 1 / sqrt(D)
 #pragma unroll
       for (int m = 0; m < 2; ++m)
 #pragma unroll
-        for (int e = 0; e < 2; ++e) { kn[m][e] = kn_next[m][e]; vn[m][e] = vn_next[m][e]; }
-      load_norms(i + 1, kn_next, vn_next);
+        for (int e = 0; e < 2; ++e) {
+          const uint32_t r = nr_next[m][e];
+          kn[m][e] = __half2float(__ushort_as_half(static_cast<unsigned short>(r & 0xffffu))) * rd;
+          vn[m][e] = VQ ? __half2float(__ushort_as_half(static_cast<unsigned short>(r >> 16))) * rd : 1.f;
+        }
+      load_norms(i + 1, nr_next);
       if (!VQ && t0 + TW > end) {
         // the row ends inside this tile: zero the value rows past it (whatever the cache holds there); the key
         // rows past it are stale codes, valid table indices, whose scores are masked

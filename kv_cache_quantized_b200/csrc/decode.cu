@@ -133,7 +133,7 @@ axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, con
   // KV head, or more (batch row, KV head) units than attend_rows has resident blocks), else attend_rows, which is
   // ahead at four query heads per KV head and few units (the long-context step: 120 against 127 us)
   const bool stream_vq = vkind == AXR_V_QUANT && (Hq / Hkv == 8 || static_cast<long>(B) * Hkv > kResident);
-  const bool stream_path = (vkind == AXR_V_F16 || stream_vq) && !paged && attend_stream_supported(d, bits) &&
+  const bool stream_path = (vkind == AXR_V_F16 || stream_vq) && !paged && attend_stream_supported(d, bits, Tcap) &&
                            (step || mode == kGatherMma || mode == kGatherDirect);
   if (stream_path) {
     const SplitPlan p =

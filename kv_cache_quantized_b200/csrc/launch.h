@@ -55,9 +55,9 @@ axr_status attend_partial_launch(int d, int bits, int G, bool vq, const DecodeAr
 axr_status encode_cache_map(CUtensorMap* map, const void* base, size_t rows, int D, int box_rows, const char* what);
 
 // Quantized keys over fp16 (vq false) or quantized row-layout values on contiguous caches, as a stream of per-warp
-// workers (attend_stream.cu); decode steps included.  Code rows of whole 16-byte chunks only
-// (attend_stream_supported); the arguments carry the plan_splits_stream split plan for kAttendStreamWorkers.
-bool attend_stream_supported(int d, int bits);
+// workers (attend_stream.cu); decode steps included.  Code rows of whole 16-byte chunks, or an even capacity
+// (attend_stream_supported); the arguments carry the plan_splits_stream split plan for its worker count.
+bool attend_stream_supported(int d, int bits, int Tcap);
 axr_status attend_stream_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st,
                                 const char* what);
 

@@ -159,11 +159,12 @@ def test_unaligned_norm_rows(vq):
 
 @pytest.mark.parametrize("vq", [False, True])
 @pytest.mark.parametrize("d,bits,G,Tcap", [(128, 4, 4, 912), (64, 2, 8, 912), (128, 3, 1, 912), (128, 4, 4, 1003),
-                                           (64, 2, 8, 1003)])
+                                           (64, 2, 8, 1003), (64, 3, 4, 912), (64, 1, 2, 1003)])
 def test_decode_step(vq, d, bits, G, Tcap):
     """axr_decode_step writes the new token exactly as axr_write_keys does and attends over it: the same bits in the
     cache, the same output as a separate append + attend, and parity with the oracle over the full cache.  Tcap 1003
-    leaves the norm rows unaligned (norms read from global memory rather than staged with the tiles)."""
+    leaves the norm rows unaligned (norms read from global memory rather than staged with the tiles); with rows of
+    8 or 24 bytes (d = 64, b = 1, 3) an even capacity takes the streaming kernel and an odd one the row kernel."""
     B, Hkv, T = 3, 2, 900
     Hq = Hkv * G
     k, v, s, kc, kn, vc, vn = oracle_cache(B, Hkv, T, d, bits, 950 + d + bits + G, vq)
