@@ -74,15 +74,13 @@ def _lead_in():
 
 def _step_kernel(w) -> str:
     """The decode kernel the library runs for a contiguous decode step of this workload: the streaming kernel for
-    fp16 values, and for quantized values at eight query heads per KV head or more than 296 (batch row, KV head)
-    units; the row kernel otherwise."""
-    stream = (not w.v_quant) or w.Hq // w.Hkv == 8 or w.B * w.Hkv > 296
+    fp16 values, and for quantized values from 2^18 (token, KV head) units or at eight query heads per KV head; the
+    row kernel otherwise."""
+    stream = (not w.v_quant) or w.Hq // w.Hkv == 8 or w.B * w.Hkv * w.T >= 1 << 18
     return "attend_stream_kernel" if stream else "attend_rows_kernel"
 
 
-TRAFFIC = {
-    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.581845e6 + 1.457408e6),
-}
+TRAFFIC = {}
 
 WORKLOADS = {
     "long_context": W.LONG_CONTEXT,

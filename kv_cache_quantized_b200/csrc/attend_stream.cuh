@@ -9,11 +9,13 @@
 //   fp16 values: A = V^T, read with ldmatrix.trans from the 128-byte-swizzled TMA boxes of the value rows; B = P^T
 //       as hi and lo fp16 planes (fp32-level weights, so that the result does not depend on where the splits fall),
 //       gathered from the score lanes with four shuffles per 16 tokens;
-//   quantized values: A = V^T from the hi-only copies of the key/value pair table (one lookup of a code byte gives
-//       the fp16 pair (v_2p, v_2p+1) of a token; two byte permutes of the pairs of tokens k and k + 1 give two A
-//       registers, as in attend_rows.cuh); B = P^T times the value norm and 1 / sqrt(D), fp16 (the table's hi plane
-//       holds the centroids to 2^-11); the product stays in the rotated domain and the merge applies the one inverse
-//       transform.
+//   quantized values: the contraction runs over (token t, half s) and the columns over (head h, half s'), with
+//       A[p][(t, s)] = v_t,2p+s and B[(t, s)][(h, s')] = [s = s'] p_t,h n^V_t / sqrt(D), so that
+//       C[p][(h, s')] = O^T[2 p + s'][h]: one lookup in the hi-only copies of the key/value pair table (the fp16
+//       pair (v_2p, v_2p+1) of a token's code byte) is one A register as it is, and B is P^T with a zero beside
+//       every weight.  An MMA covers 16 coordinate pairs x 8 tokens x 4 heads; fp16 weights (the table's hi plane
+//       holds the centroids to 2^-11); the product stays in the rotated domain and the merge applies the one
+//       inverse transform.
 //
 // Every warp is an independent worker over (batch row, KV head, split) items with a ring of NS stages of its own: a
 // stage holds TW tokens' value rows (fp16: D / 64 tiled TMA boxes; quantized: one bulk copy of code rows) and key
@@ -50,7 +52,8 @@ struct StreamPlan {
   static constexpr size_t bytes = 1024 + OFF_MBAR + (size_t)WARPS * NS * 8;  // + the alignment slack
   static constexpr int NT = MmaB<D, G>::NT;              // n-tiles of heads (2: heads 4..7)
   static constexpr int MTV = D / 16;                     // m-tiles of the value product (16 coordinates)
-  static constexpr int NBV = R / 8;                      // quantized values: bytes of lane g's run of a row
+  static constexpr int MPQ = D / 32;                     // quantized values: m-tiles of 16 coordinate pairs
+  static constexpr int NBV = R / 8;                      // bytes of lane g's run of a row: pairs D/16 g .. + D/16
   static constexpr int NWV = (NBV + 3) / 4 + 1;          // its words, plus a zero word
   static_assert(R % 8 == 0 && (TW * R) % 16 == 0, "tiles of code rows in whole 16-byte chunks");
   static_assert(TW == 32, "two 16-token groups per tile");
@@ -87,10 +90,6 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
   // the lane's key copy in the pair table, and (quantized values) its hi-only value copy
   const uint32_t repk = static_cast<uint32_t>(lane & 15) << (VQ ? 3 : 4);
   const uint32_t repv = 128u + (static_cast<uint32_t>(lane) << 2);
-  // quantized values: lanes with odd t fetch token k + 1 before k (rows of both parities in every half-warp: no bank
-  // conflicts), so their byte permutes take the two pairs the other way round
-  const int tf = t & 1;
-  const uint32_t sel_lo = tf ? 0x1054u : 0x5410u, sel_hi = tf ? 0x3276u : 0x7632u;
   const int a_row = (lane & 7) + 8 * (lane >> 4), a_col = 8 * ((lane >> 3) & 1);  // ldmatrix.trans rows of V^T
   const float rd = rsqrtf(static_cast<float>(D));
   // items are dealt across the blocks first (item blockIdx.x + gridDim.x (warp + WARPS k)), so that a launch with
@@ -171,12 +170,19 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     };
     for (int i = 0; i < NS && i < ntiles; ++i) issue(i);
 
-    // O^T: (coordinate 16 mt + g (+ 8), head 2 t (+ 1)); quantized values: coordinates 2 (MTV g + mt) (+ 1)
-    float acc[MTV][4];
+    // fp16 values: O^T (coordinate 16 mt + g (+ 8), head 2 t (+ 1)); quantized values: head 4 nt + t, coordinates
+    // D/8 g + 4 mt + e
+    float acc[MTV][4], accq[NT][P::MPQ][4];
 #pragma unroll
     for (int mt = 0; mt < MTV; ++mt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[mt][e] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int mt = 0; mt < P::MPQ; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) accq[nt][mt][e] = 0.f;
     float m_run[NT], l_lane[NT];  // head 4 nt + t
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) { m_run[nt] = -INFINITY; l_lane[nt] = 0.f; }
@@ -275,7 +281,14 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
       bool moved = false;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) moved |= alpha[nt] != 1.f;
-      if (__any_sync(0xffffffffu, moved)) {
+      if (VQ && __any_sync(0xffffffffu, moved)) {  // this lane's columns are its own heads 4 nt + t
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < P::MPQ; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) accq[nt][mt][e] *= alpha[nt];
+      } else if (!VQ && __any_sync(0xffffffffu, moved)) {
         float al[2];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
@@ -294,6 +307,41 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         }
       }
 
+      if constexpr (VQ) {
+        // ---- O^T += V^T P^T per 8 tokens: lane (g, t) takes tokens t and t + 4 of the step (A columns 2 t, 2 t + 1
+        // and 2 t + 8, 2 t + 9) and pairs D/16 g + 2 mt (A row g) and + 1 (row g + 8) of m-tile mt
+#pragma unroll
+        for (int m = 0; m < 2; ++m)
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks) {
+            const int ta = 16 * m + 8 * ks + t;  // the step's token t; token t + 4 is ta + 4
+            uint32_t b0[NT], b1[NT];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+              // weights of tokens ta, ta + 4 for head 4 nt + g / 2: held by lanes (t, g / 2) and (t + 4, g / 2) as
+              // their token 16 m + g' + 8 ks
+              const float w = z[m][nt][ks] * vn[m][ks];
+              const float xa = __shfl_sync(0xffffffffu, w, 4 * t + (g >> 1));
+              const float xb = __shfl_sync(0xffffffffu, w, 4 * (t + 4) + (g >> 1));
+              b0[nt] = (g & 1) ? pack_h2(0.f, xa) : pack_h2(xa, 0.f);
+              b1[nt] = (g & 1) ? pack_h2(0.f, xb) : pack_h2(xb, 0.f);
+            }
+            uint32_t wa[P::NWV], wb[P::NWV];
+            load_run<R, P::NBV, false>(st, ta * R + g * P::NBV, wa);
+            load_run<R, P::NBV, false>(st, (ta + 4) * R + g * P::NBV, wb);
+#pragma unroll
+            for (int x = (P::NBV + 3) / 4; x < P::NWV; ++x) wa[x] = wb[x] = 0u;
+#pragma unroll
+            for (int mt = 0; mt < P::MPQ; ++mt) {
+              const uint32_t a0 = *reinterpret_cast<const uint32_t*>(tab + kv_off<BITS>(wa, 2 * mt, repv));
+              const uint32_t a1 = *reinterpret_cast<const uint32_t*>(tab + kv_off<BITS>(wa, 2 * mt + 1, repv));
+              const uint32_t a2 = *reinterpret_cast<const uint32_t*>(tab + kv_off<BITS>(wb, 2 * mt, repv));
+              const uint32_t a3 = *reinterpret_cast<const uint32_t*>(tab + kv_off<BITS>(wb, 2 * mt + 1, repv));
+#pragma unroll
+              for (int nt = 0; nt < NT; ++nt) mma16816(accq[nt][mt], a0, a1, a2, a3, b0[nt], b1[nt]);
+            }
+          }
+      } else {
       // ---- O^T += V^T P^T per 16-token group: B = P^T (tokens 2 t, 2 t + 1 | + 8, + 9; head g)
 #pragma unroll
       for (int m = 0; m < 2; ++m) {
@@ -303,48 +351,26 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int src = 4 * (2 * t + u) + (g & 3);  // the lane holding token 2 t + u (+ 8 e) of head g % 4 (+ 4)
-            float x = __shfl_sync(0xffffffffu, z[m][0][e] * vn[m][e], src);
+            float x = __shfl_sync(0xffffffffu, z[m][0][e], src);
             if constexpr (NT > 1) {
-              const float y = __shfl_sync(0xffffffffu, z[m][NT - 1][e] * vn[m][e], src);
+              const float y = __shfl_sync(0xffffffffu, z[m][NT - 1][e], src);
               x = g >= 4 ? y : x;
             } else {
               x = g < G ? x : 0.f;
             }
             pv[e][u] = x;
           }
-        if constexpr (VQ) {
-          // the weights p n^V / sqrt(D) in fp16; A = V^T from the value codes of tokens k0, k0 + 1, k0 + 8, k0 + 9
-          const uint32_t b0 = pack_h2(pv[0][0], pv[0][1]), b1 = pack_h2(pv[1][0], pv[1][1]);
-          const int k0 = 16 * m + 2 * t;
-          uint32_t w[4][P::NWV];
-          load_run<R, P::NBV, false>(st, (k0 + tf) * R + g * P::NBV, w[0]);
-          load_run<R, P::NBV, false>(st, (k0 + 1 - tf) * R + g * P::NBV, w[1]);
-          load_run<R, P::NBV, false>(st, (k0 + 8 + tf) * R + g * P::NBV, w[2]);
-          load_run<R, P::NBV, false>(st, (k0 + 9 - tf) * R + g * P::NBV, w[3]);
+        uint32_t bh0, bl0, bh1, bl1;
+        split_h2(pv[0][0], pv[0][1], bh0, bl0);
+        split_h2(pv[1][0], pv[1][1], bh1, bl1);
 #pragma unroll
-          for (int r = 0; r < 4; ++r)
-#pragma unroll
-            for (int x = (P::NBV + 3) / 4; x < P::NWV; ++x) w[r][x] = 0u;
-#pragma unroll
-          for (int mt = 0; mt < MTV; ++mt) {
-            uint32_t x[4];  // hi fp16 pairs (v_2p, v_2p+1) of the four tokens, p = MTV g + mt
-#pragma unroll
-            for (int r = 0; r < 4; ++r) x[r] = *reinterpret_cast<const uint32_t*>(tab + kv_off<BITS>(w[r], mt, repv));
-            mma16816(acc[mt], __byte_perm(x[0], x[1], sel_lo), __byte_perm(x[0], x[1], sel_hi),
-                     __byte_perm(x[2], x[3], sel_lo), __byte_perm(x[2], x[3], sel_hi), b0, b1);
-          }
-        } else {
-          uint32_t bh0, bl0, bh1, bl1;
-          split_h2(pv[0][0], pv[0][1], bh0, bl0);
-          split_h2(pv[1][0], pv[1][1], bh1, bl1);
-#pragma unroll
-          for (int mt = 0; mt < MTV; ++mt) {
-            uint32_t va[4];
-            ldsm_x4_t(sV + swz<TW>(16 * m + a_row, 16 * mt + a_col), va[0], va[1], va[2], va[3]);
-            mma16816(acc[mt], va[0], va[1], va[2], va[3], bh0, bh1);
-            mma16816(acc[mt], va[0], va[1], va[2], va[3], bl0, bl1);
-          }
+        for (int mt = 0; mt < MTV; ++mt) {
+          uint32_t va[4];
+          ldsm_x4_t(sV + swz<TW>(16 * m + a_row, 16 * mt + a_col), va[0], va[1], va[2], va[3]);
+          mma16816(acc[mt], va[0], va[1], va[2], va[3], bh0, bh1);
+          mma16816(acc[mt], va[0], va[1], va[2], va[3], bl0, bl1);
         }
+      }
       }
 
       // the stage is free once every lane's reads (and zeroing writes) of it are done: each lane orders its own
@@ -369,16 +395,29 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         a.ws_l[part0 + static_cast<size_t>(h) * a.splits] = l;
       }
     }
+    if constexpr (VQ) {
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const int h = 2 * t + c;
-      if (h < G) {
-        float* dst = a.ws_o + (part0 + static_cast<size_t>(h) * a.splits) * D;
+      for (int nt = 0; nt < NT; ++nt) {
+        const int h = 4 * nt + t;
+        if (h < G) {
+          float* dst = a.ws_o + (part0 + static_cast<size_t>(h) * a.splits) * D + (D / 8) * g;
 #pragma unroll
-        for (int mt = 0; mt < MTV; ++mt) {
-          const int r0 = VQ ? 2 * (MTV * g + mt) : 16 * mt + g, r1 = VQ ? r0 + 1 : r0 + 8;
-          dst[r0] = acc[mt][c];
-          dst[r1] = acc[mt][2 + c];
+          for (int mt = 0; mt < P::MPQ; ++mt)
+            *reinterpret_cast<float4*>(dst + 4 * mt) =
+                make_float4(accq[nt][mt][0], accq[nt][mt][1], accq[nt][mt][2], accq[nt][mt][3]);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int h = 2 * t + c;
+        if (h < G) {
+          float* dst = a.ws_o + (part0 + static_cast<size_t>(h) * a.splits) * D;
+#pragma unroll
+          for (int mt = 0; mt < MTV; ++mt) {
+            dst[16 * mt + g] = acc[mt][c];
+            dst[16 * mt + g + 8] = acc[mt][2 + c];
+          }
         }
       }
     }

@@ -129,10 +129,11 @@ axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, con
   DecodeArgs a = base_args(B, Hq, Hkv, T, Tcap, seq_lens, q, scale * kLog2e);
   const int mode = g_gather.load();
   // row-layout values on a contiguous cache, keys through warp-level MMAs (attend and decode step): the streaming
-  // kernel for fp16 values; for quantized values where it measured faster than attend_rows (eight query heads per
-  // KV head, or more (batch row, KV head) units than attend_rows has resident blocks), else attend_rows, which is
-  // ahead at four query heads per KV head and few units (the long-context step: 120 against 127 us)
-  const bool stream_vq = vkind == AXR_V_QUANT && (Hq / Hkv == 8 || static_cast<long>(B) * Hkv > kResident);
+  // kernel; for quantized values only from 2^18 (token, KV head) units or at eight query heads per KV head, since
+  // below that the row kernel's shorter setup measured ahead (B = 1, T = 4096: 21.5 against 25.6 us; the
+  // long-context step: 107 against 122 us the other way)
+  const bool stream_vq = vkind == AXR_V_QUANT &&
+                         (Hq / Hkv == 8 || static_cast<long>(B) * Hkv * T >= (1L << 18));
   const bool stream_path = (vkind == AXR_V_F16 || stream_vq) && !paged && attend_stream_supported(d, bits, Tcap) &&
                            (step || mode == kGatherMma || mode == kGatherDirect);
   if (stream_path) {
@@ -158,13 +159,9 @@ axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, con
   if (vkind == AXR_V_QUANT_TILED) return attend_tiled_launch(bits, G, mode == kGatherTensor, a, as_stream(stream));
   // fp16 values in AXR_GATHER_TABLE mode: the literal table in shared memory, values on the CUDA cores
   if (mode == kGatherTable && !vq) return table_attend_launch(d, bits, G, a, as_stream(stream));
-  // row-layout values: keys scored through warp-level MMAs in AXR_GATHER_MMA mode, else on CUDA cores
-  if (mode == kGatherMma || mode == kGatherDirect) {
-    // fp16 values: one warp per token range through scores, softmax and the value product (no block barrier);
-    // quantized values: scoring and value warps one tile apart
-    if (!vq && attend_fused_supported(d, bits)) return attend_fused_launch(d, bits, G, vq, a, as_stream(stream));
-    return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));
-  }
+  // row-layout values the streaming kernel does not take: keys scored through warp-level MMAs in AXR_GATHER_MMA
+  // mode (scoring and value warps one tile apart), else on CUDA cores
+  if (mode == kGatherMma || mode == kGatherDirect) return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));
   return attend_partial_launch(d, bits, G, vq, a, as_stream(stream), w);
 }
 }  // namespace

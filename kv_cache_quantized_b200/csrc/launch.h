@@ -38,11 +38,6 @@ void launch_reduce(const DecodeArgs& a, cudaStream_t st) {
   cudaLaunchKernelEx(&cfg, attend_reduce_kernel<D, VQ, EXACT>, a);
 }
 
-// Row-layout cache, one warp per token range through scores, softmax and the value product, all as warp-level MMAs
-// (attend_fused.cu); only for rows of whole 16-byte chunks (attend_fused_supported).  Used for fp16 values.
-bool attend_fused_supported(int d, int bits);
-axr_status attend_fused_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st);
-
 // Row-layout cache, quantized keys scored through warp-level MMAs (attend_rows.cu); vq: values quantized.
 axr_status attend_rows_launch(int d, int bits, int G, bool vq, const DecodeArgs& a, cudaStream_t st);
 

@@ -222,13 +222,13 @@ def test_decode_step(vq, d, bits, G, Tcap):
     parity.check_outputs(out, want)
 
 
-@pytest.mark.parametrize("B,T", [(8, 4096), (40, 512)])
+@pytest.mark.parametrize("B,T", [(8, 4096), (40, 1024)])
 @pytest.mark.parametrize("vq", [False, True])
 def test_decode_step_many_items(vq, B, T):
     """More (batch row, KV head, split) items than resident blocks, ragged rows (one full, one of a single token):
     blocks carry several items, some of them holding a new token.  The step writes each token exactly as
-    axr_write_keys does and gives the output of attend over the completed cache.  B = 40 gives 320 (batch row,
-    KV head) units: quantized values then take the streaming kernel too."""
+    axr_write_keys does and gives the output of attend over the completed cache.  Both shapes hold at least 2^18
+    (token, KV head) units, so quantized values take the streaming kernel as fp16 values do."""
     Hkv, G, d, bits = 8, 4, 128, 4
     Tcap = T + 8
     Hq = Hkv * G
@@ -272,9 +272,10 @@ def test_decode_step_many_items(vq, B, T):
 
 @pytest.mark.parametrize("d,bits", [(128, 4), (128, 2), (64, 4)])
 def test_attend_many_units_quantized_values(d, bits):
-    """Quantized values over more (batch row, KV head) units than the row kernel keeps resident (B = 40, Hkv = 8):
-    the streaming kernel's quantized-value path, ragged rows, against the oracle on sampled batch rows."""
-    B, Hkv, G, T, Tcap = 40, 8, 4, 300, 320
+    """Quantized values over 40 x 8 x 1024 >= 2^18 (token, KV head) units: the streaming kernel's quantized-value
+    path at four query heads per KV head, ragged rows (empty, one token, full), against the oracle on sampled batch
+    rows."""
+    B, Hkv, G, T, Tcap = 40, 8, 4, 1024, 1040
     Hq = Hkv * G
     k = W.lognormal_rows((B, Hkv, T, d), 1200 + d + bits, dtype=np.float16)
     v = W.lognormal_rows((B, Hkv, T, d), 1201 + d + bits, dtype=np.float16)
