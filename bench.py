@@ -80,7 +80,11 @@ def _step_kernel(w) -> str:
     return "attend_stream_kernel" if stream else "attend_rows_kernel"
 
 
-TRAFFIC = {}
+TRAFFIC = {
+    # attend_stream_kernel<128, 4, 4, quantized V>, DRAM read + write per launch at B = 4 (mean of three launches,
+    # profiles/attend_stream_long_context.md), scaled by the units to B = 8
+    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.777003e6 + 1.149867e6),
+}
 
 WORKLOADS = {
     "long_context": W.LONG_CONTEXT,

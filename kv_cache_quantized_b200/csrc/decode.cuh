@@ -655,27 +655,64 @@ attend_partial_kernel(const __grid_constant__ DecodeArgs a) {
 // Merge of the splits for one (batch, query head) per block, D threads.  With quantized values the merged vector
 // is still in the rotated domain and is mapped back once: out = s .* H(o).  EXACT: the splits' maxima are integers
 // (a log2 domain of integers), and every rescale is the exact power of two 2^(m_s - M).
+// The maximum over the splits and the weight of each split are computed once, in parallel across the block (the
+// weights into shared memory, a chunk at a time), so that thread j's sum over the splits of coordinate j is a run of
+// independent loads rather than a chain through m and l.
 template <int D, bool VQ, bool EXACT = false>
 __global__ void __launch_bounds__(D) attend_reduce_kernel(const __grid_constant__ DecodeArgs a) {
+  constexpr int CH = 512;  // splits per chunk of weights
   __shared__ float vec[D];
-  const int bh = blockIdx.x, j = threadIdx.x;
+  __shared__ float wsh[CH];
+  __shared__ float red[D / kWarp];
+  const int bh = blockIdx.x, j = threadIdx.x, lane = j & (kWarp - 1), warp = j / kWarp;
   // launched as a programmatic dependent of the decode kernel: its partials are complete and visible after this
   asm volatile("griddepcontrol.wait;\n" ::: "memory");
-  const float* m = a.ws_m + static_cast<size_t>(bh) * a.splits;
-  const float* l = a.ws_l + static_cast<size_t>(bh) * a.splits;
-  const float* o = a.ws_o + static_cast<size_t>(bh) * a.splits * D;
+  const int S = a.splits;
+  const float* m = a.ws_m + static_cast<size_t>(bh) * S;
+  const float* l = a.ws_l + static_cast<size_t>(bh) * S;
+  const float* o = a.ws_o + static_cast<size_t>(bh) * S * D;
   float M = -INFINITY;
-  for (int s = 0; s < a.splits; ++s) M = fmaxf(M, m[s]);
+  for (int s = j; s < S; s += D) M = fmaxf(M, m[s]);
+  M = warp_max(M);
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = red[0];
+#pragma unroll
+  for (int w = 1; w < D / kWarp; ++w) M = fmaxf(M, red[w]);
+  __syncthreads();  // every thread has read red before it is reused for the sum
   float Ls = 0.f, acc = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < a.splits; ++s) {
-      const float w = (m[s] == -INFINITY) ? 0.f
-                      : EXACT             ? ldexpf(1.f, static_cast<int>(m[s] - M))
-                                          : exp2f(m[s] - M);
-      Ls = fmaf(w, l[s], Ls);
-      acc = fmaf(w, o[static_cast<size_t>(s) * D + j], acc);
+  if (M != -INFINITY) {  // uniform over the block
+    for (int c0 = 0; c0 < S; c0 += CH) {
+      const int n = min(CH, S - c0);
+      for (int s = j; s < n; s += D) {
+        const float ms = m[c0 + s];
+        const float w = (ms == -INFINITY) ? 0.f
+                        : EXACT           ? ldexpf(1.f, static_cast<int>(ms - M))
+                                          : exp2f(ms - M);
+        wsh[s] = w;
+        Ls = fmaf(w, l[c0 + s], Ls);
+      }
+      __syncthreads();
+      const float* oc = o + static_cast<size_t>(c0) * D + j;
+      int s = 0;
+      for (; s + 4 <= n; s += 4) {
+        const float o0 = oc[static_cast<size_t>(s) * D], o1 = oc[static_cast<size_t>(s + 1) * D];
+        const float o2 = oc[static_cast<size_t>(s + 2) * D], o3 = oc[static_cast<size_t>(s + 3) * D];
+        acc = fmaf(wsh[s], o0, acc);
+        acc = fmaf(wsh[s + 1], o1, acc);
+        acc = fmaf(wsh[s + 2], o2, acc);
+        acc = fmaf(wsh[s + 3], o3, acc);
+      }
+      for (; s < n; ++s) acc = fmaf(wsh[s], oc[static_cast<size_t>(s) * D], acc);
+      __syncthreads();  // the chunk's weights are read before the next chunk writes them
     }
   }
+  Ls = warp_sum(Ls);
+  if (lane == 0) red[warp] = Ls;
+  __syncthreads();
+  Ls = red[0];
+#pragma unroll
+  for (int w = 1; w < D / kWarp; ++w) Ls += red[w];
   const float r = Ls > 0.f ? acc / Ls : 0.f;
   if constexpr (!VQ) {
     a.out[static_cast<size_t>(bh) * D + j] = r;
