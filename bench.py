@@ -110,8 +110,11 @@ def _bytes_per_key_head(w):
 
 
 class ClockSampler:
-    """SM clock, power and throttle reasons sampled every 200 ms (nvidia-smi single-shot queries from a thread)
-    while the timed region runs."""
+    """SM clock, power and throttle reasons sampled every 200 ms while the timed region runs: read-only NVML queries
+    from a thread (no process is forked while calls are timed: a fork of a large process stalls its threads, and a
+    stalled launch would leave the GPU idle inside a step's events).  Without NVML bindings, one nvidia-smi process
+    in its looping mode, started before the region and stopped after it.  Samples are kept in nvidia-smi's CSV form
+    (the fields of FIELDS)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -123,14 +126,23 @@ class ClockSampler:
         self.lines = []
         self._stop = None
         self._thread = None
+        self._proc = None
 
-    def _poll(self):
+    def _nvml_line(self, nv, h):
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        act = lambda bit: "Active" if r & bit else "Not Active"
+        return (f"{self.index}, {sm}, {mx}, {pw:.2f}, {r:#x}, {act(nv.nvmlClocksThrottleReasonHwSlowdown)}, "
+                f"{act(nv.nvmlClocksThrottleReasonHwThermalSlowdown)}, "
+                f"{act(nv.nvmlClocksThrottleReasonSwThermalSlowdown)}, {act(nv.nvmlClocksThrottleReasonSwPowerCap)}")
+
+    def _poll(self, nv, h):
         while True:  # one sample at entry, then every period, and one more when stopped
             try:
-                out = subprocess.run(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                                      "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
-                self.lines += [ln for ln in out.stdout.splitlines() if ln.strip()]
-            except (OSError, subprocess.SubprocessError):
+                self.lines.append(self._nvml_line(nv, h))
+            except Exception:  # noqa: BLE001 -- a failed query ends the sampling, not the benchmark
                 return
             if self._stop.is_set():
                 return
@@ -138,14 +150,44 @@ class ClockSampler:
 
     def __enter__(self):
         import threading
+        try:
+            import pynvml as nv
+            import torch
+            nv.nvmlInit()
+            try:
+                nidx = torch.cuda._get_nvml_device_index(self.index)
+            except Exception:  # noqa: BLE001
+                nidx = self.index
+            h = nv.nvmlDeviceGetHandleByIndex(nidx)
+            self._nvml_line(nv, h)
+        except Exception:  # noqa: BLE001 -- no NVML bindings: nvidia-smi's looping mode
+            try:
+                self._proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                               "--format=csv,noheader,nounits", "-lms",
+                                               str(int(self.period * 1000))],
+                                              stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                time.sleep(0.3)
+            except OSError:
+                self._proc = None
+            return self
         self._stop = threading.Event()
-        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread = threading.Thread(target=self._poll, args=(nv, h), daemon=True)
         self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        self._stop.set()
-        self._thread.join(timeout=10)
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=10)
+        if self._proc is not None:
+            time.sleep(0.25)
+            self._proc.terminate()
+            try:
+                out, _ = self._proc.communicate(timeout=10)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+                out, _ = self._proc.communicate()
+            self.lines += [ln for ln in (out or "").splitlines() if ln.strip()]
 
     def summary(self):
         sm, mx, reasons = [], [], set()
@@ -590,11 +632,12 @@ def run_axr(args, w):
                  "frac": dbytes / (ms / 1e3) / 1e9 / _peaks()[0], "algorithmic_bytes": dbytes}
         del kd, vd
 
-    # the same decode step through paged pools (shuffled block tables) at two block sizes
+    # the same decode step through paged pools (shuffled block tables) at three block sizes: blocks of 32 tokens and
+    # more go through the streaming kernel (a tile never spans two blocks), 16-token blocks through the row kernel
     paged = None
     if not args.no_codecs and w.v_quant:
         paged = {}
-        for bt in (16, 256):
+        for bt in (16, 32, 256):
             nb = T // bt
             perm = torch.randperm(B * nb, generator=torch.Generator().manual_seed(bt)).to(dev)
             table = perm.view(B, nb).to(torch.int32).contiguous()
@@ -609,7 +652,8 @@ def run_axr(args, w):
                                                           vnorms=pvn, out=out, workspace=wsp))
             ab = _bytes_per_key_head(w) * B * Hkv * T
             paged[f"bt{bt}"] = {"ms": ms, "achieved_gbs": ab / (ms / 1e3) / 1e9,
-                                "frac": ab / (ms / 1e3) / 1e9 / _peaks()[0], "algorithmic_bytes": ab}
+                                "frac": ab / (ms / 1e3) / 1e9 / _peaks()[0], "algorithmic_bytes": ab,
+                                "kernel": "attend_stream_kernel" if bt >= 32 else "attend_rows_kernel"}
             del pk, pn, pvc, pvn
         paged["contiguous"] = {"ms": float(np.mean(attend_ms))}
 

@@ -8,12 +8,13 @@
 namespace axr {
 namespace {
 
-template <int D, int BITS, int G, bool VQ>
+template <int D, int BITS, int G, bool VQ, bool PAGED = false>
 axr_status launch(const DecodeArgs& a, cudaStream_t st, const char* what) {
   using P = StreamPlan<D, BITS, G, VQ>;
   static_assert(P::WARPS * kSmCount == (VQ ? kAttendStreamWorkersQ : kAttendStreamWorkers) && P::TW == kStreamTile,
                 "the split plan's worker model");
-  auto k = attend_stream_kernel<D, BITS, G, VQ>;
+  static_assert(!PAGED || VQ, "paged pools with quantized values only");
+  auto k = attend_stream_kernel<D, BITS, G, VQ, PAGED>;
   axr_status rs = ensure_smem(k, P::bytes, what);
   if (rs != AXR_OK) return rs;
   const size_t rows = static_cast<size_t>(a.B) * a.Hkv * a.Tcap;  // TMA row coordinates are 32-bit
@@ -31,6 +32,18 @@ axr_status launch(const DecodeArgs& a, cudaStream_t st, const char* what) {
 
 template <int D, int BITS>
 axr_status by_g(int G, bool vq, const DecodeArgs& a, cudaStream_t st, const char* w) {
+  if (a.block_table) {  // paged pools (quantized values, blocks of at least kStreamTile tokens)
+    if (!vq || (1 << a.block_shift) < kStreamTile)
+      return set_error(AXR_EUNSUPPORTED, "%s: the streaming kernel's paged pools take quantized values in blocks of "
+                       "at least %d tokens", w, kStreamTile);
+    switch (G) {
+      case 1: return launch<D, BITS, 1, true, true>(a, st, w);
+      case 2: return launch<D, BITS, 2, true, true>(a, st, w);
+      case 4: return launch<D, BITS, 4, true, true>(a, st, w);
+      case 8: return launch<D, BITS, 8, true, true>(a, st, w);
+    }
+    return set_error(AXR_EUNSUPPORTED, "%s: G=%d", w, G);
+  }
   switch (G) {
     case 1: return vq ? launch<D, BITS, 1, true>(a, st, w) : launch<D, BITS, 1, false>(a, st, w);
     case 2: return vq ? launch<D, BITS, 2, true>(a, st, w) : launch<D, BITS, 2, false>(a, st, w);

@@ -60,8 +60,10 @@ struct StreamPlan {
   static_assert(bytes <= 227 * 1024, "shared memory of one block");
 };
 
-// vmap: the TMA map of the fp16 value cache (fp16 values only).
-template <int D, int BITS, int G, bool VQ>
+// vmap: the TMA map of the fp16 value cache (fp16 values only).  PAGED: the rows of each (batch row, KV head) come
+// through the block table (RowMap); blocks of at least TW tokens, so that a tile (its first token a multiple of TW)
+// never spans two blocks and stays one run of rows.
+template <int D, int BITS, int G, bool VQ, bool PAGED = false>
 __global__ void __launch_bounds__(StreamPlan<D, BITS, G, VQ>::THREADS, 1)
 attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant__ CUtensorMap vmap) {
   using P = StreamPlan<D, BITS, G, VQ>;
@@ -108,7 +110,7 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     const int start = split * a.chunk;
     const int end = min(start + a.chunk, len);
     const int ntiles = end > start ? (end - start + TW - 1) / TW : 0;
-    const size_t row0 = (static_cast<size_t>(b) * a.Hkv + hk) * a.Tcap;
+    const RowMap<PAGED> rm = row_map<PAGED>(a, b, hk);  // cache row of each token (contiguous or paged)
     const float* qg = a.q + (static_cast<size_t>(b) * a.Hq + hk * G) * D;
     // the ring is idle between items: it holds the transformed queries and the write path's index scratch
     float* qs = reinterpret_cast<float*>(ring);
@@ -117,8 +119,8 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     if (a.knew != nullptr && len > 0 && start <= len - 1 && len - 1 < end) {
       // decode step: this item holds the new token (position len - 1): write its key and value through the write
       // path before any of the item's copies is issued
-      append_row<D, BITS, VQ>(a, b, hk, row0 + len - 1, 0, lane, scratch);
-      append_row<D, BITS, VQ>(a, b, hk, row0 + len - 1, 1, lane, scratch);
+      append_row<D, BITS, VQ>(a, b, hk, rm(len - 1), 0, lane, scratch);
+      append_row<D, BITS, VQ>(a, b, hk, rm(len - 1), 1, lane, scratch);
       __threadfence();                                           // the stores reach the device-wide view ...
       asm volatile("fence.proxy.async.global;\n" ::: "memory");  // ... and the async proxy of the copies
     }
@@ -152,20 +154,21 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
         const int s = static_cast<int>((seq + i) % NS);
         uint8_t* st = ring + static_cast<size_t>(s) * P::STAGE;
         const int t0 = start + i * TW;
+        const size_t r0 = rm(t0);  // the tile's first row; its rows are consecutive
         // the tile's code rows, rounded up to whole 16-byte chunks: with rows of 8 or 24 bytes (d = 64, b = 1, 3)
         // an odd row count takes one row more, which lies inside the row's capacity (the launcher requires Tcap
-        // even, and a tile that ends at Tcap has an even row count)
+        // even, and a tile that ends at Tcap has an even row count) or inside the tile's block (paged pools)
         const uint32_t cb = static_cast<uint32_t>((min(TW, end - t0) * R + 15) / 16 * 16);
         if constexpr (VQ) {
           mbar_arrive_expect_tx(mbar + s, 2 * cb);
-          bulk_copy_g2s(st, static_cast<const uint8_t*>(a.v) + (row0 + t0) * R, cb, mbar + s);
+          bulk_copy_g2s(st, static_cast<const uint8_t*>(a.v) + r0 * R, cb, mbar + s);
         } else {
           mbar_arrive_expect_tx(mbar + s, static_cast<uint32_t>(P::VPLANE) + cb);
 #pragma unroll
           for (int bx = 0; bx < P::NBX; ++bx)
-            tma_load_2d(st + bx * P::BOX, &vmap, bx * P::BOXC, static_cast<int>(row0) + t0, mbar + s);
+            tma_load_2d(st + bx * P::BOX, &vmap, bx * P::BOXC, static_cast<int>(r0), mbar + s);
         }
-        bulk_copy_g2s(st + P::VPLANE, a.kcodes + (row0 + t0) * R, cb, mbar + s);
+        bulk_copy_g2s(st + P::VPLANE, a.kcodes + r0 * R, cb, mbar + s);
       }
     };
     for (int i = 0; i < NS && i < ntiles; ++i) issue(i);
@@ -192,6 +195,7 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
     // loads, since a decode step writes one of them in this launch
     auto load_norms = [&](int i, uint32_t (&nr)[2][2]) {
       const int t0 = start + i * TW;
+      const size_t r0 = i < ntiles ? rm(t0) : 0;
 #pragma unroll
       for (int m = 0; m < 2; ++m)
 #pragma unroll
@@ -199,8 +203,9 @@ attend_stream_kernel(const __grid_constant__ DecodeArgs a, const __grid_constant
           const int tok = t0 + 16 * m + g + 8 * e;
           uint32_t r = 0u;  // norms 0 past the end (fp16 +0)
           if (i < ntiles && tok < end) {
-            r = __half_as_ushort(__ldcg(a.knorms + row0 + tok));
-            if constexpr (VQ) r |= static_cast<uint32_t>(__half_as_ushort(__ldcg(a.vnorms + row0 + tok))) << 16;
+            const size_t row = r0 + static_cast<size_t>(tok - t0);
+            r = __half_as_ushort(__ldcg(a.knorms + row));
+            if constexpr (VQ) r |= static_cast<uint32_t>(__half_as_ushort(__ldcg(a.vnorms + row))) << 16;
           }
           nr[m][e] = r;
         }

@@ -134,7 +134,10 @@ axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, con
   // long-context step: 107 against 122 us the other way)
   const bool stream_vq = vkind == AXR_V_QUANT &&
                          (Hq / Hkv == 8 || static_cast<long>(B) * Hkv * T >= (1L << 18));
-  const bool stream_path = (vkind == AXR_V_F16 || stream_vq) && !paged && attend_stream_supported(d, bits, Tcap) &&
+  // paged pools too, with quantized values in blocks of at least one streaming tile (a tile never spans two blocks)
+  const bool stream_path = (vkind == AXR_V_F16 || stream_vq) &&
+                           (!paged || (stream_vq && block_tokens >= kStreamTile)) &&
+                           attend_stream_supported(d, bits, Tcap) &&
                            (step || mode == kGatherMma || mode == kGatherDirect);
   if (stream_path) {
     const SplitPlan p =
@@ -148,10 +151,10 @@ axr_status attend_impl(const char* w, const float* q, const uint8_t* kcodes, con
   a.knew = reinterpret_cast<const __half*>(knew); a.vnew = reinterpret_cast<const __half*>(vnew);
   const int G = Hq / Hkv;
   const bool vq = vkind == AXR_V_QUANT;
-  if (stream_path) return attend_stream_launch(d, bits, G, vq, a, as_stream(stream), w);
   if (paged) {
     a.block_table = block_table; a.max_blocks = max_blocks; a.block_shift = shift;
   }
+  if (stream_path) return attend_stream_launch(d, bits, G, vq, a, as_stream(stream), w);
   // decode step and paged pools: the kernel that writes the new token in its prologue and reads rows through the
   // block table (scores through warp-level MMAs)
   if (step || paged) return attend_rows_launch(d, bits, G, vq, a, as_stream(stream));

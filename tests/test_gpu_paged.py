@@ -146,3 +146,77 @@ def test_paged_argument_errors():
     kn2 = torch.zeros((8, Hkv, 48), dtype=torch.float16, device="cuda")
     with pytest.raises(Exception, match="power of two"):
         ops.attend_decode_paged(q, kc2, kn2, s, bits, table, vcodes=kc2, vnorms=kn2)
+
+
+# Pools the streaming kernel takes: quantized values, at least 2^18 (token, KV head) units or eight query heads per
+# KV head, and blocks of at least its 32-token tile.  (d, bits, G, B, Hkv, T, bt)
+STREAM_CASES = [(128, 4, 4, 4, 8, 8192, 32), (128, 4, 4, 4, 8, 8192, 256), (64, 3, 8, 2, 2, 1000, 64)]
+
+
+@pytest.mark.parametrize("d,bits,G,B,Hkv,T,bt", STREAM_CASES)
+def test_paged_streaming_kernel(d, bits, G, B, Hkv, T, bt):
+    """Paged pools through the streaming kernel: attend and decode step give the contiguous cache's results bit for
+    bit (the same kernel arithmetic, split plan and rows, only addressed through a shuffled block table), the step
+    writes its token through the table, and sampled heads match the oracle on the host inputs."""
+    Hq = Hkv * G
+    shape = (B, Hkv, T, d)
+    k = W.lognormal_rows(shape, 70 + bt + d, dtype=np.float16)
+    v = W.lognormal_rows(shape, 71 + bt + d, dtype=np.float16)
+    s = W.sign_vector(d, 72)
+    q = W.normal((B, Hq, d), 73, np.float32)
+    lens = np.array([T, T // 2 + 1, 33, T - 7][:B], np.int32)
+    st, tq, tl = cuda(s), cuda(q), cuda(lens)
+    kc, kn = ops.write_keys(cuda(k), st, bits)
+    vc, vn = ops.write_keys(cuda(v), st, bits)
+    mb = -(-T // bt)
+    nblocks = B * mb + 5
+    rng = np.random.default_rng(bt + d)
+    table = cuda(rng.permutation(nblocks)[:B * mb].reshape(B, mb).astype(np.int32))
+
+    def pool(x, noise):
+        """x [B, Hkv, T, ...] scattered into a pool [nblocks, Hkv, bt, ...] through the table; spare blocks hold
+        noise."""
+        pad = torch.zeros((B, Hkv, mb * bt) + tuple(x.shape[3:]), dtype=x.dtype, device="cuda")
+        pad[:, :, :T] = x
+        p = noise((nblocks, Hkv, bt) + tuple(x.shape[3:]))
+        blocks = pad.reshape((B, Hkv, mb, bt) + tuple(x.shape[3:])).transpose(1, 2)
+        p[table.long().reshape(-1)] = blocks.reshape((B * mb, Hkv, bt) + tuple(x.shape[3:]))
+        return p
+
+    codes_noise = lambda shp: torch.randint(0, 256, shp, dtype=torch.uint8, device="cuda")
+    norms_noise = lambda shp: (torch.rand(shp, device="cuda") * 4).half()
+    kcp, knp = pool(kc, codes_noise), pool(kn, norms_noise)
+    vcp, vnp = pool(vc, codes_noise), pool(vn, norms_noise)
+
+    out_c = ops.attend_decode(tq, kc, kn, st, bits, vcodes=vc, vnorms=vn, seq_lens=tl, T=T)
+    out_p = ops.attend_decode_paged(tq, kcp, knp, st, bits, table, seq_lens=tl, T=T, vcodes=vcp, vnorms=vnp)
+    assert torch.equal(out_p, out_c)
+
+    # the decode step over stale rows at each row's last position, in both layouts
+    pos = lens - 1
+    knew = cuda(np.stack([k[b, :, pos[b]] for b in range(B)]))
+    vnew = cuda(np.stack([v[b, :, pos[b]] for b in range(B)]))
+    kc_s, kn_s, vc_s, vn_s = kc.clone(), kn.clone(), vc.clone(), vn.clone()
+    kcp_s, knp_s, vcp_s, vnp_s = kcp.clone(), knp.clone(), vcp.clone(), vnp.clone()
+    tab = table.cpu().numpy()
+    for b in range(B):
+        p, o = tab[b, pos[b] // bt], pos[b] % bt
+        kc_s[b, :, pos[b]] = 0x5a; kn_s[b, :, pos[b]] = 3.0; vc_s[b, :, pos[b]] = 0xa5; vn_s[b, :, pos[b]] = 2.0
+        kcp_s[p, :, o] = 0x5a; knp_s[p, :, o] = 3.0; vcp_s[p, :, o] = 0xa5; vnp_s[p, :, o] = 2.0
+    step_c = ops.decode_step(tq, knew, vnew, kc_s, kn_s, st, bits, vcodes=vc_s, vnorms=vn_s, seq_lens=tl, T=T)
+    step_p = ops.decode_step_paged(tq, knew, vnew, kcp_s, knp_s, st, bits, table, seq_lens=tl, T=T, vcodes=vcp_s,
+                                   vnorms=vnp_s)
+    assert torch.equal(step_p, step_c)
+    for got, want in ((kcp_s, kcp), (knp_s, knp), (vcp_s, vcp), (vnp_s, vnp)):
+        assert torch.equal(got, want)  # the written rows are the writer's, the rest untouched
+
+    out, got = out_p.cpu().numpy(), step_p.cpu().numpy()
+    scale = 1.0 / math.sqrt(d)
+    for b, h in [(0, 0), (B - 1, Hq - 1), (1, Hq // 2 + 1), (B - 1, 3)]:
+        hk, n = h // G, lens[b]
+        okc, okn = oracle.write(k[b, hk, :n], s, bits)
+        ovc, ovn = oracle.write(v[b, hk, :n], s, bits)
+        want = oracle.decode_attention(q[b:b + 1, h:h + 1], okc[None, None], okn[None, None], s, bits, scale,
+                                       vcodes=ovc[None, None], vn16=ovn[None, None])
+        parity.check_outputs(out[b:b + 1, h:h + 1], want)
+        parity.check_outputs(got[b:b + 1, h:h + 1], want)
