@@ -81,9 +81,9 @@ def _step_kernel(w) -> str:
 
 
 TRAFFIC = {
-    # attend_stream_kernel<128, 4, 4, quantized V>, DRAM read + write per launch at B = 4 (mean of three launches,
-    # profiles/attend_stream_long_context.md), scaled by the units to B = 8
-    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.777003e6 + 1.149867e6),
+    # attend_stream_kernel<128, 4, 4, quantized V> (16 warps per SM), DRAM read + write per launch at B = 4 (mean of
+    # three launches of the counters-only ncu capture kept under profiles/), scaled by the units to B = 8
+    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.652075e6 + 1.630037e6),
 }
 
 WORKLOADS = {
@@ -497,17 +497,20 @@ def run_axr(args, w):
     launches_per_step = 2  # the decode kernel (with the new token's write) + the split merge
 
     stream = torch.cuda.current_stream()
-    for _ in range(args.warmup):
-        step(q, knew, vnew)
-    torch.cuda.synchronize()
-
     # --- timed region: K steps, L2 flushed between steps (outside the per-step events) ---
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    if ws > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
+    # The clock sampler starts first and the W warm-up steps (flushed like the timed ones) run right before the timed
+    # steps, so that no idle gap (the sampler's start-up) separates the two.
     with ClockSampler(local) as clk:
+        for _ in range(args.warmup):
+            flush()
+            _lead_in()
+            step(q, knew, vnew)
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
         for i in range(args.steps):
             flush()
             _lead_in()
@@ -520,6 +523,7 @@ def run_axr(args, w):
         dist.barrier()
     step_ms = sum(e0.elapsed_time(e2) for e0, _, e2 in ev)
     attend_ms = [e0.elapsed_time(e2) for e0, _, e2 in ev]  # the whole step is one decode call
+    step_stats = {"min": min(attend_ms), "median": float(np.median(attend_ms)), "max": max(attend_ms)}
     clocks = clk.summary()
 
     # --- end to end through the public API: pinned host inputs in, result out, every step ---
@@ -681,7 +685,7 @@ def run_axr(args, w):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": step_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": DTYPE, "data": "synthetic",
+        "dtype": DTYPE, "data": "synthetic", "step_ms_rank0": step_stats,
         "config": {"workload": w.name, "B": B, "T": T, "Hq": Hq, "Hkv": Hkv, "d": d, "bits": bits,
                    "values": "quantized b=%d" % bits if w.v_quant else "fp16", "parallelism": f"replicas x{ws}",
                    "l2": "flushed between steps outside the per-step events: a 256 MiB write, then a 256 MiB read of "

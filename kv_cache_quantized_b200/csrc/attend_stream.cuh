@@ -35,7 +35,7 @@ template <int D, int BITS, int G, bool VQ>
 struct StreamPlan {
   static constexpr int TW = 32;                          // tokens per warp tile
   static constexpr int NS = 2;                           // stages per warp
-  static constexpr int WARPS = VQ ? 12 : 8;              // warps per block (one block per SM)
+  static constexpr int WARPS = VQ ? 16 : 8;              // warps per block (one block per SM)
   static constexpr int THREADS = 32 * WARPS;
   static constexpr int R = D * BITS / 8;                 // bytes of a key code row
   static constexpr int BOXC = 64;                        // value coordinates per TMA box

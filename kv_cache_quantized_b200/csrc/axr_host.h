@@ -70,7 +70,7 @@ inline SplitPlan plan_splits(int B, int Hkv, int T, long resident = kResident, i
 constexpr int kStreamTile = 32;
 constexpr int kDenseWorkers = 4 * kSmCount;
 constexpr int kAttendStreamWorkers = 8 * kSmCount;   // fp16 values
-constexpr int kAttendStreamWorkersQ = 12 * kSmCount; // quantized values
+constexpr int kAttendStreamWorkersQ = 16 * kSmCount; // quantized values
 inline SplitPlan plan_splits_stream(int B, int Hkv, int T, int workers) {
   return plan_splits(B, Hkv, T, workers, kStreamTile, 2, 2.0);
 }
