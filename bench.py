@@ -83,7 +83,7 @@ def _step_kernel(w) -> str:
 TRAFFIC = {
     # attend_stream_kernel<128, 4, 4, quantized V> (16 warps per SM), DRAM read + write per launch at B = 4 (mean of
     # three launches of the counters-only ncu capture kept under profiles/), scaled by the units to B = 8
-    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.652075e6 + 1.630037e6),
+    "long_context_b8_t32768_hq32_hkv8_d128_b4_kvquant": 2 * (138.575189e6 + 1.367979e6),
 }
 
 WORKLOADS = {

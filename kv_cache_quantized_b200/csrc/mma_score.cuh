@@ -282,4 +282,59 @@ __device__ __forceinline__ void mma_scores16(const uint8_t* st, int row0, const 
   }
 }
 
+// mma_scores16 for the two 16-token groups of a 32-token tile (rows row0 .. row0 + 15 into out[0], row0 + 16 ..
+// row0 + 31 into out[1]) in one pass over K: the four accumulator chains (two groups x tokens g, g + 8) take turns,
+// so that each MMA's successor in its chain issues three MMAs later.  Each chain sums its products in the order
+// mma_scores16 does, so the scores are the same bit for bit.
+template <int D, int BITS, int G, bool SWZ = true, bool KV = false>
+__device__ __forceinline__ void mma_scores16x2(const uint8_t* st, int row0, const uint8_t* tab, uint32_t rep16,
+                                               const MmaB<D, G>& B, int lane,
+                                               float (&out)[2][MmaB<D, G>::NT][2]) {
+  constexpr int R = D * BITS / 8, KT = MmaB<D, G>::KT, NT = MmaB<D, G>::NT;
+  constexpr int NB = R / 4;
+  constexpr int NW = (NB + 3) / 4 + 1;
+  const int gq = lane >> 2, tq = lane & 3;
+  uint32_t w[4][NW];  // tokens g, g + 8 of group 0, then of group 1
+#pragma unroll
+  for (int x = 0; x < 4; ++x) {
+    load_run<R, NB, SWZ>(st, (row0 + 16 * (x >> 1) + gq + 8 * (x & 1)) * R + tq * NB, w[x]);
+#pragma unroll
+    for (int i = (NB + 3) / 4; i < NW; ++i) w[x][i] = 0u;
+  }
+  float c[4][NT][4];
+#pragma unroll
+  for (int x = 0; x < 4; ++x)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c[x][nt][i] = 0.f;
+  auto off = [&](const uint32_t* wr, int i) {
+    if constexpr (KV) return kv_off<BITS>(wr, i, rep16);
+    else return hilo_off16<BITS>(wr, i, rep16);
+  };
+#pragma unroll
+  for (int kk = 0; kk < KT; ++kk) {
+    uint2 e[4][2];
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      e[x][0] = *reinterpret_cast<const uint2*>(tab + off(w[x], 2 * kk));
+      e[x][1] = *reinterpret_cast<const uint2*>(tab + off(w[x], 2 * kk + 1));
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+        mma_m16n8k16(c[x][nt], e[x][0].x, e[x][0].y, e[x][1].x, e[x][1].y, B.bh[nt][kk][0], B.bh[nt][kk][1]);
+  }
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const float* cc = c[2 * m + i][nt];
+        out[m][nt][i] = (cc[0] + cc[1]) + (cc[2] + cc[3]);
+      }
+}
+
 }  // namespace axr
