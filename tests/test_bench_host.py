@@ -58,3 +58,42 @@ def test_step_kernel_label_follows_the_library_routing():
     assert bench._step_kernel(W.LLAMA8B_DECODE) == "attend_stream_kernel"
     assert bench._step_kernel(dataclasses.replace(W.LONG_CONTEXT, B=1, T=4096)) == "attend_rows_kernel"
     assert bench._step_kernel(dataclasses.replace(W.LONG_CONTEXT, B=1, T=4096, Hq=64)) == "attend_stream_kernel"
+
+
+class _FakeNvml:
+    """The NVML calls the clock sampler makes, answering fixed readings (no GPU, no driver)."""
+    NVML_CLOCK_SM = 1
+    nvmlClocksThrottleReasonSwPowerCap = 0x4
+    nvmlClocksThrottleReasonHwSlowdown = 0x8
+    nvmlClocksThrottleReasonSwThermalSlowdown = 0x20
+    nvmlClocksThrottleReasonHwThermalSlowdown = 0x40
+
+    def __init__(self, sm, reasons):
+        self.sm, self.reasons = sm, reasons
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        return self.sm
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 812_500  # mW
+
+    def nvmlDeviceGetCurrentClocksThrottleReasons(self, h):
+        return self.reasons
+
+
+def test_clock_sampler_reads_nvml_samples_into_the_summary():
+    """NVML readings become nvidia-smi-style CSV samples: the summary takes the median SM clock, the maximum and the
+    throttle reasons seen (sw_power_cap is reported, an idle reason is not)."""
+    c = bench.ClockSampler(0)
+    c.lines.append(c._nvml_line(_FakeNvml(1965, 0x0), None))
+    c.lines.append(c._nvml_line(_FakeNvml(1890, 0x4), None))
+    c.lines.append(c._nvml_line(_FakeNvml(1950, 0x1), None))
+    assert c.lines[0].split(", ")[1:4] == ["1965", "1965", "812.50"]
+    s = c.summary()
+    assert s == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    c2 = bench.ClockSampler(0)
+    c2.lines.append(c2._nvml_line(_FakeNvml(1200, 0x8 | 0x40), None))
+    assert c2.summary()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
