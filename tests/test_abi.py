@@ -218,3 +218,29 @@ def test_codec_argument_errors_host(L):
     assert L.axr_pot_score(FAKE, FAKE + 8, FAKE, None, 2, 8, 2, 100, 100, 128, 3, 0, 0.1, FAKE, None, None) == 1
     assert L.axr_pot_attend_decode(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 2, 100, 100, 128, 2, 1, 0.1, FAKE, FAKE, 16,
                                    None) == 4
+
+
+def _plan(B, Hkv, T, workers, tile, min_tiles, setup):
+    """The split rule, restated: the split count minimising ceil(items / workers) x (tiles per split + setup), chunks
+    of whole tiles, at least min_tiles long; the first minimum wins."""
+    units, tt = B * Hkv, -(-T // tile)
+    best, plan = None, (1, tile)
+    for s in range(1, max(1, min(tt // min_tiles, 4096)) + 1):
+        tiles = -(-tt // s)
+        splits = -(-tt // tiles)
+        cost = -(-(units * splits) // workers) * (tiles + setup)
+        if best is None or cost < best - 1e-9:
+            best, plan = cost, (splits, tiles * tile)
+    return plan
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,T,d", [(8, 32, 8, 32768, 128), (1, 32, 8, 4096, 128), (64, 32, 8, 131072, 64),
+                                         (3, 16, 4, 3000, 128), (8, 32, 8, 8192, 128)])
+def test_attend_workspace_holds_every_kernels_split_plan(L, B, Hq, Hkv, T, d):
+    """The workspace query covers the largest split plan of the kernels that may run: the row kernel (296 workers,
+    128-token tiles) and the streaming kernels (one worker per warp: 592 dense, 1184 fp16 values, 2368 quantized
+    values; 32-token tiles); the long-context step's plan is 37 splits of 896 tokens."""
+    s = max([_plan(B, Hkv, T, 296, 128, 4, 0.5)[0]] + [_plan(B, Hkv, T, w, 32, 2, 2.0)[0] for w in (592, 1184, 2368)])
+    parts = B * Hq * s
+    assert L.axr_attend_workspace_bytes(B, Hq, Hkv, T, d) == -(-(parts * d * 4 + 2 * parts * 4) // 256) * 256
+    assert _plan(8, 8, 32768, 2368, 32, 2, 2.0) == (37, 896)
