@@ -573,11 +573,17 @@ def run_axr(args, w):
         variants["rows_decode_step"] = {"ms": float(np.mean(attend_ms)),
                             "achieved_gbs": ab / (float(np.mean(attend_ms)) / 1e3) / 1e9, "algorithmic_bytes": ab}
 
-    # the scorer alone (axr_score) on the same cache, every table read mode, L2 flushed before each call
+    # the scorer alone (axr_score) on the same cache, L2 flushed before each call: the default read (the factored
+    # table on mma.sync) and the literal table as its ablation; with --variants also the other read modes (codes
+    # loaded straight into registers, the tcgen05 tensor cores, the CUDA cores)
     scorer = {}
+    roles = {"mma": "default read: factored table on mma.sync", "table": "ablation: the literal table in shared memory",
+             "direct": "variant: codes straight into registers", "tensor": "variant: tcgen05 with TMEM operands",
+             "factored": "variant: factored table on the CUDA cores"}
     if not args.no_scorer:
         sc_out = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
-        for mode in ("mma", "direct", "tensor", "factored", "table"):
+        modes = ("mma", "table") + (("direct", "tensor", "factored") if args.variants else ())
+        for mode in modes:
             ops.set_gather(mode)
             for _ in range(3):
                 ops.score(q, kc, kn, signs, bits, scale=1.0 / math.sqrt(d), out=sc_out)
@@ -595,7 +601,7 @@ def run_axr(args, w):
             cbytes = (R + 2) * B * Hkv * T             # codes + norms only
             scorer[mode] = {"ms": ms, "achieved_gbs": sbytes / (ms / 1e3) / 1e9, "algorithmic_bytes": sbytes,
                             "achieved_gbs_codes_norms": cbytes / (ms / 1e3) / 1e9,
-                            "algorithmic_bytes_codes_norms": cbytes}
+                            "algorithmic_bytes_codes_norms": cbytes, "role": roles[mode]}
         ops.set_gather("mma")
         # the literal table where byte-indexed multi-coordinate tables apply (b <= 2: 8 or 4 coordinates per
         # 8-bit field), against the factored MMA read of the same codes, at this shape
@@ -861,7 +867,8 @@ def main(argv=None):
                     help="override the workload's batch size, or the selector's layer count (small ncu cases)")
     ap.add_argument("--no-scorer", action="store_true", help="skip the separate axr_score measurement")
     ap.add_argument("--variants", action="store_true",
-                    help="also time the attend over the tiled value layout (MMA and tcgen05 value products)")
+                    help="also time the attend over the tiled value layout (MMA and tcgen05 value products) and the "
+                         "scorer's other read modes (direct register loads, tcgen05, CUDA cores)")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense fp16 bandwidth reference")
     ap.add_argument("--no-codecs", action="store_true", help="skip the LOOKAT / PoT / literal-table measurements")
     ap.add_argument("--sweep", action="store_true",
