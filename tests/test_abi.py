@@ -244,3 +244,43 @@ def test_attend_workspace_holds_every_kernels_split_plan(L, B, Hq, Hkv, T, d):
     parts = B * Hq * s
     assert L.axr_attend_workspace_bytes(B, Hq, Hkv, T, d) == -(-(parts * d * 4 + 2 * parts * 4) // 256) * 256
     assert _plan(8, 8, 32768, 2368, 32, 2, 2.0) == (37, 896)
+
+
+def _prototypes():
+    """name -> list of parameter declarations, from the AXR_API prototypes of include/*.h."""
+    out = {}
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = re.sub(r"/\*.*?\*/", " ", open(os.path.join(ROOT, "include", f)).read(), flags=re.S)
+            for m in re.finditer(r"AXR_API\s+([\w\s\*]+?)\b(axr_\w+)\s*\(([^)]*)\)", txt):
+                params = [p.strip() for p in m.group(3).split(",")]
+                out[m.group(2)] = (m.group(1).strip(), [] if params in ([""], ["void"]) else params)
+    return out
+
+
+def _ctype_of(decl):
+    if "*" in decl:
+        return "ptr"
+    base = decl.rsplit(None, 1)[0].replace("const", "").strip()
+    return {"int": ctypes.c_int, "float": ctypes.c_float, "size_t": ctypes.c_size_t, "int64_t": ctypes.c_int64,
+            "axr_vkind": ctypes.c_int, "axr_gather": ctypes.c_int, "axr_dtype": ctypes.c_int,
+            "uint32_t": ctypes.c_uint32}.get(base, base)
+
+
+def test_binding_signatures_match_the_header():
+    """Every ctypes signature of the binding has the header's return type and parameter count, and each parameter the
+    header's kind: a pointer where the header has one, the matching integer or float type elsewhere."""
+    protos = _prototypes()
+    assert set(protos) == set(_abi.SIGNATURES)
+    for name, (ret, params) in protos.items():
+        res, args = _abi.SIGNATURES[name]
+        want_res = {"axr_status": ctypes.c_int, "int": ctypes.c_int, "axr_gather": ctypes.c_int,
+                    "size_t": ctypes.c_size_t, "const char*": ctypes.c_char_p}[ret.replace(" *", "*")]
+        assert res is want_res, f"{name}: returns {ret}, bound as {res}"
+        assert len(args) == len(params), f"{name}: {len(args)} ctypes arguments, {len(params)} in the header"
+        for decl, ct in zip(params, args):
+            want = _ctype_of(decl)
+            if want == "ptr":
+                assert ct in (ctypes.c_void_p, ctypes.c_char_p), f"{name}: {decl!r} bound as {ct}"
+            else:
+                assert ct is want or ct == want, f"{name}: {decl!r} bound as {ct}, header wants {want}"
